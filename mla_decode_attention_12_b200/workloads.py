@@ -1,0 +1,228 @@
+"""Seeded synthetic inputs for MLA decoding: the five decode workloads and generic problems.
+
+This module draws random numbers and lays them out; it holds none of the
+attention arithmetic, so both the CUDA path and the FP64 oracle can take their
+inputs from it.  All arrays are numpy; 16-bit floats are returned as their raw
+bit patterns (``uint16``) so that both sides see identical bytes.
+
+Layouts (the ones the library's C ABI takes):
+
+* ``q``            ``[batch, s_q, h_q, d_qk]`` 16-bit, row-major.
+* ``kvcache``      ``[num_blocks, page_size, h_kv, d_qk]`` 16-bit; a token row is the
+                   latent part (first 512 columns, also V) then the RoPE part.
+* ``block_table``  ``[batch, max_blocks_per_seq]`` int32 physical page ids, a seeded
+                   Fisher-Yates permutation of the pages; unused slots are -1.
+* ``cache_seqlens`` ``[batch]`` int32.
+
+The workloads follow the decode configurations the pages benchmark (paged
+cache with 64-token pages, MQA mode d_qk = 576 / d_v = 512, variable sequence
+lengths; "FlashMLA" usage page and the upstream FlashMLA documentation,
+"Performance" and "Usage / MLA Decoding").
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+PAGE = 64
+BF16 = 0
+FP16 = 1
+
+
+@dataclasses.dataclass
+class Problem:
+    """One decode call's inputs (host arrays) plus its shape parameters."""
+
+    name: str
+    q: np.ndarray            # uint16 [b, s_q, h_q, d_qk]
+    kvcache: np.ndarray      # uint16 [num_blocks, page, h_kv, d_qk]
+    block_table: np.ndarray  # int32 [b, max_blocks]
+    cache_seqlens: np.ndarray  # int32 [b]
+    dtype: int               # 0 = bfloat16, 1 = float16
+    causal: bool
+    scale: float
+    dv: int = 512
+    page_size: int = PAGE
+    active_heads: int | None = None  # heads >= this are zero-filled (padded heads)
+    seed: int = 0
+
+    @property
+    def batch(self) -> int:
+        return self.q.shape[0]
+
+    @property
+    def s_q(self) -> int:
+        return self.q.shape[1]
+
+    @property
+    def h_q(self) -> int:
+        return self.q.shape[2]
+
+    @property
+    def d_qk(self) -> int:
+        return self.q.shape[3]
+
+    @property
+    def h_kv(self) -> int:
+        return self.kvcache.shape[2]
+
+    @property
+    def num_blocks(self) -> int:
+        return self.kvcache.shape[0]
+
+    def visible(self) -> np.ndarray:
+        """[b, s_q] number of cached tokens each query token attends (causal: bottom-right)."""
+        L = self.cache_seqlens.astype(np.int64)[:, None]
+        if not self.causal:
+            return np.broadcast_to(L, (self.batch, self.s_q)).copy()
+        s = np.arange(self.s_q, dtype=np.int64)[None, :]
+        return np.clip(L - self.s_q + 1 + s, 0, L)
+
+    def flops(self) -> float:
+        """2 * (d_qk + d_v) per visible (query row, key) pair, all heads."""
+        return 2.0 * (self.d_qk + self.dv) * float(self.visible().sum()) * self.h_q
+
+    def kv_bytes(self) -> int:
+        """Cached rows read once: sum_b L_b * h_kv * d_qk * 2 bytes."""
+        return int(self.cache_seqlens.astype(np.int64).sum()) * self.h_kv * self.d_qk * 2
+
+    def io_bytes(self) -> int:
+        """Algorithmic bytes: KV once + Q + O (16-bit) + LSE (fp32)."""
+        rows = self.batch * self.s_q * self.h_q
+        return self.kv_bytes() + rows * (self.d_qk * 2 + self.dv * 2 + 4)
+
+
+def _round_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> bfloat16 bit patterns, round to nearest even."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    rounded = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
+    return rounded.astype(np.uint16)
+
+
+def to_bits(x: np.ndarray, dtype: int) -> np.ndarray:
+    """float32 -> 16-bit bit patterns (bfloat16 RNE or IEEE float16 RNE)."""
+    if dtype == BF16:
+        return _round_bf16_bits(x)
+    return np.ascontiguousarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
+def _normal_bits(rng: np.random.Generator, shape, std: float, dtype: int) -> np.ndarray:
+    out = np.empty(shape, np.uint16)
+    flat = out.reshape(-1)
+    chunk = 1 << 24
+    for i in range(0, flat.size, chunk):
+        n = min(chunk, flat.size - i)
+        x = rng.standard_normal(n, dtype=np.float32)
+        if std != 1.0:
+            x *= np.float32(std)
+        flat[i:i + n] = to_bits(x, dtype)
+    return out
+
+
+def make_problem(
+    seqlens,
+    *,
+    s_q: int = 1,
+    h_q: int = 16,
+    d_qk: int = 576,
+    h_kv: int = 1,
+    dtype: int = BF16,
+    causal: bool = False,
+    std: float = 1.0,
+    scale: float | None = None,
+    seed: int = 0,
+    active_heads: int | None = None,
+    poison: bool = False,
+    extra_pages: int = 0,
+    extra_table_cols: int = 0,
+    name: str = "problem",
+) -> Problem:
+    """Seeded problem with the given sequence lengths.
+
+    ``poison`` fills what a correct kernel must never use with NaN: the tail
+    rows of each sequence's last page and every page no sequence owns
+    (``extra_pages`` of them).  Unused block-table slots are always -1.
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+    seqlens = np.asarray(seqlens, dtype=np.int32)
+    b = seqlens.size
+    nblk = [(int(L) + PAGE - 1) // PAGE for L in seqlens]
+    used = int(sum(nblk))
+    num_blocks = max(1, used + extra_pages)
+    max_blocks = max(1, max(nblk) if nblk else 1) + extra_table_cols
+
+    q = _normal_bits(rng, (b, s_q, h_q, d_qk), std, dtype)
+    if active_heads is not None and active_heads < h_q:
+        q[:, :, active_heads:, :] = 0
+    kv = _normal_bits(rng, (num_blocks, PAGE, h_kv, d_qk), std, dtype)
+
+    perm = rng.permutation(num_blocks).astype(np.int32)
+    table = np.full((b, max_blocks), -1, np.int32)
+    pos = 0
+    for i, n in enumerate(nblk):
+        table[i, :n] = perm[pos:pos + n]
+        pos += n
+
+    if poison:
+        nan_bits = np.uint16(0x7FC0) if dtype == BF16 else np.uint16(0x7E00)
+        for i, L in enumerate(seqlens):
+            n = nblk[i]
+            if n and int(L) % PAGE:
+                kv[table[i, n - 1], int(L) % PAGE:, :, :] = nan_bits
+        for p in perm[pos:]:
+            kv[p] = nan_bits
+
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    return Problem(name=name, q=q, kvcache=kv, block_table=table, cache_seqlens=seqlens,
+                   dtype=dtype, causal=causal, scale=float(scale), active_heads=active_heads,
+                   seed=seed)
+
+
+# ----------------------------------------------------------------------------
+# The five decode workloads.  Workload k draws from seed 1000 + k.
+# ----------------------------------------------------------------------------
+
+WORKLOADS = ("tiny", "compute", "spec_padded", "long_split", "fp16_norope")
+
+
+def workload_seqlens(name: str, rng: np.random.Generator) -> np.ndarray:
+    if name == "tiny":
+        return np.array([256, 193], np.int32)
+    if name == "compute":
+        return rng.integers(1024, 8192, size=64, endpoint=True).astype(np.int32)
+    if name == "spec_padded":
+        return rng.integers(4096 - 512, 4096 + 512, size=128, endpoint=True).astype(np.int32)
+    if name == "long_split":
+        return np.array([65536, 49152, 32768, 8192], np.int32)
+    if name == "fp16_norope":
+        u = rng.uniform(math.log(512), math.log(16384), size=32)
+        return np.floor(np.exp(u)).astype(np.int32)
+    raise KeyError(name)
+
+
+def make_workload(name: str, *, poison: bool = False, seqlens=None) -> Problem:
+    """One of the five decode workloads (synthetic data, fixed seed 1000 + index).
+
+    ``seqlens`` overrides the sequence lengths (for scaled-down parity cases with
+    the same head / dtype / mask structure).
+    """
+    k = WORKLOADS.index(name) + 1
+    seed = 1000 + k
+    rng = np.random.Generator(np.random.PCG64(seed + 7919))
+    L = workload_seqlens(name, rng) if seqlens is None else np.asarray(seqlens, np.int32)
+    common = dict(seed=seed, poison=poison, name=name)
+    if name == "tiny":
+        return make_problem(L, s_q=1, h_q=16, d_qk=576, **common)
+    if name == "compute":
+        return make_problem(L, s_q=1, h_q=128, d_qk=576, **common)
+    if name == "spec_padded":
+        return make_problem(L, s_q=2, h_q=64, d_qk=576, causal=True, active_heads=16, **common)
+    if name == "long_split":
+        return make_problem(L, s_q=1, h_q=128, d_qk=576, **common)
+    if name == "fp16_norope":
+        return make_problem(L, s_q=4, h_q=64, d_qk=512, causal=True, dtype=FP16, std=0.5,
+                            **common)
+    raise KeyError(name)

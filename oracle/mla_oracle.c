@@ -1,0 +1,288 @@
+/*
+ * Plain FP64 CPU oracle for MLA decoding over a paged latent KV cache.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+ * this file; only the test-suite, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header, table or helper with the CUDA
+ * path.
+ *
+ * What it computes is the plain definition of the operation, written out with
+ * no blocking, fusion or reordering:
+ *
+ *   For each request b, query token s < s_q and query head h < h_q
+ *   (kv head g = h / (h_q / h_kv)):
+ *     n      = causal ? clamp(L_b - s_q + 1 + s, 0, L_b) : L_b
+ *     k_j    = kvcache[block_table[b][j / page]][j % page][g][0 : d_qk]   (j < n)
+ *     v_j    = k_j[0 : dv]        (V is the leading dv columns of the same row)
+ *     x_j    = scale * <q[b,s,h,:], k_j>
+ *     LSE    = log sum_j exp(x_j)         (natural log, computed as M + log sum exp(x_j - M))
+ *     O      = sum_j exp(x_j - LSE) v_j
+ *   and for n == 0: O = 0, LSE = -inf.
+ *
+ * Sources (page title, section):
+ *   - "FlashMLA" usage page (deepep.org): get_mla_metadata / flash_mla_with_kvcache
+ *     call, its arguments q, kvcache, block_table, cache_seqlens, dv, causal; the
+ *     kernel's three stages Q-K product, softmax with scaling, output.
+ *   - Upstream FlashMLA documentation, "Usage / MLA Decoding": return values
+ *     (out, lse), lse = log-sum-exp of the attention scores per query head;
+ *     "MLA Mode" footnote: MQA mode is head_dim_k = 576 with head_dim_v = 512.
+ *   - Upstream FlashMLA documentation, FP8 KV cache format: a token row is the
+ *     512-wide NoPE (latent) part followed by the 64-wide RoPE part, so V is the
+ *     leading 512 columns of the row.
+ *   - Upstream FlashMLA documentation, "Sparse MLA Prefill / Equivalent PyTorch
+ *     code": the softmax written out (max, log-sum-exp, weights exp(P - lse)).
+ * Readings where the pages are silent (each is listed in the design notes):
+ *   LSE is the natural log of the scaled logits; causal alignment is bottom-right
+ *   (the last query token sees all L_b tokens); scale is an argument.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ */
+/* 16-bit float decoding, written from the IEEE-754 / bfloat16 layouts. */
+/* ------------------------------------------------------------------ */
+
+/* bfloat16: the upper 16 bits of an IEEE-754 binary32. */
+static double oracle_bf16_to_double(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* IEEE-754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+static double oracle_fp16_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)m, -24); /* subnormal: m * 2^-14 * 2^-10 */
+    } else if (e == 31) {
+        v = (m == 0) ? INFINITY : NAN;
+    } else {
+        v = ldexp((double)(m | 0x400), e - 25); /* (1 + m/1024) * 2^(e-15) */
+    }
+    return sign ? -v : v;
+}
+
+double mla_oracle_half_to_double(uint16_t h, int dtype)
+{
+    return dtype == 0 ? oracle_bf16_to_double(h) : oracle_fp16_to_double(h);
+}
+
+int mla_oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Shape of one problem; plain struct so the ctypes side can fill it. */
+typedef struct {
+    int batch, s_q, h_q, h_kv, d_qk, dv;
+    int page_size, max_blocks_per_seq, num_blocks;
+    int dtype;   /* 0 = bfloat16, 1 = float16 */
+    int causal;  /* bottom-right aligned */
+    double scale;
+} mla_oracle_shape;
+
+/* Number of cached tokens visible to query token s of request b. */
+static long oracle_visible(const mla_oracle_shape* sh, long L, int s)
+{
+    if (!sh->causal) return L;
+    long n = L - sh->s_q + 1 + s;
+    if (n < 0) n = 0;
+    if (n > L) n = L;
+    return n;
+}
+
+/*
+ * Attention of one (b, s, h) over the visible tokens j with lo <= j < hi.
+ * Writes dv outputs and returns the LSE of that token range; an empty range
+ * gives O = 0 and LSE = -inf.  With lo = 0, hi = L_b this is the full result;
+ * other ranges give the partial results that the split / combine invariant
+ * uses.
+ */
+static double oracle_one_row(const mla_oracle_shape* sh, const uint16_t* q,
+                             const uint16_t* kv, const int32_t* block_table,
+                             long L, int b, int s, int h, long lo, long hi,
+                             double* x /* scratch, >= hi-lo */, double* qrow,
+                             double* o_row)
+{
+    const int d_qk = sh->d_qk, dv = sh->dv, P = sh->page_size;
+    const int g = h / (sh->h_q / sh->h_kv);
+    long n = oracle_visible(sh, L, s);
+    if (hi > n) hi = n;
+    if (lo < 0) lo = 0;
+    for (int d = 0; d < dv; ++d) o_row[d] = 0.0;
+    if (hi <= lo) return -INFINITY;
+
+    const uint16_t* qp = q + (((size_t)b * sh->s_q + s) * sh->h_q + h) * (size_t)d_qk;
+    for (int d = 0; d < d_qk; ++d) qrow[d] = mla_oracle_half_to_double(qp[d], sh->dtype);
+
+    /* x_j = scale * <q, k_j>, k_j gathered through the block table. */
+    double M = -INFINITY;
+    for (long j = lo; j < hi; ++j) {
+        long page = block_table[(size_t)b * sh->max_blocks_per_seq + j / P];
+        const uint16_t* kp = kv + (((size_t)page * P + (j % P)) * sh->h_kv + g) * (size_t)d_qk;
+        double acc = 0.0;
+        for (int d = 0; d < d_qk; ++d) acc += qrow[d] * mla_oracle_half_to_double(kp[d], sh->dtype);
+        x[j - lo] = sh->scale * acc;
+        if (x[j - lo] > M) M = x[j - lo];
+    }
+    /* LSE = M + log sum exp(x_j - M) */
+    double sum = 0.0;
+    for (long j = lo; j < hi; ++j) sum += exp(x[j - lo] - M);
+    double lse = M + log(sum);
+    /* O = sum_j exp(x_j - LSE) v_j, v_j = k_j[0:dv] */
+    for (long j = lo; j < hi; ++j) {
+        long page = block_table[(size_t)b * sh->max_blocks_per_seq + j / P];
+        const uint16_t* vp = kv + (((size_t)page * P + (j % P)) * sh->h_kv + g) * (size_t)d_qk;
+        double w = exp(x[j - lo] - lse);
+        for (int d = 0; d < dv; ++d) o_row[d] += w * mla_oracle_half_to_double(vp[d], sh->dtype);
+    }
+    return lse;
+}
+
+static long oracle_max_len(const mla_oracle_shape* sh, const int32_t* seqlens)
+{
+    long mx = 1;
+    for (int b = 0; b < sh->batch; ++b)
+        if (seqlens[b] > mx) mx = seqlens[b];
+    return mx;
+}
+
+/*
+ * Partial attention over the token range [lo, hi) of every request (the same
+ * range for all requests; hi is clipped to each row's visible length).
+ * o: [batch, s_q, h_q, dv] f64, lse: [batch, s_q, h_q] f64.
+ * Returns 0 on success, -1 on bad arguments.
+ */
+int mla_oracle_decode_range(const mla_oracle_shape* sh, const uint16_t* q, const uint16_t* kv,
+                            const int32_t* block_table, const int32_t* seqlens, long lo,
+                            long hi, double* o, double* lse)
+{
+    if (sh->batch < 0 || sh->s_q <= 0 || sh->h_q <= 0 || sh->h_kv <= 0 ||
+        sh->h_q % sh->h_kv != 0 || sh->dv > sh->d_qk || sh->page_size <= 0)
+        return -1;
+    const long maxlen = oracle_max_len(sh, seqlens);
+    const long rows = (long)sh->batch * sh->s_q * sh->h_q;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* x = (double*)malloc(sizeof(double) * (size_t)maxlen);
+        double* qrow = (double*)malloc(sizeof(double) * (size_t)sh->d_qk);
+        if (!x || !qrow) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long r = 0; r < rows; ++r) {
+                int h = (int)(r % sh->h_q);
+                int s = (int)((r / sh->h_q) % sh->s_q);
+                int b = (int)(r / ((long)sh->h_q * sh->s_q));
+                long L = seqlens[b];
+                long h_end = hi < 0 ? L : hi;
+                lse[r] = oracle_one_row(sh, q, kv, block_table, L, b, s, h, lo, h_end, x, qrow,
+                                        o + (size_t)r * sh->dv);
+            }
+        }
+        free(x);
+        free(qrow);
+    }
+    return err ? -1 : 0;
+}
+
+/* Full attention: the range [0, L_b) of each request. */
+int mla_oracle_decode(const mla_oracle_shape* sh, const uint16_t* q, const uint16_t* kv,
+                      const int32_t* block_table, const int32_t* seqlens, double* o,
+                      double* lse)
+{
+    return mla_oracle_decode_range(sh, q, kv, block_table, seqlens, 0, -1, o, lse);
+}
+
+/*
+ * Same as mla_oracle_decode but only for the listed flat rows r = (b*s_q+s)*h_q+h;
+ * used to check sampled outputs of large problems.  o: [n_rows, dv], lse: [n_rows].
+ */
+int mla_oracle_decode_rows(const mla_oracle_shape* sh, const uint16_t* q, const uint16_t* kv,
+                           const int32_t* block_table, const int32_t* seqlens,
+                           const int64_t* row_ids, long n_rows, double* o, double* lse)
+{
+    const long maxlen = oracle_max_len(sh, seqlens);
+    const long rows = (long)sh->batch * sh->s_q * sh->h_q;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* x = (double*)malloc(sizeof(double) * (size_t)maxlen);
+        double* qrow = (double*)malloc(sizeof(double) * (size_t)sh->d_qk);
+        if (!x || !qrow) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long i = 0; i < n_rows; ++i) {
+                long r = row_ids[i];
+                if (r < 0 || r >= rows) {
+#pragma omp atomic write
+                    err = 1;
+                    continue;
+                }
+                int h = (int)(r % sh->h_q);
+                int s = (int)((r / sh->h_q) % sh->s_q);
+                int b = (int)(r / ((long)sh->h_q * sh->s_q));
+                long L = seqlens[b];
+                lse[i] = oracle_one_row(sh, q, kv, block_table, L, b, s, h, 0, L, x, qrow,
+                                        o + (size_t)i * sh->dv);
+            }
+        }
+        free(x);
+        free(qrow);
+    }
+    return err ? -1 : 0;
+}
+
+/*
+ * Merge of n_parts partial results of the same rows, each the attention over a
+ * disjoint token range:  LSE = log sum_k exp(lse_k),  O = sum_k exp(lse_k - LSE) O_k.
+ * Parts with lse_k = -inf carry no tokens and get weight 0; if every part is
+ * empty the result is O = 0, LSE = -inf.  This is the exact identity that makes
+ * splitting the KV range and combining afterwards equal to the unsplit result
+ * (the split-KV and combine kernels named on the "FlashMLA vLLM Optimization"
+ * page, background section).
+ * o_parts: [n_parts, rows, dv], lse_parts: [n_parts, rows]; o: [rows, dv], lse: [rows].
+ */
+void mla_oracle_combine(int n_parts, long rows, int dv, const double* o_parts,
+                        const double* lse_parts, double* o, double* lse)
+{
+    for (long r = 0; r < rows; ++r) {
+        double M = -INFINITY;
+        for (int k = 0; k < n_parts; ++k)
+            if (lse_parts[(size_t)k * rows + r] > M) M = lse_parts[(size_t)k * rows + r];
+        for (int d = 0; d < dv; ++d) o[(size_t)r * dv + d] = 0.0;
+        if (M == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double sum = 0.0;
+        for (int k = 0; k < n_parts; ++k) sum += exp(lse_parts[(size_t)k * rows + r] - M);
+        double L = M + log(sum);
+        lse[r] = L;
+        for (int k = 0; k < n_parts; ++k) {
+            double w = exp(lse_parts[(size_t)k * rows + r] - L);
+            if (w == 0.0) continue;
+            const double* op = o_parts + ((size_t)k * rows + r) * dv;
+            for (int d = 0; d < dv; ++d) o[(size_t)r * dv + d] += w * op[d];
+        }
+    }
+}
