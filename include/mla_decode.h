@@ -1,0 +1,174 @@
+/*
+ * mla_decode.h -- C ABI of the Blackwell (sm_100a) MLA decoding library.
+ *
+ * Multi-head latent attention (MLA) decoding over a paged latent KV cache, in
+ * the "MQA mode" of the upstream FlashMLA documentation ("MLA Mode" footnote to
+ * the support matrix): every query head attends one shared latent KV head whose
+ * cached rows are d_qk = 576 wide (512 latent columns, then 64 RoPE columns) or
+ * d_qk = 512 wide (no RoPE part); V is the leading d_v = 512 columns of the same
+ * rows.  Cached tokens sit in 64-token pages found through a block table.
+ *
+ * The call sequence is the one the "FlashMLA" usage page (deepep.org) shows:
+ * mla_get_metadata once per decoding step (its result is reused by every
+ * layer), then mla_decode_with_kvcache once per layer, which returns (o, lse).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named "device" are CUDA device pointers; "host" ones are host memory.
+ *   - The caller allocates and owns every buffer.  The library allocates no
+ *     memory and keeps no state between calls (apart from a per-process cache
+ *     of one CUDA driver entry point).
+ *   - Calls taking a stream enqueue work on it and return without
+ *     synchronising; results are ready when the stream reaches that point.
+ *     A stream of NULL means the legacy default stream.
+ *   - Invalid arguments are rejected on the host before anything is enqueued;
+ *     the return value says why (mla_status_string gives a message).
+ *   - Errors that only the device can see (a block-table entry outside the
+ *     cache, a pipeline wait that ran out of time) are recorded in a status
+ *     word at the start of the workspace; mla_read_device_status reads it.
+ *
+ * Array layouts (all row-major / C order):
+ *   q             [batch, s_q, h_q, d_qk]             bf16 or fp16
+ *   kvcache       [num_blocks, 64, h_kv, d_qk]        same dtype as q
+ *   block_table   [batch, max_blocks_per_seq] int32   physical page ids; only the
+ *                                                     first ceil(L_b / 64) entries
+ *                                                     of row b are read
+ *   cache_seqlens [batch] int32                       L_b >= 0
+ *   o             [batch, s_q, h_q, 512]              same dtype as q
+ *   lse           [batch, s_q, h_q] float32           natural log
+ *   tile_md       [num_parts, 8] int32                scheduler output (opaque)
+ *   num_splits    [batch * row_groups + 1] int32      scheduler output, prefix sums
+ */
+#ifndef MLA_DECODE_H_
+#define MLA_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_PAGE_SIZE 64       /* tokens per KV-cache page ("block size of 64") */
+#define MLA_HEAD_DIM_V 512     /* d_v: the latent width */
+#define MLA_MD_INTS 8          /* int32 entries per row of tile_md */
+#define MLA_ROWS_PER_GROUP 128 /* query rows (s_q * h_q) handled per row group */
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misaligned buffer, ... */
+    MLA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+    MLA_ERR_WORKSPACE = 3,    /* workspace smaller than mla_decode_workspace_bytes */
+    MLA_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
+    MLA_ERR_TIMEOUT = 5,      /* device: a pipeline wait gave up (kernel returned early) */
+    MLA_ERR_DEVICE_CHECK = 6  /* device: a needed block-table entry was outside [0, num_blocks),
+                                 or a sequence needs more than max_blocks_per_seq pages */
+} mla_status;
+
+typedef enum { MLA_BF16 = 0, MLA_FP16 = 1 } mla_dtype;
+
+/* Message for a status code; never NULL. */
+MLA_API const char* mla_status_string(int status);
+
+/*
+ * Number of scheduler partitions for a device: one per pair of SMs (the
+ * decode kernel runs one two-CTA cluster per partition).  On success writes
+ * *num_parts (> 0).  Errors: MLA_ERR_INVALID_ARG (null), MLA_ERR_CUDA (no such
+ * device).
+ */
+MLA_API mla_status mla_num_sm_parts(int device, int* num_parts);
+
+/*
+ * Sizes of the scheduler outputs for a problem: *tile_md_ints = num_parts * 8,
+ * *num_splits_ints = batch * ceil(heads_per_kv / 128) + 1.
+ * heads_per_kv = s_q * h_q / h_kv, as in get_mla_metadata's second argument.
+ */
+MLA_API mla_status mla_metadata_sizes(int batch, int heads_per_kv, int h_kv, int num_parts,
+                              size_t* tile_md_ints, size_t* num_splits_ints);
+
+/*
+ * Tile scheduler ("FlashMLA" usage page: get_mla_metadata(cache_seqlens,
+ * s_q * h_q // h_kv, h_kv) returns tile_scheduler_metadata and num_splits; the
+ * page's Tile Scheduler "distributes work across GPU resources").
+ *
+ * Splits the work -- for each request b and row group of 128 query rows, the
+ * ceil(L_b / 64) pages of its cache plus a fixed per-chunk overhead -- into
+ * num_parts contiguous ranges of nearly equal cost.  A (request, row group)
+ * whose pages fall into more than one range is split; num_splits holds the
+ * prefix sums of the split counts, and the decode call merges split results.
+ *
+ *   cache_seqlens  device [batch] int32
+ *   heads_per_kv   s_q * h_q / h_kv (> 0)
+ *   h_kv           number of KV heads (must be 1: MQA mode)
+ *   num_parts      from mla_num_sm_parts (the same value must be passed to decode)
+ *   tile_md        device [num_parts, 8] int32, written
+ *   num_splits     device [batch * row_groups + 1] int32, written
+ * Runs one small kernel on `stream`; no host synchronisation.
+ */
+MLA_API mla_status mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv,
+                            int num_parts, int32_t* tile_md, int32_t* num_splits, void* stream);
+
+/* Same schedule computed on the host: every pointer is host memory. */
+MLA_API mla_status mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per_kv,
+                                 int h_kv, int num_parts, int32_t* tile_md, int32_t* num_splits);
+
+/*
+ * Bytes of device workspace mla_decode_with_kvcache needs: a 256-byte status
+ * header plus float32 partial outputs and LSEs for up to
+ * batch * row_groups + num_parts splits of 128 rows each.
+ * Returns 0 for invalid sizes.
+ */
+MLA_API size_t mla_decode_workspace_bytes(int batch, int s_q, int h_q, int h_kv, int num_parts);
+
+/*
+ * Dense MLA decoding with a paged KV cache ("FlashMLA" usage page:
+ * flash_mla_with_kvcache(q, kvcache, block_table, cache_seqlens, dv,
+ * tile_scheduler_metadata, num_splits, causal) -> (o, lse); upstream FlashMLA
+ * documentation, "Usage / MLA Decoding": lse is the log-sum-exp of the
+ * attention scores per query head).
+ *
+ * For request b, query token s and head h (kv head 0):
+ *   n      = causal ? clamp(L_b - s_q + 1 + s, 0, L_b) : L_b   (bottom-right mask)
+ *   x_j    = softmax_scale * <q[b,s,h,:], k_j>,  k_j = cached row j (j < n)
+ *   lse    = log(sum_j exp(x_j))                 (-inf when n = 0)
+ *   o      = sum_j exp(x_j - lse) * k_j[0:512]   (0 when n = 0)
+ *
+ *   q, kvcache      device, dtype `dtype`, 16-byte aligned
+ *   d_qk            576 or 512;  dv must be 512;  h_kv must be 1;  page_size must be 64
+ *   block_table     device int32 [batch, max_blocks_per_seq]
+ *   cache_seqlens   device int32 [batch]  (the same array given to mla_get_metadata)
+ *   tile_md, num_splits, num_parts   from mla_get_metadata for this batch
+ *   causal          0 or 1
+ *   softmax_scale   > 0, or <= 0 for 1/sqrt(d_qk)
+ *   o               device [batch, s_q, h_q, 512], dtype `dtype`, 16-byte aligned, written
+ *   lse             device float32 [batch, s_q, h_q], written
+ *   workspace       device, >= mla_decode_workspace_bytes(...), 256-byte aligned
+ * Enqueues the split-KV kernel and the combine kernel on `stream`.  Calls
+ * sharing one workspace must not run concurrently.
+ */
+MLA_API mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, int h_q, int d_qk,
+                                   const void* kvcache, int num_blocks, int page_size, int h_kv,
+                                   const int32_t* block_table, int max_blocks_per_seq,
+                                   const int32_t* cache_seqlens, int dv, int dtype,
+                                   const int32_t* tile_md, int num_parts,
+                                   const int32_t* num_splits, int causal, float softmax_scale,
+                                   void* o, float* lse, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/*
+ * Reads the device status word of a workspace (synchronises `stream`).
+ * *device_status receives MLA_OK or the first device-side error recorded by a
+ * decode call that used this workspace; clear != 0 resets it to MLA_OK.
+ */
+MLA_API mla_status mla_read_device_status(void* workspace, int clear, int* device_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H_ */

@@ -1,1 +1,16 @@
-"""Blackwell-native (sm_100a) MLA decoding over a paged latent KV cache."""
+"""Blackwell-native (sm_100a) MLA decoding over a paged latent KV cache.
+
+Public calls (the names of the pages' API; "FlashMLA" usage page, deepep.org):
+
+* :func:`get_mla_metadata` -- tile-scheduler metadata, once per decoding step;
+* :func:`flash_mla_with_kvcache` -- one decode call per layer, returns ``(o, lse)``.
+
+Both are thin wrappers over the C ABI in ``include/mla_decode.h``; the kernels
+live in ``csrc/``.  ``workloads`` generates seeded synthetic inputs.
+"""
+from .api import (flash_mla_with_kvcache, get_mla_metadata, get_mla_metadata_host, metadata_sizes,
+                  num_sm_parts, read_device_status, workspace_bytes)
+from ._lib import MLAError
+
+__all__ = ["flash_mla_with_kvcache", "get_mla_metadata", "get_mla_metadata_host", "metadata_sizes",
+           "num_sm_parts", "read_device_status", "workspace_bytes", "MLAError"]

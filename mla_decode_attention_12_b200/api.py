@@ -1,0 +1,163 @@
+"""PyTorch-facing calls with the names of the pages' API.
+
+``get_mla_metadata`` and ``flash_mla_with_kvcache`` follow the call sequence of
+the "FlashMLA" usage page (deepep.org): metadata once per decoding step, then
+one decode call per layer returning ``(o, lse)``.  Torch provides device memory
+and the current stream; the arithmetic is done by the C library's kernels.
+
+Inputs on the CPU are accepted too: they are copied to the current CUDA device
+(non-blocking from pinned memory), the kernels run there, and the outputs are
+copied back.  This is the end-to-end path with host buffers.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+
+_DTYPES = {torch.bfloat16: 0, torch.float16: 1}
+_workspaces: dict = {}
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def num_sm_parts(device=None) -> int:
+    """Scheduler partitions of a device (one per pair of SMs)."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else torch.device(device).index or 0)
+    out = ctypes.c_int(0)
+    _lib.check(_lib.load().mla_num_sm_parts(dev.index, ctypes.byref(out)), "mla_num_sm_parts")
+    return out.value
+
+
+def metadata_sizes(batch: int, heads_per_kv: int, h_kv: int, num_parts: int):
+    a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _lib.check(_lib.load().mla_metadata_sizes(batch, heads_per_kv, h_kv, num_parts, ctypes.byref(a),
+                                              ctypes.byref(b)), "mla_metadata_sizes")
+    return a.value, b.value
+
+
+def get_mla_metadata(cache_seqlens: torch.Tensor, heads_per_kv: int, h_kv: int = 1, num_parts: int | None = None):
+    """Tile-scheduler metadata for one decoding step.
+
+    ``cache_seqlens``: int32 [batch] on a CUDA device.  ``heads_per_kv`` is
+    ``s_q * h_q // h_kv``.  Returns ``(tile_scheduler_metadata [num_parts, 8] int32,
+    num_splits [batch * ceil(heads_per_kv / 128) + 1] int32)`` on the same device.
+    """
+    if not cache_seqlens.is_cuda or cache_seqlens.dtype != torch.int32 or not cache_seqlens.is_contiguous():
+        raise ValueError("cache_seqlens must be a contiguous int32 CUDA tensor")
+    dev = cache_seqlens.device
+    if num_parts is None:
+        num_parts = num_sm_parts(dev)
+    batch = cache_seqlens.numel()
+    n_md, n_ns = metadata_sizes(batch, heads_per_kv, h_kv, num_parts)
+    md = torch.empty(n_md, dtype=torch.int32, device=dev).view(num_parts, 8)
+    ns = torch.empty(n_ns, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _lib.check(_lib.load().mla_get_metadata(_ptr(cache_seqlens), batch, heads_per_kv, h_kv, num_parts,
+                                                _ptr(md), _ptr(ns), _stream(dev)), "mla_get_metadata")
+    return md, ns
+
+
+def get_mla_metadata_host(cache_seqlens, heads_per_kv: int, h_kv: int = 1, num_parts: int = 74):
+    """The same schedule computed on the host (numpy in, numpy out)."""
+    import numpy as np
+
+    sl = np.ascontiguousarray(cache_seqlens, dtype=np.int32)
+    n_md, n_ns = metadata_sizes(sl.size, heads_per_kv, h_kv, num_parts)
+    md = np.zeros(n_md, np.int32)
+    ns = np.zeros(n_ns, np.int32)
+    _lib.check(_lib.load().mla_get_metadata_host(sl.ctypes.data, sl.size, heads_per_kv, h_kv, num_parts,
+                                                 md.ctypes.data, ns.ctypes.data), "mla_get_metadata_host")
+    return md.reshape(num_parts, 8), ns
+
+
+def workspace_bytes(batch: int, s_q: int, h_q: int, h_kv: int, num_parts: int) -> int:
+    n = _lib.load().mla_decode_workspace_bytes(batch, s_q, h_q, h_kv, num_parts)
+    if n == 0:
+        raise ValueError("invalid sizes for the decode workspace")
+    return n
+
+
+def get_workspace(nbytes: int, device: torch.device) -> torch.Tensor:
+    """A cached, grow-only workspace per (device, stream); its status header starts zeroed."""
+    key = (device.index, _stream(device))
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        ws[:256].zero_()
+        _workspaces[key] = ws
+    return ws
+
+
+def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: torch.Tensor,
+                           cache_seqlens: torch.Tensor, dv: int, tile_scheduler_metadata: torch.Tensor,
+                           num_splits: torch.Tensor, causal: bool = False, softmax_scale: float | None = None,
+                           workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                           lse: torch.Tensor | None = None):
+    """MLA decode over a paged cache; returns ``(o [b, s_q, h_q, dv], lse [b, s_q, h_q] float32)``.
+
+    ``q`` [b, s_q, h_q, d_qk] and ``kvcache`` [num_blocks, 64, h_kv, d_qk] are bf16 or
+    fp16; ``block_table`` [b, max_blocks] and ``cache_seqlens`` [b] are int32.  With
+    every tensor on the CPU the call copies them to the current CUDA device and the
+    results back (host-buffer path).
+    """
+    host = not q.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        nb = q.is_pinned()
+        q, kvcache, block_table, cache_seqlens = (t.to(dev, non_blocking=nb) for t in
+                                                  (q, kvcache, block_table, cache_seqlens))
+        tile_scheduler_metadata = tile_scheduler_metadata.to(dev, non_blocking=nb)
+        num_splits = num_splits.to(dev, non_blocking=nb)
+    dev = q.device
+    if q.dtype not in _DTYPES or kvcache.dtype != q.dtype:
+        raise ValueError("q and kvcache must both be bfloat16 or both float16")
+    for name, t in (("q", q), ("kvcache", kvcache), ("block_table", block_table),
+                    ("cache_seqlens", cache_seqlens), ("tile_scheduler_metadata", tile_scheduler_metadata),
+                    ("num_splits", num_splits)):
+        if not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must be contiguous and on {dev}")
+    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32:
+        raise ValueError("block_table and cache_seqlens must be int32")
+    b, s_q, h_q, d_qk = q.shape
+    num_blocks, page, h_kv, d2 = kvcache.shape
+    if d2 != d_qk or block_table.dim() != 2 or block_table.shape[0] != b or cache_seqlens.numel() != b:
+        raise ValueError("inconsistent shapes")
+    num_parts = tile_scheduler_metadata.shape[0]
+    if out is None:
+        out = torch.empty(b, s_q, h_q, dv, dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty(b, s_q, h_q, dtype=torch.float32, device=dev)
+    need = workspace_bytes(b, s_q, h_q, h_kv, num_parts)
+    if workspace is None:
+        workspace = get_workspace(need, dev)
+    scale = float(softmax_scale) if softmax_scale is not None else 1.0 / math.sqrt(d_qk)
+    with torch.cuda.device(dev):
+        st = _lib.load().mla_decode_with_kvcache(
+            _ptr(q), b, s_q, h_q, d_qk, _ptr(kvcache), num_blocks, page, h_kv, _ptr(block_table),
+            block_table.shape[1], _ptr(cache_seqlens), dv, _DTYPES[q.dtype], _ptr(tile_scheduler_metadata),
+            num_parts, _ptr(num_splits), int(bool(causal)), scale, _ptr(out), _ptr(lse), _ptr(workspace),
+            workspace.numel(), _stream(dev))
+    _lib.check(st, "mla_decode_with_kvcache")
+    if host:
+        return out.cpu(), lse.cpu()
+    return out, lse
+
+
+def read_device_status(workspace: torch.Tensor, clear: bool = True) -> int:
+    """Device-side status recorded in a workspace (synchronises the current stream)."""
+    v = ctypes.c_int(0)
+    dev = workspace.device
+    with torch.cuda.device(dev):
+        _lib.check(_lib.load().mla_read_device_status(_ptr(workspace), int(clear), ctypes.byref(v), _stream(dev)),
+                   "mla_read_device_status")
+    return v.value

@@ -1,0 +1,97 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects bad
+arguments on the host before touching the GPU (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mla_decode_attention_12_b200 import _lib, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "mla_decode.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MLA_API\s+[\w\s\*]*?\b(mla_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for must in ("mla_get_metadata", "mla_decode_with_kvcache", "mla_decode_workspace_bytes"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert _lib.status_string(code)
+    assert _lib.status_string(99) == "unknown status"
+
+
+def test_sizes(lib):
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.mla_metadata_sizes(64, 128, 1, 74, ctypes.byref(a), ctypes.byref(b)) == 0
+    assert (a.value, b.value) == (74 * 8, 64 + 1)
+    assert lib.mla_metadata_sizes(32, 256, 1, 74, ctypes.byref(a), ctypes.byref(b)) == 0
+    assert b.value == 32 * 2 + 1
+    assert lib.mla_metadata_sizes(-1, 128, 1, 74, ctypes.byref(a), ctypes.byref(b)) == 1
+    # workspace: header + (NV + parts) * 128 * (1 + 512) floats
+    nv, parts = 64, 74
+    want = 256 + ((nv + parts) * 128 * 4 + 255) // 256 * 256 + (nv + parts) * 128 * 512 * 4
+    assert lib.mla_decode_workspace_bytes(64, 1, 128, 1, 74) == want
+    assert lib.mla_decode_workspace_bytes(64, 0, 128, 1, 74) == 0
+
+
+def _decode(lib, **over):
+    fake = 1 << 20  # aligned non-null "device" pointers: validation must reject before any use
+    args = dict(q=fake, batch=2, s_q=1, h_q=16, d_qk=576, kvcache=fake, num_blocks=8, page_size=64, h_kv=1,
+                block_table=fake, max_blocks=4, seqlens=fake, dv=512, dtype=0, md=fake, num_parts=74,
+                num_splits=fake, causal=0, scale=0.0, o=fake, lse=fake, ws=fake,
+                ws_bytes=1 << 40, stream=None)
+    args.update(over)
+    return lib.mla_decode_with_kvcache(*args.values())
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), 1), (dict(o=None), 1), (dict(ws=None), 1), (dict(block_table=None), 1),
+    (dict(batch=-1), 1), (dict(s_q=0), 1), (dict(h_q=0), 1), (dict(num_blocks=0), 1),
+    (dict(causal=2), 1), (dict(dtype=7), 1), (dict(q=(1 << 20) + 2), 1), (dict(ws=(1 << 20) + 16), 1),
+    (dict(page_size=32), 2), (dict(h_kv=2), 2), (dict(d_qk=192), 2), (dict(dv=256), 2),
+    (dict(ws_bytes=1000), 3),
+])
+def test_decode_rejects_bad_arguments(lib, over, code):
+    assert _decode(lib, **over) == code
+
+
+def test_decode_empty_batch_is_a_no_op(lib):
+    assert _decode(lib, batch=0, q=None, o=None) == 0
+
+
+def test_metadata_rejects_bad_arguments(lib):
+    fake = 1 << 20
+    assert lib.mla_get_metadata(fake, 4, 0, 1, 74, fake, fake, None) == 1
+    assert lib.mla_get_metadata(fake, 4, 128, 2, 74, fake, fake, None) == 2
+    assert lib.mla_get_metadata(fake, 4, 128, 1, 0, fake, fake, None) == 1
+    assert lib.mla_get_metadata(None, 4, 128, 1, 74, fake, fake, None) == 1
+
+
+def test_host_metadata_rejects_negative_lengths(lib):
+    import numpy as np
+
+    sl = np.array([5, -1], np.int32)
+    md = np.zeros(74 * 8, np.int32)
+    ns = np.zeros(3, np.int32)
+    assert lib.mla_get_metadata_host(sl.ctypes.data, 2, 16, 1, 74, md.ctypes.data, ns.ctypes.data) == 1
