@@ -161,6 +161,35 @@ MLA_API mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, in
                                    void* stream);
 
 /*
+ * The two stages of mla_decode_with_kvcache, for callers that schedule or time
+ * them separately (the split-KV / combine kernel pair named on the "FlashMLA
+ * vLLM Optimization" page, background section).  Calling mla_decode_splitkv
+ * and then mla_decode_combine on one stream with the same arguments is exactly
+ * mla_decode_with_kvcache.
+ *
+ * mla_decode_splitkv: same arguments and checks as mla_decode_with_kvcache.
+ *   Each (request, row group) processed by one partition is written to o / lse
+ *   directly; one spread over several partitions leaves float32 partial results
+ *   in the workspace.
+ * mla_decode_combine: merges those partial results into o / lse
+ *   (lse = log sum_k exp(lse_k), o = sum_k exp(lse_k - lse) o_k); batch, s_q,
+ *   h_q, h_kv, dv, dtype, num_splits, num_parts, o, lse and workspace must be
+ *   the ones given to mla_decode_splitkv.
+ */
+MLA_API mla_status mla_decode_splitkv(const void* q, int batch, int s_q, int h_q, int d_qk,
+                                      const void* kvcache, int num_blocks, int page_size, int h_kv,
+                                      const int32_t* block_table, int max_blocks_per_seq,
+                                      const int32_t* cache_seqlens, int dv, int dtype,
+                                      const int32_t* tile_md, int num_parts,
+                                      const int32_t* num_splits, int causal, float softmax_scale,
+                                      void* o, float* lse, void* workspace, size_t workspace_bytes,
+                                      void* stream);
+
+MLA_API mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int dtype,
+                                      const int32_t* num_splits, int num_parts, void* o, float* lse,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Reads the device status word of a workspace (synchronises `stream`).
  * *device_status receives MLA_OK or the first device-side error recorded by a
  * decode call that used this workspace; clear != 0 resets it to MLA_OK.

@@ -45,22 +45,31 @@ def metadata_sizes(batch: int, heads_per_kv: int, h_kv: int, num_parts: int):
     return a.value, b.value
 
 
-def get_mla_metadata(cache_seqlens: torch.Tensor, heads_per_kv: int, h_kv: int = 1, num_parts: int | None = None):
+def get_mla_metadata(cache_seqlens: torch.Tensor, heads_per_kv: int, h_kv: int = 1, num_parts: int | None = None,
+                     out=None):
     """Tile-scheduler metadata for one decoding step.
 
     ``cache_seqlens``: int32 [batch] on a CUDA device.  ``heads_per_kv`` is
     ``s_q * h_q // h_kv``.  Returns ``(tile_scheduler_metadata [num_parts, 8] int32,
-    num_splits [batch * ceil(heads_per_kv / 128) + 1] int32)`` on the same device.
+    num_splits [batch * ceil(heads_per_kv / 128) + 1] int32)`` on the same device;
+    ``out`` = (md, ns) writes into existing tensors instead.
     """
     if not cache_seqlens.is_cuda or cache_seqlens.dtype != torch.int32 or not cache_seqlens.is_contiguous():
         raise ValueError("cache_seqlens must be a contiguous int32 CUDA tensor")
     dev = cache_seqlens.device
+    if out is not None and num_parts is None:
+        num_parts = out[0].shape[0]
     if num_parts is None:
         num_parts = num_sm_parts(dev)
     batch = cache_seqlens.numel()
     n_md, n_ns = metadata_sizes(batch, heads_per_kv, h_kv, num_parts)
-    md = torch.empty(n_md, dtype=torch.int32, device=dev).view(num_parts, 8)
-    ns = torch.empty(n_ns, dtype=torch.int32, device=dev)
+    if out is not None:
+        md, ns = out
+        if md.numel() != n_md or ns.numel() != n_ns or md.dtype != torch.int32 or ns.dtype != torch.int32:
+            raise ValueError("metadata output tensors have the wrong size or dtype")
+    else:
+        md = torch.empty(n_md, dtype=torch.int32, device=dev).view(num_parts, 8)
+        ns = torch.empty(n_ns, dtype=torch.int32, device=dev)
     with torch.cuda.device(dev):
         _lib.check(_lib.load().mla_get_metadata(_ptr(cache_seqlens), batch, heads_per_kv, h_kv, num_parts,
                                                 _ptr(md), _ptr(ns), _stream(dev)), "mla_get_metadata")
@@ -98,6 +107,60 @@ def get_workspace(nbytes: int, device: torch.device) -> torch.Tensor:
     return ws
 
 
+class DecodeCall:
+    """Marshalled arguments of one decode call (device tensors), reusable across stages."""
+
+    def __init__(self, q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata, num_splits,
+                 causal=False, softmax_scale=None, workspace=None, out=None, lse=None):
+        dev = q.device
+        if q.dtype not in _DTYPES or kvcache.dtype != q.dtype:
+            raise ValueError("q and kvcache must both be bfloat16 or both float16")
+        for name, t in (("q", q), ("kvcache", kvcache), ("block_table", block_table),
+                        ("cache_seqlens", cache_seqlens), ("tile_scheduler_metadata", tile_scheduler_metadata),
+                        ("num_splits", num_splits)):
+            if not t.is_contiguous() or t.device != dev:
+                raise ValueError(f"{name} must be contiguous and on {dev}")
+        if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32:
+            raise ValueError("block_table and cache_seqlens must be int32")
+        b, s_q, h_q, d_qk = q.shape
+        num_blocks, page, h_kv, d2 = kvcache.shape
+        if d2 != d_qk or block_table.dim() != 2 or block_table.shape[0] != b or cache_seqlens.numel() != b:
+            raise ValueError("inconsistent shapes")
+        num_parts = tile_scheduler_metadata.shape[0]
+        if out is None:
+            out = torch.empty(b, s_q, h_q, dv, dtype=q.dtype, device=dev)
+        if lse is None:
+            lse = torch.empty(b, s_q, h_q, dtype=torch.float32, device=dev)
+        if workspace is None:
+            workspace = get_workspace(workspace_bytes(b, s_q, h_q, h_kv, num_parts), dev)
+        scale = float(softmax_scale) if softmax_scale is not None else 1.0 / math.sqrt(d_qk)
+        self.device = dev
+        self.out, self.lse, self.workspace = out, lse, workspace
+        self._keep = (q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits)
+        self.args = (_ptr(q), b, s_q, h_q, d_qk, _ptr(kvcache), num_blocks, page, h_kv, _ptr(block_table),
+                     block_table.shape[1], _ptr(cache_seqlens), dv, _DTYPES[q.dtype],
+                     _ptr(tile_scheduler_metadata), num_parts, _ptr(num_splits), int(bool(causal)), scale,
+                     _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel())
+        self.combine_args = (b, s_q, h_q, h_kv, dv, _DTYPES[q.dtype], _ptr(num_splits), num_parts, _ptr(out),
+                             _ptr(lse), _ptr(workspace), workspace.numel())
+
+    def run(self):
+        """Split-KV kernel then combine kernel (mla_decode_with_kvcache)."""
+        with torch.cuda.device(self.device):
+            _lib.check(_lib.load().mla_decode_with_kvcache(*self.args, _stream(self.device)),
+                       "mla_decode_with_kvcache")
+        return self.out, self.lse
+
+    def splitkv(self):
+        with torch.cuda.device(self.device):
+            _lib.check(_lib.load().mla_decode_splitkv(*self.args, _stream(self.device)), "mla_decode_splitkv")
+
+    def combine(self):
+        with torch.cuda.device(self.device):
+            _lib.check(_lib.load().mla_decode_combine(*self.combine_args, _stream(self.device)),
+                       "mla_decode_combine")
+
+
 def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: torch.Tensor,
                            cache_seqlens: torch.Tensor, dv: int, tile_scheduler_metadata: torch.Tensor,
                            num_splits: torch.Tensor, causal: bool = False, softmax_scale: float | None = None,
@@ -107,47 +170,19 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
 
     ``q`` [b, s_q, h_q, d_qk] and ``kvcache`` [num_blocks, 64, h_kv, d_qk] are bf16 or
     fp16; ``block_table`` [b, max_blocks] and ``cache_seqlens`` [b] are int32.  With
-    every tensor on the CPU the call copies them to the current CUDA device and the
-    results back (host-buffer path).
+    ``q`` on the CPU the inputs are copied to the current CUDA device (non-blocking
+    when pinned) and the results copied back (host-buffer path).
     """
     host = not q.is_cuda
     if host:
         dev = torch.device("cuda", torch.cuda.current_device())
         nb = q.is_pinned()
-        q, kvcache, block_table, cache_seqlens = (t.to(dev, non_blocking=nb) for t in
-                                                  (q, kvcache, block_table, cache_seqlens))
-        tile_scheduler_metadata = tile_scheduler_metadata.to(dev, non_blocking=nb)
-        num_splits = num_splits.to(dev, non_blocking=nb)
-    dev = q.device
-    if q.dtype not in _DTYPES or kvcache.dtype != q.dtype:
-        raise ValueError("q and kvcache must both be bfloat16 or both float16")
-    for name, t in (("q", q), ("kvcache", kvcache), ("block_table", block_table),
-                    ("cache_seqlens", cache_seqlens), ("tile_scheduler_metadata", tile_scheduler_metadata),
-                    ("num_splits", num_splits)):
-        if not t.is_contiguous() or t.device != dev:
-            raise ValueError(f"{name} must be contiguous and on {dev}")
-    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32:
-        raise ValueError("block_table and cache_seqlens must be int32")
-    b, s_q, h_q, d_qk = q.shape
-    num_blocks, page, h_kv, d2 = kvcache.shape
-    if d2 != d_qk or block_table.dim() != 2 or block_table.shape[0] != b or cache_seqlens.numel() != b:
-        raise ValueError("inconsistent shapes")
-    num_parts = tile_scheduler_metadata.shape[0]
-    if out is None:
-        out = torch.empty(b, s_q, h_q, dv, dtype=q.dtype, device=dev)
-    if lse is None:
-        lse = torch.empty(b, s_q, h_q, dtype=torch.float32, device=dev)
-    need = workspace_bytes(b, s_q, h_q, h_kv, num_parts)
-    if workspace is None:
-        workspace = get_workspace(need, dev)
-    scale = float(softmax_scale) if softmax_scale is not None else 1.0 / math.sqrt(d_qk)
-    with torch.cuda.device(dev):
-        st = _lib.load().mla_decode_with_kvcache(
-            _ptr(q), b, s_q, h_q, d_qk, _ptr(kvcache), num_blocks, page, h_kv, _ptr(block_table),
-            block_table.shape[1], _ptr(cache_seqlens), dv, _DTYPES[q.dtype], _ptr(tile_scheduler_metadata),
-            num_parts, _ptr(num_splits), int(bool(causal)), scale, _ptr(out), _ptr(lse), _ptr(workspace),
-            workspace.numel(), _stream(dev))
-    _lib.check(st, "mla_decode_with_kvcache")
+        q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits = (
+            t.to(dev, non_blocking=nb) for t in
+            (q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits))
+    call = DecodeCall(q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata, num_splits,
+                      causal=causal, softmax_scale=softmax_scale, workspace=workspace, out=out, lse=lse)
+    out, lse = call.run()
     if host:
         return out.cpu(), lse.cpu()
     return out, lse

@@ -114,6 +114,7 @@ struct DecodeParams {
     int* status;
     int batch, s_q, h_q, rows, groups, max_blocks, num_blocks, causal, box_rows;
     float scale_log2;
+    int dtype, d_qk, num_parts;  // host-side dispatch only
 };
 
 // ------------------------------------------------------------------ helpers
@@ -812,20 +813,21 @@ size_t mla_decode_workspace_bytes(int batch, int s_q, int h_q, int h_kv, int num
     return bytes;
 }
 
-mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache,
-                                   int num_blocks, int page_size, int h_kv, const int32_t* block_table,
-                                   int max_blocks_per_seq, const int32_t* cache_seqlens, int dv, int dtype,
-                                   const int32_t* tile_md, int num_parts, const int32_t* num_splits, int causal,
-                                   float softmax_scale, void* o, float* lse, void* workspace,
-                                   size_t workspace_bytes, void* stream)
+// Validates the arguments and fills the kernel parameters and tensor maps.
+static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache,
+                                 int num_blocks, int page_size, int h_kv, const int32_t* block_table,
+                                 int max_blocks_per_seq, const int32_t* cache_seqlens, int dv, int dtype,
+                                 const int32_t* tile_md, int num_parts, const int32_t* num_splits, int causal,
+                                 float softmax_scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                                 DecodeParams& prm, CUtensorMap* maps)
 {
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
         num_parts <= 0 || (causal != 0 && causal != 1))
         return MLA_ERR_INVALID_ARG;
     if (dtype != MLA_BF16 && dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
     if (page_size != kPage || h_kv != 1 || (d_qk != 576 && d_qk != 512) || dv != kDv) return MLA_ERR_UNSUPPORTED;
-    if (batch == 0) return MLA_OK;
-    if (!q || !kvcache || !block_table || !cache_seqlens || !tile_md || !num_splits || !o || !lse || !workspace)
+    if (batch > 0 && (!q || !kvcache || !block_table || !cache_seqlens || !tile_md || !num_splits || !o || !lse ||
+                      !workspace))
         return MLA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kvcache) & 15) ||
         (reinterpret_cast<uintptr_t>(o) & 15) || (reinterpret_cast<uintptr_t>(workspace) & 255))
@@ -833,42 +835,16 @@ mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, int h_q, i
     const int rows = s_q * h_q;
     const int groups = row_groups(rows);
     const size_t need = mla_decode_workspace_bytes(batch, s_q, h_q, h_kv, num_parts);
-    if (workspace_bytes < need) return MLA_ERR_WORKSPACE;
+    if (batch > 0 && workspace_bytes < need) return MLA_ERR_WORKSPACE;
     if (static_cast<long long>(num_blocks) * kPage >= (1ll << 31)) return MLA_ERR_UNSUPPORTED;
     if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt(static_cast<float>(d_qk));
-
-    const CUtensorMapDataType dt =
-        dtype == MLA_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const int box_rows = rows < kRowsPerGroup ? rows : kRowsPerGroup;
-    CUtensorMap tq128, tq64, tkv128, tkv64;
-    const uint64_t row_bytes = static_cast<uint64_t>(d_qk) * 2;
-    bool ok = encode_3d(&tq128, q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 64, box_rows,
-                        CU_TENSOR_MAP_SWIZZLE_128B) &&
-              encode_2d(&tkv128, kvcache, dt, d_qk, static_cast<uint64_t>(num_blocks) * kPage, row_bytes, 64,
-                        kPage, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (ok && d_qk == 576)
-        ok = encode_3d(&tq64, q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 32, box_rows,
-                       CU_TENSOR_MAP_SWIZZLE_64B) &&
-             encode_2d(&tkv64, kvcache, dt, d_qk, static_cast<uint64_t>(num_blocks) * kPage, row_bytes, 32, kPage,
-                       CU_TENSOR_MAP_SWIZZLE_64B);
-    else {
-        tq64 = tq128;
-        tkv64 = tkv128;
-    }
-    if (!ok) return MLA_ERR_CUDA;
-
-    const size_t slots = workspace_slots(batch, groups, num_parts);
-    DecodeParams prm{};
+    prm = DecodeParams{};
     prm.block_table = block_table;
     prm.seqlens = cache_seqlens;
     prm.md = tile_md;
     prm.num_splits = num_splits;
     prm.o = o;
     prm.lse = lse;
-    prm.status = static_cast<int*>(workspace);
-    prm.lse_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader);
-    prm.o_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader +
-                                           align_up(slots * kRowsPerGroup * sizeof(float), 256));
     prm.batch = batch;
     prm.s_q = s_q;
     prm.h_q = h_q;
@@ -877,25 +853,122 @@ mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, int h_q, i
     prm.max_blocks = max_blocks_per_seq;
     prm.num_blocks = num_blocks;
     prm.causal = causal;
-    prm.box_rows = box_rows;
+    prm.box_rows = rows < kRowsPerGroup ? rows : kRowsPerGroup;
     prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+    prm.dtype = dtype;
+    prm.d_qk = d_qk;
+    prm.num_parts = num_parts;
+    if (batch == 0) return MLA_OK;
+    const size_t slots = workspace_slots(batch, groups, num_parts);
+    prm.status = static_cast<int*>(workspace);
+    prm.lse_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader);
+    prm.o_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader +
+                                           align_up(slots * kRowsPerGroup * sizeof(float), 256));
+    if (!maps) return MLA_OK;
 
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int grid = 2 * num_parts;
+    const CUtensorMapDataType dt =
+        dtype == MLA_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const uint64_t row_bytes = static_cast<uint64_t>(d_qk) * 2;
+    const uint64_t kv_rows = static_cast<uint64_t>(num_blocks) * kPage;
+    bool ok = encode_3d(&maps[0], q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 64, prm.box_rows,
+                        CU_TENSOR_MAP_SWIZZLE_128B) &&
+              encode_2d(&maps[2], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (ok && d_qk == 576)
+        ok = encode_3d(&maps[1], q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 32, prm.box_rows,
+                       CU_TENSOR_MAP_SWIZZLE_64B) &&
+             encode_2d(&maps[3], kvcache, dt, d_qk, kv_rows, row_bytes, 32, kPage, CU_TENSOR_MAP_SWIZZLE_64B);
+    else {
+        maps[1] = maps[0];
+        maps[3] = maps[2];
+    }
+    return ok ? MLA_OK : MLA_ERR_CUDA;
+}
+
+static mla_status launch_splitkv_stage(const DecodeParams& prm, const CUtensorMap* maps, cudaStream_t st)
+{
+    const int grid = 2 * prm.num_parts;
     cudaError_t e;
-    if (d_qk == 576)
-        e = dtype == MLA_FP16 ? launch_splitkv<true, true>(grid, st, tq128, tq64, tkv128, tkv64, prm)
-                              : launch_splitkv<true, false>(grid, st, tq128, tq64, tkv128, tkv64, prm);
+    if (prm.d_qk == 576)
+        e = prm.dtype == MLA_FP16 ? launch_splitkv<true, true>(grid, st, maps[0], maps[1], maps[2], maps[3], prm)
+                                  : launch_splitkv<true, false>(grid, st, maps[0], maps[1], maps[2], maps[3], prm);
     else
-        e = dtype == MLA_FP16 ? launch_splitkv<false, true>(grid, st, tq128, tq64, tkv128, tkv64, prm)
-                              : launch_splitkv<false, false>(grid, st, tq128, tq64, tkv128, tkv64, prm);
-    if (e != cudaSuccess) return MLA_ERR_CUDA;
-    dim3 cgrid(batch * groups, 4);
-    if (dtype == MLA_FP16)
+        e = prm.dtype == MLA_FP16 ? launch_splitkv<false, true>(grid, st, maps[0], maps[1], maps[2], maps[3], prm)
+                                  : launch_splitkv<false, false>(grid, st, maps[0], maps[1], maps[2], maps[3], prm);
+    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+static mla_status launch_combine_stage(const DecodeParams& prm, cudaStream_t st)
+{
+    dim3 cgrid(prm.batch * prm.groups, 4);
+    if (prm.dtype == MLA_FP16)
         mla_combine_kernel<true><<<cgrid, 256, 0, st>>>(prm);
     else
         mla_combine_kernel<false><<<cgrid, 256, 0, st>>>(prm);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+#define MLA_DECODE_ARGS                                                                                          \
+    q, batch, s_q, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, block_table, max_blocks_per_seq,            \
+        cache_seqlens, dv, dtype, tile_md, num_parts, num_splits, causal, softmax_scale, o, lse, workspace,      \
+        workspace_bytes
+
+mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache,
+                                   int num_blocks, int page_size, int h_kv, const int32_t* block_table,
+                                   int max_blocks_per_seq, const int32_t* cache_seqlens, int dv, int dtype,
+                                   const int32_t* tile_md, int num_parts, const int32_t* num_splits, int causal,
+                                   float softmax_scale, void* o, float* lse, void* workspace,
+                                   size_t workspace_bytes, void* stream)
+{
+    DecodeParams prm;
+    CUtensorMap maps[4];
+    mla_status s = prepare_decode(MLA_DECODE_ARGS, prm, maps);
+    if (s != MLA_OK || batch == 0) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = launch_splitkv_stage(prm, maps, st);
+    if (s != MLA_OK) return s;
+    return launch_combine_stage(prm, st);
+}
+
+mla_status mla_decode_splitkv(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache,
+                              int num_blocks, int page_size, int h_kv, const int32_t* block_table,
+                              int max_blocks_per_seq, const int32_t* cache_seqlens, int dv, int dtype,
+                              const int32_t* tile_md, int num_parts, const int32_t* num_splits, int causal,
+                              float softmax_scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                              void* stream)
+{
+    DecodeParams prm;
+    CUtensorMap maps[4];
+    mla_status s = prepare_decode(MLA_DECODE_ARGS, prm, maps);
+    if (s != MLA_OK || batch == 0) return s;
+    return launch_splitkv_stage(prm, maps, static_cast<cudaStream_t>(stream));
+}
+
+mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int dtype, const int32_t* num_splits,
+                              int num_parts, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                              void* stream)
+{
+    if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_parts <= 0) return MLA_ERR_INVALID_ARG;
+    if (dtype != MLA_BF16 && dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
+    if (h_kv != 1 || dv != kDv) return MLA_ERR_UNSUPPORTED;
+    if (batch == 0) return MLA_OK;
+    if (!num_splits || !o || !lse || !workspace) return MLA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return MLA_ERR_INVALID_ARG;
+    if (workspace_bytes < mla_decode_workspace_bytes(batch, s_q, h_q, h_kv, num_parts)) return MLA_ERR_WORKSPACE;
+    const int rows = s_q * h_q;
+    const int groups = row_groups(rows);
+    const size_t slots = workspace_slots(batch, groups, num_parts);
+    DecodeParams prm{};
+    prm.num_splits = num_splits;
+    prm.o = o;
+    prm.lse = lse;
+    prm.rows = rows;
+    prm.groups = groups;
+    prm.batch = batch;
+    prm.dtype = dtype;
+    prm.lse_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader);
+    prm.o_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader +
+                                           align_up(slots * kRowsPerGroup * sizeof(float), 256));
+    return launch_combine_stage(prm, static_cast<cudaStream_t>(stream));
 }
 
 mla_status mla_read_device_status(void* workspace, int clear, int* device_status, void* stream)
