@@ -55,52 +55,56 @@
 
 namespace mla {
 
-constexpr int kThreads = 192;          // 4 softmax warps + TMA warp + MMA warp
-constexpr int kTmaWarp = 4;
+constexpr int kThreads = 224;          // 4 softmax warps + Q/K loader + MMA issuer + V loader
+constexpr int kKWarp = 4;
 constexpr int kMmaWarp = 5;
+constexpr int kVWarp = 6;
 constexpr int kDv = 512;
-constexpr int kDvHalf = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 0;         // O half: columns [0, 256)
-constexpr uint32_t kTmemS = 256;       // S/P buffers: [256, 320), [320, 384)
+constexpr uint32_t kTmemO = 0;         // O: columns [0, 256)
+constexpr uint32_t kTmemS = 256;       // S buffers: [256, 288), [288, 320)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 constexpr int kWorkspaceHeader = 256;
 
+// Shared-memory plan of one CTA (each CTA of the pair owns 64 query rows).
 template <bool kRope>
 struct Layout {
-    static constexpr int kBoxes = 4;                                   // 64-column SW128 boxes per CTA
-    static constexpr int kQBytes = kBoxes * 16384 + (kRope ? 8192 : 0);   // 128 rows
-    static constexpr int kStageBytes = kBoxes * 8192 + (kRope ? 4096 : 0);  // 64 tokens
-    static constexpr int kStages = kRope ? 3 : 4;
-    static constexpr int kXBytes = 128 * 64 * 4;                       // peer partial logits
-    static constexpr int kKSlices = kBoxes * 4 + (kRope ? 2 : 0);      // K=16 MMA steps for S
+    static constexpr int kBoxes = kRope ? 9 : 8;               // 64-column boxes in a d_qk row
+    static constexpr int kQBytes = kBoxes * 8192;              // Q: 64 rows x d_qk, one SW128 box per 64 columns
+    static constexpr int kKBytes = kBoxes * 4096;              // K: this CTA's 32 tokens of a page x d_qk
+    static constexpr int kVBytes = 4 * 8192;                   // V: 64 tokens x this CTA's 256 d_v columns
+    static constexpr int kPBytes = 8192;                       // P: 64 rows x 64 tokens, 16-bit
+    static constexpr int kKSteps = kBoxes * 4;                 // K=16 MMA steps of Q K^T
     static constexpr int kOffQ = 0;
-    static constexpr int kOffKV = kOffQ + kQBytes;
-    static constexpr int kOffX = kOffKV + kStages * kStageBytes;
-    static constexpr int kOffBar = kOffX + kXBytes;
+    static constexpr int kOffK = kOffQ + kQBytes;              // 2 stages
+    static constexpr int kOffV = kOffK + 2 * kKBytes;          // 2 stages
+    static constexpr int kOffP = kOffV + 2 * kVBytes;          // 2 buffers
+    static constexpr int kOffRed = kOffP + 2 * kPBytes;        // 2 x 128 floats: row max / sum halves
+    static constexpr int kOffBar = kOffRed + 1024;
     static constexpr int kBarBytes = 512;
-    static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;      // + alignment slack
+    static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
 };
 
-// Barrier slots (8 bytes each) inside the barrier area.
 enum BarSlot : int {
-    kBarQFull = 0,
-    kBarQFree = 1,
-    kBarSFull = 2,    // 2 slots
-    kBarPFull = 4,
-    kBarPvDone = 5,
-    kBarOFull = 6,
-    kBarOFree = 7,
-    kBarDrain = 8,
-    kBarXFull = 9,    // 4 slots
-    kBarXFree = 13,   // 4 slots
-    kBarKvFull = 17,  // kStages slots
-    kBarKvEmpty = 21, // kStages slots
-    kBarCount = 25
+    kBarQFull = 0,    // leader: Q of both CTAs landed (transaction bytes)
+    kBarQFree = 1,    // both: the chunk's Q K^T MMAs completed
+    kBarKFull = 2,    // leader, 2 stages
+    kBarKEmpty = 4,   // both, 2 stages
+    kBarVFull = 6,    // leader, 2 stages
+    kBarVEmpty = 8,   // both, 2 stages
+    kBarSFull = 10,   // both, 2 S buffers
+    kBarPFull = 12,   // leader, 2 P buffers, 8 warps (4 per CTA)
+    kBarPvDone = 14,  // both, 2 P buffers
+    kBarOFull = 16,   // both
+    kBarOFree = 17,   // leader, 8 warps
+    kBarDrain = 18,   // leader
+    kBarTail = 19,    // both: V load of a sequence's last page (local)
+    kBarPair = 20,    // both: 2 slots, rendezvous of softmax warps {w, w ^ 2} (64 threads)
+    kBarCount = 22
 };
-constexpr int kOffTmemSlot = kBarCount * 8;       // uint32 written by tcgen05.alloc
-constexpr int kOffAbort = kOffTmemSlot + 4;       // int abort flag
+constexpr int kOffTmemSlot = kBarCount * 8;  // uint32 written by tcgen05.alloc
+constexpr int kOffAbort = kOffTmemSlot + 4;  // int abort flag
 
 struct DecodeParams {
     const int32_t* block_table;
@@ -140,10 +144,11 @@ struct Sync {
     // Bounded wait for phase `parity` of `bar`.  Returns false on abort / timeout.
     __device__ bool wait(uint32_t bar, uint32_t parity) const
     {
-        if (mbar_try_wait(bar, parity)) return true;
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         const uint64_t t0 = global_timer_ns();
         while (true) {
-            for (int i = 0; i < 32; ++i)
+            for (int i = 0; i < 256; ++i)
                 if (mbar_try_wait(bar, parity)) return true;
             if (aborted()) return false;
             if (global_timer_ns() - t0 > kWaitTimeoutNs) {
@@ -182,212 +187,273 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, bool fp16)
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ int page_of(const DecodeParams& p, const int32_t* table, int blk)
+{
+    int page = blk < p.max_blocks ? __ldg(table + blk) : -1;
+    if (page < 0 || page >= p.num_blocks) {
+        atomicCAS(p.status, 0, MLA_ERR_DEVICE_CHECK);
+        page = 0;  // keep every load inside the cache; the status word reports the error
+    }
+    return page;
+}
+
 // ------------------------------------------------------------------ split-KV kernel
+// One cluster of two CTAs (an SM pair) per scheduler partition.  CTA c owns
+// query rows [64c, 64c+64) of each 128-row group.  The even CTA issues
+// two-SM tcgen05 MMAs (cta_group::2, M = 128):
+//   S = Q K^T  (N = 64 tokens of a page; CTA c supplies tokens [32c, 32c+32))
+//   O += P V   (N = 256 d_v columns per MMA; CTA c supplies its 128 of them)
+// so each CTA receives the full logits of its own rows without any software
+// exchange, and each KV byte is read from HBM once.
+//
+// Tensor memory of each CTA ("2x2" data-path layout of the pair MMA: lanes
+// 0-63 hold the first half of N for the 64 rows, lanes 64-127 the second):
+//   O   columns [0, 256):  d_v chunk i (256 wide) at [128 i, 128 i + 128)
+//   S   columns [256, 288) and [288, 320): two page buffers
+// Thread t of the softmax warps owns row t % 64 and token / d_v half t / 64.
 template <bool kRope, bool kFp16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    mla_splitkv_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_q64,
-                       const __grid_constant__ CUtensorMap tm_kv128, const __grid_constant__ CUtensorMap tm_kv64,
-                       const DecodeParams p)
+    mla_splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const DecodeParams p)
 {
     using L = Layout<kRope>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_addr(smem);
     const uint32_t s_q = s_base + L::kOffQ;
-    const uint32_t s_kv = s_base + L::kOffKV;
-    const uint32_t s_x = s_base + L::kOffX;
+    const uint32_t s_k = s_base + L::kOffK;
+    const uint32_t s_v = s_base + L::kOffV;
+    const uint32_t s_p = s_base + L::kOffP;
     const uint32_t s_bar = s_base + L::kOffBar;
+    float* red = reinterpret_cast<float*>(smem + L::kOffRed);
     auto bar = [&](int slot) { return s_bar + 8u * slot; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t cta = cluster_cta_rank();
-    const uint32_t peer = cta ^ 1u;
+    const bool leader = (cta == 0);
     const int part = blockIdx.x >> 1;
+    auto lead_bar = [&](int slot) { return map_to_cta(bar(slot), 0); };  // leader's barrier, cluster address
 
     // ---------------- set-up
     if (threadIdx.x == 0) {
         mbar_init(bar(kBarQFull), 1);
         mbar_init(bar(kBarQFree), 1);
-        mbar_init(bar(kBarSFull + 0), 1);
-        mbar_init(bar(kBarSFull + 1), 1);
-        mbar_init(bar(kBarPFull), 4);
-        mbar_init(bar(kBarPvDone), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(kBarKFull + s), 1);
+            mbar_init(bar(kBarKEmpty + s), 1);
+            mbar_init(bar(kBarVFull + s), 1);
+            mbar_init(bar(kBarVEmpty + s), 1);
+            mbar_init(bar(kBarSFull + s), 1);
+            mbar_init(bar(kBarPFull + s), 8);
+            mbar_init(bar(kBarPvDone + s), 1);
+        }
         mbar_init(bar(kBarOFull), 1);
-        mbar_init(bar(kBarOFree), 4);
+        mbar_init(bar(kBarOFree), 8);
         mbar_init(bar(kBarDrain), 1);
-        for (int w = 0; w < 4; ++w) {
-            mbar_init(bar(kBarXFull + w), 1);
-            mbar_init(bar(kBarXFree + w), 32);
-        }
-        for (int s = 0; s < L::kStages; ++s) {
-            mbar_init(bar(kBarKvFull + s), 1);
-            mbar_init(bar(kBarKvEmpty + s), 1);
-        }
+        mbar_init(bar(kBarTail), 1);
+        mbar_init(bar(kBarPair + 0), 64);
+        mbar_init(bar(kBarPair + 1), 64);
         *reinterpret_cast<volatile int*>(smem + L::kOffBar + kOffAbort) = 0;
         fence_mbar_init();
     }
-    // Query rows beyond the loaded box stay zero (finite) for the whole kernel.
-    if (p.box_rows < kRowsPerGroup) {
+    // Query rows past the loaded box stay zero (finite) for the whole kernel.
+    if (p.box_rows < 64) {
         uint4* q4 = reinterpret_cast<uint4*>(smem + L::kOffQ);
         for (int i = threadIdx.x; i < L::kQBytes / 16; i += kThreads) q4[i] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(s_bar + kOffTmemSlot, kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(s_bar + kOffTmemSlot, kTmemCols);
+        tmem_relinquish_pair();
     }
-    if (warp == kTmaWarp && lane == 0) {
-        prefetch_tensormap(&tm_q128);
-        prefetch_tensormap(&tm_kv128);
-        if (kRope) {
-            prefetch_tensormap(&tm_q64);
-            prefetch_tensormap(&tm_kv64);
-        }
+    if (warp == kKWarp && lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
     }
     tc_fence_before();
     __syncthreads();
-    cluster_sync();  // peer barriers initialised before any remote arrive / store
+    cluster_sync();  // both CTAs' barriers initialised before any remote arrive / transaction
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kOffBar + kOffTmemSlot);
 
-    Sync sync{s_bar + kOffAbort, map_to_cta(s_bar + kOffAbort, peer), p.status};
+    Sync sync{s_bar + kOffAbort, map_to_cta(s_bar + kOffAbort, cta ^ 1u), p.status};
     const int32_t* md = p.md + part * kMdInts;
     ChunkIter chunks{md[0], md[1], md[2], md[3], p.groups, p.seqlens};
     const int begin_vb = md[0];
     const int begin_split = md[4];
-    const uint32_t col0 = 256u * cta;          // first latent column of this CTA
-    const uint32_t rope_col = 512u + 32u * cta;
 
-    if (warp == kTmaWarp) {
-        // ============================ TMA producer ============================
+    if (warp == kKWarp) {
+        // ============================ Q and K producer ============================
         if (lane == 0) {
+            const uint32_t q_tx = L::kBoxes * p.box_rows * 128;
             uint32_t g = 0, k = 0;
             int vb, lo, hi;
             bool ok = true;
-            bool q_issued = false;
-            const uint32_t q_tx = p.box_rows * (L::kBoxes * 128 + (kRope ? 64 : 0));
             while (ok && chunks.next(vb, lo, hi)) {
                 if (hi <= lo) continue;
                 const int b = vb / p.groups, rg = vb % p.groups;
                 if (!(ok = sync.wait(bar(kBarQFree), (k & 1) ^ 1))) break;
-                mbar_arrive_expect_tx(bar(kBarQFull), q_tx);
-                q_issued = true;
+                if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * q_tx);
                 for (int i = 0; i < L::kBoxes; ++i)
-                    tma_load_3d(s_q + i * 16384, &tm_q128, bar(kBarQFull), col0 + 64 * i, rg * kRowsPerGroup, b);
-                if (kRope)
-                    tma_load_3d(s_q + L::kBoxes * 16384, &tm_q64, bar(kBarQFull), rope_col, rg * kRowsPerGroup, b);
+                    tma_load_3d_pair(s_q + i * 8192, &tm_q, lead_bar(kBarQFull), 64 * i,
+                                     rg * kRowsPerGroup + 64 * static_cast<int>(cta), b);
                 const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
                 for (int blk = lo; blk < hi; ++blk, ++g) {
-                    const uint32_t st = g % L::kStages;
-                    if (!(ok = sync.wait(bar(kBarKvEmpty + st), ((g / L::kStages) & 1) ^ 1))) break;
-                    int page = blk < p.max_blocks ? __ldg(table + blk) : -1;
-                    if (page < 0 || page >= p.num_blocks) {
-                        atomicCAS(p.status, 0, MLA_ERR_DEVICE_CHECK);
-                        page = 0;  // keep the pipeline in bounds; the status word reports the error
-                    }
-                    const uint32_t dst = s_kv + st * L::kStageBytes;
-                    mbar_arrive_expect_tx(bar(kBarKvFull + st), L::kStageBytes);
+                    const uint32_t st = g & 1;
+                    if (!(ok = sync.wait(bar(kBarKEmpty + st), ((g >> 1) & 1) ^ 1))) break;
+                    const int page = page_of(p, table, blk);
+                    if (leader) mbar_arrive_expect_tx(bar(kBarKFull + st), 2 * L::kKBytes);
+                    const uint32_t dst = s_k + st * L::kKBytes;
                     for (int i = 0; i < L::kBoxes; ++i)
-                        tma_load_2d(dst + i * 8192, &tm_kv128, bar(kBarKvFull + st), col0 + 64 * i, page * kPage);
-                    if (kRope)
-                        tma_load_2d(dst + L::kBoxes * 8192, &tm_kv64, bar(kBarKvFull + st), rope_col, page * kPage);
+                        tma_load_2d_pair(dst + i * 4096, &tm_k, lead_bar(kBarKFull + st), 64 * i,
+                                         page * kPage + 32 * static_cast<int>(cta));
                 }
                 ++k;
             }
             if (!ok) {
-                // Let the loads already issued land before shared memory goes away:
-                // the most recent load into each stage, and the last Q load.
-                const uint64_t t0 = global_timer_ns();
-                for (uint32_t i = 0; i < L::kStages && i < g; ++i) {
-                    const uint32_t gl = g - 1 - i;
-                    while (!mbar_try_wait(bar(kBarKvFull + gl % L::kStages), (gl / L::kStages) & 1) &&
-                           global_timer_ns() - t0 < 100000000ull) {
-                    }
+                const uint64_t t0 = global_timer_ns();  // let issued loads land (see the V producer)
+                while (global_timer_ns() - t0 < 50000000ull) {
                 }
-                if (q_issued) {
-                    const uint32_t kl = k;  // chunk whose Q was issued last
-                    while (!mbar_try_wait(bar(kBarQFull), kl & 1) && global_timer_ns() - t0 < 100000000ull) {
+            }
+        }
+    } else if (warp == kVWarp) {
+        // ============================ V producer ============================
+        // The whole warp waits (uniformly) so that it can zero the rows past the end of a
+        // sequence's last page before the MMA may read them.
+        uint32_t g = 0, tails = 0;
+        int vb, lo, hi;
+        bool ok = true;
+        auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
+        while (ok && chunks.next(vb, lo, hi)) {
+            if (hi <= lo) continue;
+            const int b = vb / p.groups;
+            const int Lb = p.seqlens[b];
+            const int tail = Lb % kPage;
+            const int last_page = pages_of(Lb) - 1;
+            const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+            for (int blk = lo; blk < hi; ++blk, ++g) {
+                const uint32_t st = g & 1;
+                if (!(ok = wwait(bar(kBarVEmpty + st), ((g >> 1) & 1) ^ 1))) break;
+                const int page = page_of(p, table, blk);
+                const uint32_t dst = s_v + st * L::kVBytes;
+                const bool is_tail = (blk == last_page) && tail != 0;
+                if (lane == 0 && leader) mbar_arrive_expect_tx(bar(kBarVFull + st), 2 * L::kVBytes);
+                if (!is_tail) {
+                    if (lane == 0)
+                        for (int i = 0; i < 4; ++i) {
+                            const int box = 4 * (i >> 1) + 2 * static_cast<int>(cta) + (i & 1);
+                            tma_load_2d_pair(dst + i * 8192, &tm_v, lead_bar(kBarVFull + st), 64 * box, page * kPage);
+                        }
+                } else {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(kBarTail), L::kVBytes);
+                        for (int i = 0; i < 4; ++i) {
+                            const int box = 4 * (i >> 1) + 2 * static_cast<int>(cta) + (i & 1);
+                            tma_load_2d(dst + i * 8192, &tm_v, bar(kBarTail), 64 * box, page * kPage);
+                        }
+                    }
+                    if (!(ok = wwait(bar(kBarTail), tails & 1))) break;
+                    ++tails;
+                    // rows [tail, 64) of each of the 4 boxes: contiguous bytes [tail*128, 8192)
+                    const int per_box = (kPage - tail) * 8;  // 16-byte words
+                    for (int i = lane; i < 4 * per_box; i += 32) {
+                        const int box = i / per_box, w16 = i % per_box;
+                        *reinterpret_cast<uint4*>(smem + L::kOffV + st * L::kVBytes + box * 8192 + tail * 128 +
+                                                  w16 * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        fence_acq_rel_cluster();
+                        mbar_complete_tx_cluster(lead_bar(kBarVFull + st), L::kVBytes);
                     }
                 }
             }
         }
+        if (!ok && lane == 0) {
+            // Give loads already issued (they complete on the even CTA's barriers) time
+            // to land before shared memory goes away.
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 50000000ull) {
+            }
+        }
     } else if (warp == kMmaWarp) {
-        // ============================ MMA issuer ============================
-        if (lane == 0) {
+        // ============================ MMA issuer (even CTA) ============================
+        if (lane == 0 && leader) {
             constexpr uint32_t idesc_qk = instr_desc_f16(kFp16, 128, 64, false);
             constexpr uint32_t idesc_pv = instr_desc_f16(kFp16, 128, 256, true);
+            constexpr uint16_t both = 0x3;
             uint32_t g = 0, k = 0;
             int vb, lo, hi;
             bool ok = true;
             auto issue_pv = [&](uint32_t gp, bool first) -> bool {
-                if (!sync.wait(bar(kBarPFull), gp & 1)) return false;
+                const uint32_t pb = gp & 1;
+                if (!sync.wait(bar(kBarPFull + pb), (gp >> 1) & 1)) return false;
                 if (first && !sync.wait(bar(kBarOFree), (k & 1) ^ 1)) return false;
+                if (!sync.wait(bar(kBarVFull + (gp & 1)), (gp >> 1) & 1)) return false;
                 tc_fence_after();
-                const uint32_t st = gp % L::kStages;
-                const uint32_t p_tmem = tmem + kTmemS + 64 * (gp & 1);
-                const uint32_t v_base = s_kv + st * L::kStageBytes;
+                const uint32_t v_base = s_v + (gp & 1) * L::kVBytes;
+                const uint32_t p_base = s_p + pb * L::kPBytes;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    // B = V[16 tokens, 256 columns], MN-major SW128: 64-column groups 8 KB apart
-                    // (LBO), 8-token groups 1 KB apart (SBO).
-                    const uint64_t vdesc = smem_desc(v_base + kk * 2048, 8192, 1024, kLayoutSW128);
-                    mma_ts(tmem + kTmemO, p_tmem + 8 * kk, vdesc, idesc_pv, (first && kk == 0) ? 0u : 1u);
+                for (int i = 0; i < 2; ++i) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        // A = P[64 rows, 16 tokens] K-major; B = V[16 tokens, 128 d_v] of this CTA,
+                        // MN-major: 64-column boxes 8 KB apart (LBO), 8-token groups 1 KB apart (SBO).
+                        const uint64_t pd = smem_desc(p_base + kk * 32, 16, 1024, kLayoutSW128);
+                        const uint64_t vd = smem_desc(v_base + 2 * i * 8192 + kk * 2048, 8192, 1024, kLayoutSW128);
+                        mma_ss_pair(tmem + kTmemO + 128 * i, pd, vd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+                    }
                 }
-                mma_commit(bar(kBarKvEmpty + st));
-                mma_commit(bar(kBarPvDone));
+                mma_commit_pair(bar(kBarVEmpty + (gp & 1)), both);
+                mma_commit_pair(bar(kBarPvDone + pb), both);
                 return true;
             };
             while (ok && chunks.next(vb, lo, hi)) {
                 const int n = hi - lo;
                 if (n <= 0) continue;
                 if (!(ok = sync.wait(bar(kBarQFull), k & 1))) break;
-                tc_fence_after();
                 for (int j = 0; j < n && ok; ++j) {
                     const uint32_t gp = g + j;
-                    const uint32_t st = gp % L::kStages;
-                    if (!(ok = sync.wait(bar(kBarKvFull + st), (gp / L::kStages) & 1))) break;
+                    const uint32_t st = gp & 1;
+                    if (!(ok = sync.wait(bar(kBarKFull + st), (gp >> 1) & 1))) break;
                     tc_fence_after();
-                    const uint32_t s_tmem = tmem + kTmemS + 64 * (gp & 1);
-                    const uint32_t k_base = s_kv + st * L::kStageBytes;
+                    const uint32_t k_base = s_k + st * L::kKBytes;
 #pragma unroll
-                    for (int ks = 0; ks < L::kKSlices; ++ks) {
-                        uint64_t qd, kd;
-                        if (ks < L::kBoxes * 4) {
-                            const int box = ks >> 2, sub = ks & 3;
-                            qd = smem_desc(s_q + box * 16384 + sub * 32, 16, 1024, kLayoutSW128);
-                            kd = smem_desc(k_base + box * 8192 + sub * 32, 16, 1024, kLayoutSW128);
-                        } else {
-                            const int sub = ks - L::kBoxes * 4;
-                            qd = smem_desc(s_q + L::kBoxes * 16384 + sub * 32, 16, 512, kLayoutSW64);
-                            kd = smem_desc(k_base + L::kBoxes * 8192 + sub * 32, 16, 512, kLayoutSW64);
-                        }
-                        mma_ss(s_tmem, qd, kd, idesc_qk, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < L::kKSteps; ++ks) {
+                        const int box = ks >> 2, sub = ks & 3;
+                        const uint64_t qd = smem_desc(s_q + box * 8192 + sub * 32, 16, 1024, kLayoutSW128);
+                        const uint64_t kd = smem_desc(k_base + box * 4096 + sub * 32, 16, 1024, kLayoutSW128);
+                        mma_ss_pair(tmem + kTmemS + 32 * st, qd, kd, idesc_qk, ks > 0 ? 1u : 0u);
                     }
-                    mma_commit(bar(kBarSFull + (gp & 1)));
-                    if (j == n - 1) mma_commit(bar(kBarQFree));
+                    mma_commit_pair(bar(kBarKEmpty + st), both);
+                    mma_commit_pair(bar(kBarSFull + st), both);
+                    if (j == n - 1) mma_commit_pair(bar(kBarQFree), both);
                     if (j > 0) ok = issue_pv(gp - 1, j == 1);
                 }
                 if (ok) ok = issue_pv(g + n - 1, n == 1);
-                if (ok) mma_commit(bar(kBarOFull));
+                if (ok) mma_commit_pair(bar(kBarOFull), both);
                 g += n;
                 ++k;
             }
-            // All issued MMAs complete before tensor memory is released.
-            mma_commit(bar(kBarDrain));
+            // Every issued MMA completes before tensor memory is released.
+            mma_commit_pair(bar(kBarDrain), 0x1);
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(bar(kBarDrain), 0) && global_timer_ns() - t0 < 100000000ull) {
             }
         }
     } else {
         // ======================= softmax / correction / epilogue =======================
-        const int r = threadIdx.x;  // TMEM lane == query row within the row group
+        const int t = threadIdx.x;             // TMEM lane
+        const int r = t & 63;                  // row within this CTA's 64
+        const int h = t >> 6;                  // token half of S, d_v half of each O chunk
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t x_row = s_x + r * 256;
-        const uint32_t x_row_peer = map_to_cta(x_row, peer);
-        const uint32_t x_full_peer = map_to_cta(bar(kBarXFull + warp), peer);
-        const uint32_t x_free_peer = map_to_cta(bar(kBarXFree + warp), peer);
-        // Waits are made warp-uniform: the tcgen05 loads / stores below are warp-collective.
+        const uint32_t pair_bar = bar(kBarPair + (warp & 1));  // rendezvous of warps {w, w ^ 2}
+        uint32_t pair_phase = 0;
+        const uint32_t p_full_lead[2] = {lead_bar(kBarPFull), lead_bar(kBarPFull + 1)};
+        const uint32_t o_free_lead = lead_bar(kBarOFree);
         auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
         uint32_t g = 0, k = 0;
         int vb, lo, hi;
@@ -395,7 +461,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         while (ok && chunks.next(vb, lo, hi)) {
             const int b = vb / p.groups, rg = vb % p.groups;
             const int Lb = p.seqlens[b];
-            const int row = rg * kRowsPerGroup + r;
+            const int row = rg * kRowsPerGroup + 64 * static_cast<int>(cta) + r;
             const bool row_valid = row < p.rows;
             const int s_tok = row / p.h_q;
             int n_vis = Lb;
@@ -403,62 +469,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int nsplit = p.num_splits[vb + 1] - p.num_splits[vb];
             const int split_idx = (vb == begin_vb) ? begin_split : 0;
             const int n = hi - lo;
-            const int last_page = pages_of(Lb) - 1;
-            float m_ref = -INFINITY, l_sum = 0.f;
+            float m_ref = -INFINITY, l_half = 0.f;
 
             for (int j = 0; j < n; ++j) {
                 const uint32_t gp = g + j;
                 const uint32_t sb = gp & 1;
-                const uint32_t s_tmem = tmem + kTmemS + 64 * sb + lane_base;
                 if (!(ok = wwait(bar(kBarSFull + sb), (gp >> 1) & 1))) break;
                 tc_fence_after();
-                float s[64];
+                float x[32];
                 {
-                    uint32_t a[32], c[32];
-                    tmem_ld32(s_tmem, a);
-                    tmem_ld32(s_tmem + 32, c);
+                    uint32_t a[32];
+                    tmem_ld32(tmem + kTmemS + 32 * sb + lane_base, a);
                     tmem_wait_ld();
                     reg_fence(a);
-                    reg_fence(c);
+                    const int lim = n_vis - (lo + j) * kPage - 32 * h;  // columns >= lim are not visible
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        s[i] = __uint_as_float(a[i]);
-                        s[32 + i] = __uint_as_float(c[i]);
-                    }
+                    for (int c = 0; c < 32; ++c) x[c] = (c < lim) ? __uint_as_float(a[c]) * p.scale_log2 : -INFINITY;
                 }
-                // ---- exchange partial logits with the peer CTA
-                if (!(ok = wwait(bar(kBarXFree + warp), (gp & 1) ^ 1))) break;
-                if (lane == 0) mbar_arrive_expect_tx(bar(kBarXFull + warp), 32 * 256);
+                float mx = x[0];
 #pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4) {
-                    const uint32_t off = ((c4 ^ (r & 15)) << 4);
-                    st_async_v4(x_row_peer + off, s[4 * c4], s[4 * c4 + 1], s[4 * c4 + 2], s[4 * c4 + 3],
-                                x_full_peer);
-                }
-                if (!(ok = wwait(bar(kBarXFull + warp), gp & 1))) break;
-#pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4) {
-                    const uint32_t off = ((c4 ^ (r & 15)) << 4);
-                    float4 t;
-                    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                                 : "=f"(t.x), "=f"(t.y), "=f"(t.z), "=f"(t.w)
-                                 : "r"(x_row + off));
-                    s[4 * c4] += t.x;
-                    s[4 * c4 + 1] += t.y;
-                    s[4 * c4 + 2] += t.z;
-                    s[4 * c4 + 3] += t.w;
-                }
-                mbar_arrive_remote(x_free_peer);
-
-                // ---- mask, scale, running maximum
-                const int tok0 = (lo + j) * kPage;
-                const int lim = n_vis - tok0;  // columns >= lim are not visible
-                float mx = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    s[c] = (c < lim) ? s[c] * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, s[c]);
-                }
+                for (int c = 1; c < 32; ++c) mx = fmaxf(mx, x[c]);
+                red[sb * 128 + t] = mx;
+                mbar_arrive(pair_bar);
+                if (!(ok = wwait(pair_bar, pair_phase++ & 1))) break;
+                mx = fmaxf(mx, red[sb * 128 + (t ^ 64)]);
+                // the same decision in both halves of the row
                 float alpha = 1.f;
                 bool rescale = false;
                 if (mx > m_ref + kRescaleThreshold) {
@@ -470,117 +505,127 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
                 float rs = 0.f;
-                uint32_t pk[32];
+                uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float p0 = fast_exp2(s[2 * c] - ref);
-                    const float p1 = fast_exp2(s[2 * c + 1] - ref);
+                for (int c = 0; c < 16; ++c) {
+                    const float p0 = fast_exp2(x[2 * c] - ref);
+                    const float p1 = fast_exp2(x[2 * c + 1] - ref);
                     rs += p0 + p1;
                     pk[c] = pack2(p0, p1, kFp16);
                 }
-                l_sum = l_sum * alpha + rs;
+                l_half = l_half * alpha + rs;
 
-                // ---- previous PV done: P buffer and O are ours
-                if (j > 0 && !(ok = wwait(bar(kBarPvDone), (gp - 1) & 1))) break;
-                tc_fence_after();
                 if (__any_sync(0xffffffffu, rescale)) {
+                    // every earlier PV has completed before O is touched
+                    if (!(ok = wwait(bar(kBarPvDone + ((gp - 1) & 1)), ((gp - 1) >> 1) & 1))) break;
+                    tc_fence_after();
                     const float a = rescale ? alpha : 1.f;
 #pragma unroll 1
-                    for (int cb = 0; cb < kDvHalf / 32; ++cb) {
+                    for (int cb = 0; cb < 8; ++cb) {
                         uint32_t v[32];
-                        tmem_ld32(tmem + kTmemO + lane_base + 32 * cb, v);
+                        const uint32_t addr = tmem + kTmemO + lane_base + 32 * cb;
+                        tmem_ld32(addr, v);
                         tmem_wait_ld();
                         reg_fence(v);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
-                        tmem_st32(tmem + kTmemO + lane_base + 32 * cb, v);
+                        tmem_st32(addr, v);
+                    }
+                    tmem_wait_st();
+                }
+                // P buffer gp&1 was last read by the PV of page gp-2
+                if (gp >= 2 && !(ok = wwait(bar(kBarPvDone + sb), ((gp - 2) >> 1) & 1))) break;
+                {
+                    uint8_t* prow = smem + L::kOffP + sb * L::kPBytes + r * 128;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int chunk = (4 * h + q) ^ (r & 7);
+                        *reinterpret_cast<uint4*>(prow + chunk * 16) =
+                            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                     }
                 }
-                // ---- the sequence's last, partly filled page: zero V rows past the end so
-                //      that whatever the cache holds there cannot reach O through 0 * x.
-                if (lo + j == last_page && (Lb % kPage) != 0) {
-                    const int tail = Lb % kPage;
-                    const uint32_t st = gp % L::kStages;
-                    uint8_t* stage = smem + L::kOffKV + st * L::kStageBytes;
-                    const int per_box = (kPage - tail) * 128 / 16;
-                    for (int i = r; i < per_box * L::kBoxes; i += 128) {
-                        const int box = i / per_box, w16 = i % per_box;
-                        *reinterpret_cast<uint4*>(stage + box * 8192 + tail * 128 + w16 * 16) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                }
-                tmem_st32(s_tmem, pk);
-                tmem_wait_st();
+                fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kBarPFull));
+                if (lane == 0) {
+                    if (leader)
+                        mbar_arrive(bar(kBarPFull + sb));
+                    else
+                        mbar_arrive_remote(p_full_lead[sb]);
+                }
             }
             if (!ok) break;
 
-            // ---- epilogue
+            // ---- epilogue: full row sum from both halves, O / l, LSE
             const bool empty = (n <= 0);
+            red[256 + t] = l_half;
+            mbar_arrive(pair_bar);
+            if (!(ok = wwait(pair_bar, pair_phase++ & 1))) break;
+            const float l_other = red[256 + (t ^ 64)];
+            const float l_sum = (h == 0) ? (l_half + l_other) : (l_other + l_half);
+            mbar_arrive(pair_bar);  // red[256..] free for the next chunk once both have read it
+            if (!(ok = wwait(pair_bar, pair_phase++ & 1))) break;
             const float inv_l = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
             const float lse_v = (l_sum > 0.f) ? (m_ref + log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
             if (!empty) {
                 if (!(ok = wwait(bar(kBarOFull), k & 1))) break;
                 tc_fence_after();
             }
-            if (nsplit == 1) {
-                typedef uint4 vec_t;
-                vec_t* dst = reinterpret_cast<vec_t*>(static_cast<uint8_t*>(p.o) +
-                                                      ((static_cast<size_t>(b) * p.rows + row) * kDv + col0) * 2);
 #pragma unroll 1
-                for (int cb = 0; cb < kDvHalf / 32; ++cb) {
+            for (int i = 0; i < 2; ++i) {
+                const int col0 = 256 * i + 128 * h;  // first d_v column this thread holds in chunk i
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
                     uint32_t v[32];
                     if (!empty) {
-                        tmem_ld32(tmem + kTmemO + lane_base + 32 * cb, v);
+                        tmem_ld32(tmem + kTmemO + 128 * i + lane_base + 32 * cb, v);
                         tmem_wait_ld();
                         reg_fence(v);
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0;
+                        for (int e = 0; e < 32; ++e) v[e] = 0;
                     }
-                    uint32_t h[16];
+                    if (!row_valid) continue;
+                    if (nsplit == 1) {
+                        uint4* dst = reinterpret_cast<uint4*>(
+                            static_cast<uint8_t*>(p.o) +
+                            ((static_cast<size_t>(b) * p.rows + row) * kDv + col0 + 32 * cb) * 2);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        h[i] = pack2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l, kFp16);
-                    if (row_valid) {
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[cb * 4 + i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
-                    }
-                }
-                if (cta == 0 && row_valid) p.lse[static_cast<size_t>(b) * p.rows + row] = lse_v;
-            } else {
-                const size_t slot = static_cast<size_t>(p.num_splits[vb]) + split_idx;
-                float4* dst = reinterpret_cast<float4*>(p.o_accum + (slot * kRowsPerGroup + r) * kDv + col0);
-#pragma unroll 1
-                for (int cb = 0; cb < kDvHalf / 32; ++cb) {
-                    uint32_t v[32];
-                    if (!empty) {
-                        tmem_ld32(tmem + kTmemO + lane_base + 32 * cb, v);
-                        tmem_wait_ld();
-                        reg_fence(v);
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(
+                                pack2(__uint_as_float(v[8 * e + 0]) * inv_l, __uint_as_float(v[8 * e + 1]) * inv_l, kFp16),
+                                pack2(__uint_as_float(v[8 * e + 2]) * inv_l, __uint_as_float(v[8 * e + 3]) * inv_l, kFp16),
+                                pack2(__uint_as_float(v[8 * e + 4]) * inv_l, __uint_as_float(v[8 * e + 5]) * inv_l, kFp16),
+                                pack2(__uint_as_float(v[8 * e + 6]) * inv_l, __uint_as_float(v[8 * e + 7]) * inv_l, kFp16));
                     } else {
+                        const size_t slot = static_cast<size_t>(p.num_splits[vb]) + split_idx;
+                        float4* dst = reinterpret_cast<float4*>(
+                            p.o_accum + (slot * kRowsPerGroup + 64 * cta + r) * kDv + col0 + 32 * cb);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0;
-                    }
-                    if (row_valid) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[cb * 8 + i] = make_float4(__uint_as_float(v[4 * i]) * inv_l,
-                                                          __uint_as_float(v[4 * i + 1]) * inv_l,
-                                                          __uint_as_float(v[4 * i + 2]) * inv_l,
-                                                          __uint_as_float(v[4 * i + 3]) * inv_l);
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv_l, __uint_as_float(v[4 * e + 1]) * inv_l,
+                                                 __uint_as_float(v[4 * e + 2]) * inv_l,
+                                                 __uint_as_float(v[4 * e + 3]) * inv_l);
                     }
                 }
-                if (cta == 0) p.lse_accum[slot * kRowsPerGroup + r] = lse_v;
+            }
+            if (h == 0) {
+                if (nsplit == 1) {
+                    if (row_valid) p.lse[static_cast<size_t>(b) * p.rows + row] = lse_v;
+                } else {
+                    const size_t slot = static_cast<size_t>(p.num_splits[vb]) + split_idx;
+                    p.lse_accum[slot * kRowsPerGroup + 64 * cta + r] = lse_v;
+                }
             }
             if (!empty) {
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kBarOFree));
+                if (lane == 0) {
+                    if (leader)
+                        mbar_arrive(bar(kBarOFree));
+                    else
+                        mbar_arrive_remote(o_free_lead);
+                }
                 ++k;
             }
             g += (n > 0 ? n : 0);
@@ -590,10 +635,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ---------------- teardown
     tc_fence_before();
     __syncthreads();
-    cluster_sync();  // no remote access to this CTA's shared memory after this point
+    cluster_sync();  // no remote access to this CTA and no MMA in flight after this point
     if (warp == kMmaWarp) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc_pair(tmem, kTmemCols);
     }
 }
 
@@ -715,12 +760,11 @@ static size_t workspace_slots(int batch, int groups, int num_parts)
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 template <bool kRope, bool kFp16>
-static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorMap& q128, const CUtensorMap& q64,
-                                  const CUtensorMap& kv128, const CUtensorMap& kv64, const DecodeParams& prm)
+static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorMap* maps, const DecodeParams& prm)
 {
     auto kern = mla_splitkv_kernel<kRope, kFp16>;
     const int smem = Layout<kRope>::kSmemBytes;
-    static int configured_device = -1;  // attribute is per device; set it once per device in use
+    static int configured_device = -1;  // the attribute is per device; set it once per device in use
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -729,7 +773,7 @@ static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorM
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    kern<<<grid, kThreads, smem, stream>>>(q128, q64, kv128, kv64, prm);
+    kern<<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], prm);
     return cudaGetLastError();
 }
 
@@ -853,7 +897,7 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     prm.max_blocks = max_blocks_per_seq;
     prm.num_blocks = num_blocks;
     prm.causal = causal;
-    prm.box_rows = rows < kRowsPerGroup ? rows : kRowsPerGroup;
+    prm.box_rows = rows < 64 ? rows : 64;  // query rows per CTA of the pair
     prm.scale_log2 = softmax_scale * 1.4426950408889634f;
     prm.dtype = dtype;
     prm.d_qk = d_qk;
@@ -870,17 +914,14 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
         dtype == MLA_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const uint64_t row_bytes = static_cast<uint64_t>(d_qk) * 2;
     const uint64_t kv_rows = static_cast<uint64_t>(num_blocks) * kPage;
-    bool ok = encode_3d(&maps[0], q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 64, prm.box_rows,
-                        CU_TENSOR_MAP_SWIZZLE_128B) &&
-              encode_2d(&maps[2], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (ok && d_qk == 576)
-        ok = encode_3d(&maps[1], q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 32, prm.box_rows,
-                       CU_TENSOR_MAP_SWIZZLE_64B) &&
-             encode_2d(&maps[3], kvcache, dt, d_qk, kv_rows, row_bytes, 32, kPage, CU_TENSOR_MAP_SWIZZLE_64B);
-    else {
-        maps[1] = maps[0];
-        maps[3] = maps[2];
-    }
+    // Q: [batch][rows][d_qk], box 64 columns x (up to) 64 rows;
+    // K: cache rows, box 64 columns x 32 tokens (half a page, one CTA's share);
+    // V: cache rows, box 64 columns x 64 tokens (a page).
+    const bool ok =
+        encode_3d(&maps[0], q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 64, prm.box_rows,
+                  CU_TENSOR_MAP_SWIZZLE_128B) &&
+        encode_2d(&maps[1], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage / 2, CU_TENSOR_MAP_SWIZZLE_128B) &&
+        encode_2d(&maps[2], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B);
     return ok ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -889,11 +930,11 @@ static mla_status launch_splitkv_stage(const DecodeParams& prm, const CUtensorMa
     const int grid = 2 * prm.num_parts;
     cudaError_t e;
     if (prm.d_qk == 576)
-        e = prm.dtype == MLA_FP16 ? launch_splitkv<true, true>(grid, st, maps[0], maps[1], maps[2], maps[3], prm)
-                                  : launch_splitkv<true, false>(grid, st, maps[0], maps[1], maps[2], maps[3], prm);
+        e = prm.dtype == MLA_FP16 ? launch_splitkv<true, true>(grid, st, maps, prm)
+                                  : launch_splitkv<true, false>(grid, st, maps, prm);
     else
-        e = prm.dtype == MLA_FP16 ? launch_splitkv<false, true>(grid, st, maps[0], maps[1], maps[2], maps[3], prm)
-                                  : launch_splitkv<false, false>(grid, st, maps[0], maps[1], maps[2], maps[3], prm);
+        e = prm.dtype == MLA_FP16 ? launch_splitkv<false, true>(grid, st, maps, prm)
+                                  : launch_splitkv<false, false>(grid, st, maps, prm);
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -920,7 +961,7 @@ mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, int h_q, i
                                    size_t workspace_bytes, void* stream)
 {
     DecodeParams prm;
-    CUtensorMap maps[4];
+    CUtensorMap maps[3];
     mla_status s = prepare_decode(MLA_DECODE_ARGS, prm, maps);
     if (s != MLA_OK || batch == 0) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -937,7 +978,7 @@ mla_status mla_decode_splitkv(const void* q, int batch, int s_q, int h_q, int d_
                               void* stream)
 {
     DecodeParams prm;
-    CUtensorMap maps[4];
+    CUtensorMap maps[3];
     mla_status s = prepare_decode(MLA_DECODE_ARGS, prm, maps);
     if (s != MLA_OK || batch == 0) return s;
     return launch_splitkv_stage(prm, maps, static_cast<cudaStream_t>(stream));
