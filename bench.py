@@ -10,8 +10,8 @@ decode workloads are timed in the same run and reported under "workloads".
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronisation; each step is timed on the launching stream with CUDA
-events around each kernel; L2 is flushed between steps (a write of 2 x L2),
-outside the events.  For N > 1 GPUs each rank runs an independent replica
+events around each kernel (each kernel replays its own captured CUDA graph);
+L2 is flushed between steps (a write of 2 x L2), outside the events.  For N > 1 GPUs each rank runs an independent replica
 (the path needs no collective) and rank 0 reports the maximum step time over
 ranks.
 
@@ -175,7 +175,11 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- GPU arm
 class Runner:
-    """Device tensors and the three launches of one decode step for one workload."""
+    """Device tensors and the three launches of one decode step for one workload.
+
+    Each launch is captured once in its own CUDA graph, so replaying a step costs
+    the host a few microseconds and the GPU never waits for Python between kernels.
+    """
 
     def __init__(self, torch, mla, p: W.Problem, dev):
         self.torch, self.mla, self.p, self.dev = torch, mla, p, dev
@@ -194,19 +198,33 @@ class Runner:
         self.call = mla.DecodeCall(self.q, self.kv, self.bt, self.sl, p.dv, self.md, self.ns, causal=p.causal,
                                    softmax_scale=p.scale, workspace=ws)
         self.launches_per_step = 3
+        stages = [lambda: mla.get_mla_metadata(self.sl, self.rows, 1, out=(self.md, self.ns)),
+                  self.call.splitkv, self.call.combine]
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            for _ in range(2):
+                for f in stages:
+                    f()
+        torch.cuda.current_stream(dev).wait_stream(s)
+        torch.cuda.synchronize(dev)
+        self.graphs = []
+        for f in stages:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                f()
+            self.graphs.append(g)
+        torch.cuda.synchronize(dev)
 
     def step(self, ev=None):
-        if ev is not None:
-            ev[0].record()
-        self.mla.get_mla_metadata(self.sl, self.rows, 1, out=(self.md, self.ns))
-        if ev is not None:
-            ev[1].record()
-        self.call.splitkv()
-        if ev is not None:
-            ev[2].record()
-        self.call.combine()
-        if ev is not None:
-            ev[3].record()
+        if ev is None:
+            for g in self.graphs:
+                g.replay()
+            return
+        ev[0].record()
+        for i, g in enumerate(self.graphs):
+            g.replay()
+            ev[i + 1].record()
 
     def status(self):
         return self.mla.read_device_status(self.call.workspace, clear=True)

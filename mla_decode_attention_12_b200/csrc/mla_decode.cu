@@ -80,9 +80,10 @@ struct Layout {
     static constexpr int kOffK = kOffQ + kQBytes;              // 2 stages
     static constexpr int kOffV = kOffK + 2 * kKBytes;          // 2 stages
     static constexpr int kOffP = kOffV + 2 * kVBytes;          // 2 buffers
-    static constexpr int kOffRed = kOffP + 2 * kPBytes;        // 2 x 128 floats: row max / sum halves
-    static constexpr int kOffBar = kOffRed + 1024;
-    static constexpr int kBarBytes = 512;
+    static constexpr int kOffRed = kOffP + 2 * kPBytes;        // 3 x 128 floats: 2 page row-max halves, row sums
+    static constexpr int kRedBytes = 3 * 128 * 4;
+    static constexpr int kOffBar = kOffRed + kRedBytes;
+    static constexpr int kBarBytes = 256;
     static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
 };
 
@@ -105,6 +106,13 @@ enum BarSlot : int {
 };
 constexpr int kOffTmemSlot = kBarCount * 8;  // uint32 written by tcgen05.alloc
 constexpr int kOffAbort = kOffTmemSlot + 4;  // int abort flag
+static_assert(kOffAbort + 4 <= Layout<true>::kBarBytes, "barrier area too small");
+static_assert(Layout<true>::kSmemBytes <= 232448 && Layout<false>::kSmemBytes <= 232448,
+              "shared memory plan exceeds 227 KB");
+static_assert(Layout<true>::kOffQ % 1024 == 0 && Layout<true>::kOffK % 1024 == 0 && Layout<true>::kOffV % 1024 == 0 &&
+                  Layout<true>::kOffP % 1024 == 0 && Layout<false>::kOffK % 1024 == 0 &&
+                  Layout<false>::kOffV % 1024 == 0 && Layout<false>::kOffP % 1024 == 0,
+              "swizzled operand tiles must be 1024-byte aligned");
 
 struct DecodeParams {
     const int32_t* block_table;
@@ -381,68 +389,87 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ============================ MMA issuer (even CTA) ============================
-        if (lane == 0 && leader) {
+        // The whole warp runs the loop (so addresses and descriptors stay warp-uniform);
+        // one elected lane issues each tcgen05 instruction.
+        if (leader) {
             constexpr uint32_t idesc_qk = instr_desc_f16(kFp16, 128, 64, false);
             constexpr uint32_t idesc_pv = instr_desc_f16(kFp16, 128, 256, true);
             constexpr uint16_t both = 0x3;
+            // Base descriptors; a K step or a stage moves the start address, which is
+            // the low field of the descriptor (address >> 4).
+            const uint64_t q_desc = smem_desc(s_q, 16, 1024, kLayoutSW128);
+            const uint64_t k_desc = smem_desc(s_k, 16, 1024, kLayoutSW128);
+            const uint64_t p_desc = smem_desc(s_p, 16, 1024, kLayoutSW128);
+            const uint64_t v_desc = smem_desc(s_v, 8192, 1024, kLayoutSW128);
+            const bool issuer = elect_one();
+            auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
             uint32_t g = 0, k = 0;
             int vb, lo, hi;
             bool ok = true;
             auto issue_pv = [&](uint32_t gp, bool first) -> bool {
                 const uint32_t pb = gp & 1;
-                if (!sync.wait(bar(kBarPFull + pb), (gp >> 1) & 1)) return false;
-                if (first && !sync.wait(bar(kBarOFree), (k & 1) ^ 1)) return false;
-                if (!sync.wait(bar(kBarVFull + (gp & 1)), (gp >> 1) & 1)) return false;
+                if (!wwait(bar(kBarPFull + pb), (gp >> 1) & 1)) return false;
+                if (first && !wwait(bar(kBarOFree), (k & 1) ^ 1)) return false;
+                if (!wwait(bar(kBarVFull + pb), (gp >> 1) & 1)) return false;
                 tc_fence_after();
-                const uint32_t v_base = s_v + (gp & 1) * L::kVBytes;
-                const uint32_t p_base = s_p + pb * L::kPBytes;
+                if (issuer) {
+                    const uint64_t pd0 = p_desc + ((pb * L::kPBytes) >> 4);
+                    const uint64_t vd0 = v_desc + ((pb * L::kVBytes) >> 4);
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
+                    for (int i = 0; i < 2; ++i) {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        // A = P[64 rows, 16 tokens] K-major; B = V[16 tokens, 128 d_v] of this CTA,
-                        // MN-major: 64-column boxes 8 KB apart (LBO), 8-token groups 1 KB apart (SBO).
-                        const uint64_t pd = smem_desc(p_base + kk * 32, 16, 1024, kLayoutSW128);
-                        const uint64_t vd = smem_desc(v_base + 2 * i * 8192 + kk * 2048, 8192, 1024, kLayoutSW128);
-                        mma_ss_pair(tmem + kTmemO + 128 * i, pd, vd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            // A = P[64 rows, 16 tokens] K-major; B = V[16 tokens, 128 d_v] of this CTA,
+                            // MN-major: 64-column boxes 8 KB apart (LBO), 8-token groups 1 KB apart (SBO).
+                            mma_ss_pair(tmem + kTmemO + 128 * i, pd0 + ((kk * 32) >> 4),
+                                        vd0 + ((2 * i * 8192 + kk * 2048) >> 4), idesc_pv,
+                                        (first && kk == 0) ? 0u : 1u);
+                        }
                     }
+                    mma_commit_pair(bar(kBarVEmpty + pb), both);
+                    mma_commit_pair(bar(kBarPvDone + pb), both);
                 }
-                mma_commit_pair(bar(kBarVEmpty + (gp & 1)), both);
-                mma_commit_pair(bar(kBarPvDone + pb), both);
+                __syncwarp();
                 return true;
             };
             while (ok && chunks.next(vb, lo, hi)) {
                 const int n = hi - lo;
                 if (n <= 0) continue;
-                if (!(ok = sync.wait(bar(kBarQFull), k & 1))) break;
+                if (!(ok = wwait(bar(kBarQFull), k & 1))) break;
                 for (int j = 0; j < n && ok; ++j) {
                     const uint32_t gp = g + j;
                     const uint32_t st = gp & 1;
-                    if (!(ok = sync.wait(bar(kBarKFull + st), (gp >> 1) & 1))) break;
+                    if (!(ok = wwait(bar(kBarKFull + st), (gp >> 1) & 1))) break;
                     tc_fence_after();
-                    const uint32_t k_base = s_k + st * L::kKBytes;
+                    if (issuer) {
+                        const uint64_t kd0 = k_desc + ((st * L::kKBytes) >> 4);
 #pragma unroll
-                    for (int ks = 0; ks < L::kKSteps; ++ks) {
-                        const int box = ks >> 2, sub = ks & 3;
-                        const uint64_t qd = smem_desc(s_q + box * 8192 + sub * 32, 16, 1024, kLayoutSW128);
-                        const uint64_t kd = smem_desc(k_base + box * 4096 + sub * 32, 16, 1024, kLayoutSW128);
-                        mma_ss_pair(tmem + kTmemS + 32 * st, qd, kd, idesc_qk, ks > 0 ? 1u : 0u);
+                        for (int ks = 0; ks < L::kKSteps; ++ks) {
+                            const int box = ks >> 2, sub = ks & 3;
+                            mma_ss_pair(tmem + kTmemS + 32 * st, q_desc + ((box * 8192 + sub * 32) >> 4),
+                                        kd0 + ((box * 4096 + sub * 32) >> 4), idesc_qk, ks > 0 ? 1u : 0u);
+                        }
+                        mma_commit_pair(bar(kBarKEmpty + st), both);
+                        mma_commit_pair(bar(kBarSFull + st), both);
+                        if (j == n - 1) mma_commit_pair(bar(kBarQFree), both);
                     }
-                    mma_commit_pair(bar(kBarKEmpty + st), both);
-                    mma_commit_pair(bar(kBarSFull + st), both);
-                    if (j == n - 1) mma_commit_pair(bar(kBarQFree), both);
+                    __syncwarp();
                     if (j > 0) ok = issue_pv(gp - 1, j == 1);
                 }
                 if (ok) ok = issue_pv(g + n - 1, n == 1);
-                if (ok) mma_commit_pair(bar(kBarOFull), both);
+                if (ok && issuer) mma_commit_pair(bar(kBarOFull), both);
+                __syncwarp();
                 g += n;
                 ++k;
             }
             // Every issued MMA completes before tensor memory is released.
-            mma_commit_pair(bar(kBarDrain), 0x1);
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(bar(kBarDrain), 0) && global_timer_ns() - t0 < 100000000ull) {
+            if (issuer) {
+                mma_commit_pair(bar(kBarDrain), 0x1);
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(bar(kBarDrain), 0) && global_timer_ns() - t0 < 100000000ull) {
+                }
             }
+            __syncwarp();
         }
     } else {
         // ======================= softmax / correction / epilogue =======================
