@@ -48,6 +48,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
+#include <vector>
 
 #include "../../include/mla_decode.h"
 #include "ptx.cuh"
@@ -671,66 +672,155 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ combine kernel
 // Merges the split partial results of every virtual batch with more than one
-// split: lse = log sum_k exp(lse_k), o = sum_k exp(lse_k - lse) o_k.  One warp
-// per query row; lane i owns 16 of the 512 output columns.
+// split: lse = log sum_k exp(lse_k), o = sum_k exp(lse_k - lse) o_k (the exact
+// identity behind split-KV).  One warp per query row, 4 rows per CTA; lane i
+// owns 16 of the 512 output columns; the split weights are computed 32 at a
+// time (one per lane) and broadcast with shuffles.
 template <bool kFp16>
-__global__ void __launch_bounds__(256) mla_combine_kernel(DecodeParams p)
+__global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
 {
     const int vb = blockIdx.x;
-    const int nsplit = p.num_splits[vb + 1] - p.num_splits[vb];
+    const int slot0 = p.num_splits[vb];
+    const int nsplit = p.num_splits[vb + 1] - slot0;
     if (nsplit <= 1) return;
     const int b = vb / p.groups, rg = vb % p.groups;
-    const int slot0 = p.num_splits[vb];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = blockIdx.y * 4 + warp;
     const int rows_here = min(kRowsPerGroup, p.rows - rg * kRowsPerGroup);
-    for (int r = blockIdx.y * 8 + warp; r < rows_here; r += gridDim.y * 8) {
-        float mx = -INFINITY;
-        for (int k = lane; k < nsplit; k += 32) mx = fmaxf(mx, p.lse_accum[(size_t)(slot0 + k) * kRowsPerGroup + r]);
+    if (r >= rows_here) return;
+    const float* lse_k = p.lse_accum + static_cast<size_t>(slot0) * kRowsPerGroup + r;
+    float mx = -INFINITY;
+    for (int k = lane; k < nsplit; k += 32) mx = fmaxf(mx, lse_k[static_cast<size_t>(k) * kRowsPerGroup]);
 #pragma unroll
-        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        float sum = 0.f;
-        if (mx != -INFINITY)
-            for (int k = lane; k < nsplit; k += 32)
-                sum += expf(p.lse_accum[(size_t)(slot0 + k) * kRowsPerGroup + r] - mx);
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.f;
+    if (mx != -INFINITY)
+        for (int k = lane; k < nsplit; k += 32) sum += expf(lse_k[static_cast<size_t>(k) * kRowsPerGroup] - mx);
 #pragma unroll
-        for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        const float lse = (mx == -INFINITY) ? -INFINITY : mx + logf(sum);
-        float acc[16];
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float lse = (mx == -INFINITY) ? -INFINITY : mx + logf(sum);
+    float acc[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-        if (mx != -INFINITY) {
-            for (int k = 0; k < nsplit; ++k) {
-                const float w = expf(p.lse_accum[(size_t)(slot0 + k) * kRowsPerGroup + r] - lse);
-                if (w == 0.f) continue;
-                const float4* src =
-                    reinterpret_cast<const float4*>(p.o_accum + ((size_t)(slot0 + k) * kRowsPerGroup + r) * kDv);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 v = src[lane + 32 * i];
-                    acc[4 * i] += w * v.x;
-                    acc[4 * i + 1] += w * v.y;
-                    acc[4 * i + 2] += w * v.z;
-                    acc[4 * i + 3] += w * v.w;
-                }
+    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    if (mx != -INFINITY) {
+        const float4* src = reinterpret_cast<const float4*>(p.o_accum + (static_cast<size_t>(slot0) * kRowsPerGroup + r) * kDv) + lane;
+        const size_t stride4 = static_cast<size_t>(kRowsPerGroup) * kDv / 4;  // float4s between splits
+        for (int kb = 0; kb < nsplit; kb += 32) {
+            const int k = kb + lane;
+            const float w_mine = (k < nsplit) ? expf(lse_k[static_cast<size_t>(k) * kRowsPerGroup] - lse) : 0.f;
+            const int cnt = min(32, nsplit - kb);
+#pragma unroll 4
+            for (int kk = 0; kk < cnt; ++kk) {
+                const float w = __shfl_sync(0xffffffffu, w_mine, kk);
+                const float4* s4 = src + static_cast<size_t>(kb + kk) * stride4;
+                const float4 v0 = s4[0], v1 = s4[32], v2 = s4[64], v3 = s4[96];
+                acc[0] += w * v0.x; acc[1] += w * v0.y; acc[2] += w * v0.z; acc[3] += w * v0.w;
+                acc[4] += w * v1.x; acc[5] += w * v1.y; acc[6] += w * v1.z; acc[7] += w * v1.w;
+                acc[8] += w * v2.x; acc[9] += w * v2.y; acc[10] += w * v2.z; acc[11] += w * v2.w;
+                acc[12] += w * v3.x; acc[13] += w * v3.y; acc[14] += w * v3.z; acc[15] += w * v3.w;
             }
         }
-        const int row = rg * kRowsPerGroup + r;
-        uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.o) + ((size_t)b * p.rows + row) * kDv * 2);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            dst[lane + 32 * i] = make_uint2(pack2(acc[4 * i], acc[4 * i + 1], kFp16), pack2(acc[4 * i + 2], acc[4 * i + 3], kFp16));
-        if (lane == 0) p.lse[(size_t)b * p.rows + row] = lse;
     }
+    const int row = rg * kRowsPerGroup + r;
+    uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.o) + (static_cast<size_t>(b) * p.rows + row) * kDv * 2);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        dst[lane + 32 * i] = make_uint2(pack2(acc[4 * i], acc[4 * i + 1], kFp16), pack2(acc[4 * i + 2], acc[4 * i + 3], kFp16));
+    if (lane == 0) p.lse[static_cast<size_t>(b) * p.rows + row] = lse;
 }
 
 // ------------------------------------------------------------------ metadata kernel
-__global__ void mla_metadata_kernel(const int32_t* seqlens, int batch, int groups, int num_parts, int32_t* md,
-                                    int32_t* num_splits, int32_t* scratch_unused)
+// Exclusive prefix sum over n values held in shared memory, by one CTA.
+template <typename T>
+__device__ void block_exclusive_scan(T* data, int n, T* warp_tot, T& total)
 {
-    extern __shared__ int32_t s_len[];
-    for (int i = threadIdx.x; i < batch; i += blockDim.x) s_len[i] = seqlens[i];
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int per = (n + nt - 1) / nt;
+    const int lo = min(n, tid * per), hi = min(n, lo + per);
+    T local = 0;
+    for (int i = lo; i < hi; ++i) local += data[i];
+    // inclusive scan of the per-thread sums across the block
+    T x = local;
+    const int lane = tid & 31, w = tid >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const T y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[w] = x;
     __syncthreads();
-    if (threadIdx.x == 0) schedule(s_len, batch, groups, num_parts, md, num_splits);
+    if (w == 0) {
+        T t = (lane < (nt >> 5)) ? warp_tot[lane] : T(0);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const T y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        if (lane < (nt >> 5)) warp_tot[lane] = t;
+    }
+    __syncthreads();
+    T run = x - local + (w > 0 ? warp_tot[w - 1] : T(0));
+    total = warp_tot[(nt >> 5) - 1];
+    for (int i = lo; i < hi; ++i) {
+        const T v = data[i];
+        data[i] = run;
+        run += v;
+    }
+    __syncthreads();
+}
+
+// One CTA of kMetaThreads threads.  Dynamic shared memory: C [nv] int64,
+// pages [nv] int32, extra-split counts [nv] int32, begins [num_parts] int32 x 2.
+constexpr int kMetaThreads = 1024;
+
+__global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_t* seqlens, int batch, int groups,
+                                                                    int num_parts, int32_t* md, int32_t* num_splits)
+{
+    extern __shared__ __align__(16) uint8_t meta_smem[];
+    __shared__ long long warp_tot_ll[32];
+    __shared__ int warp_tot_i[32];
+    const int nv = batch * groups;
+    long long* C = reinterpret_cast<long long*>(meta_smem);
+    int32_t* pages = reinterpret_cast<int32_t*>(C + nv);
+    int32_t* extra = pages + nv;
+    int32_t* begins = extra + nv;  // [num_parts][2]
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+        pages[v] = pages_of(seqlens[v / groups]);
+        C[v] = pages[v] + kFixedCost;
+        extra[v] = 0;
+    }
+    __syncthreads();
+    long long total = 0;
+    block_exclusive_scan(C, nv, warp_tot_ll, total);
+    for (int p = threadIdx.x; p < num_parts; p += blockDim.x) {
+        int32_t m[kMdInts];
+        partition_range(p, num_parts, C, pages, nv, total, m);
+        begins[2 * p] = m[0];
+        begins[2 * p + 1] = m[1];
+        for (int i = 0; i < kMdInts; ++i) md[p * kMdInts + i] = m[i];
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < num_parts; p += blockDim.x) {
+        const int bv = begins[2 * p], bb = begins[2 * p + 1];
+        if (bb > 0) {
+            int idx = 1;
+            for (int q = p - 1; q >= 0 && begins[2 * q] == bv && begins[2 * q + 1] > 0; --q) ++idx;
+            md[p * kMdInts + 4] = idx;
+            atomicAdd(&extra[bv], 1);
+        }
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) extra[v] += 1;  // splits of vb
+    __syncthreads();
+    int nsplit_total = 0;
+    block_exclusive_scan(extra, nv, warp_tot_i, nsplit_total);
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) num_splits[v] = extra[v];
+    if (threadIdx.x == 0) num_splits[nv] = nsplit_total;
+}
+
+static size_t metadata_smem_bytes(int nv, int num_parts)
+{
+    return static_cast<size_t>(nv) * (8 + 4 + 4) + static_cast<size_t>(num_parts) * 8 + 16;
 }
 
 // ------------------------------------------------------------------ host side
@@ -855,7 +945,11 @@ mla_status mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int he
     if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
     for (int b = 0; b < batch; ++b)
         if (cache_seqlens[b] < 0) return MLA_ERR_INVALID_ARG;
-    schedule(cache_seqlens, batch, row_groups(heads_per_kv), num_parts, tile_md, num_splits);
+    const int groups = row_groups(heads_per_kv);
+    const size_t nv = static_cast<size_t>(batch) * groups;
+    std::vector<long long> C(nv + 1);
+    std::vector<int32_t> pages(nv + 1);
+    schedule_host(cache_seqlens, batch, groups, num_parts, tile_md, num_splits, C.data(), pages.data());
     return MLA_OK;
 }
 
@@ -866,10 +960,22 @@ mla_status mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_p
         (batch > 0 && !cache_seqlens))
         return MLA_ERR_INVALID_ARG;
     if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
-    if (batch > 12000) return MLA_ERR_UNSUPPORTED;  // sequence lengths are staged in shared memory
-    mla_metadata_kernel<<<1, 256, static_cast<size_t>(batch) * sizeof(int32_t) + 16,
-                          static_cast<cudaStream_t>(stream)>>>(cache_seqlens, batch, row_groups(heads_per_kv),
-                                                               num_parts, tile_md, num_splits, nullptr);
+    const int nv = batch * row_groups(heads_per_kv);
+    const size_t smem = metadata_smem_bytes(nv, num_parts);
+    if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;  // the schedule is built in one CTA's shared memory
+    if (smem > 48 * 1024) {
+        static int configured_device = -1;
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+        if (configured_device != dev) {
+            if (cudaFuncSetAttribute(mla_metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+                cudaSuccess)
+                return MLA_ERR_CUDA;
+            configured_device = dev;
+        }
+    }
+    mla_metadata_kernel<<<1, kMetaThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+        cache_seqlens, batch, row_groups(heads_per_kv), num_parts, tile_md, num_splits);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -967,11 +1073,12 @@ static mla_status launch_splitkv_stage(const DecodeParams& prm, const CUtensorMa
 
 static mla_status launch_combine_stage(const DecodeParams& prm, cudaStream_t st)
 {
-    dim3 cgrid(prm.batch * prm.groups, 4);
+    const int rows_max = prm.rows < kRowsPerGroup ? prm.rows : kRowsPerGroup;
+    dim3 cgrid(prm.batch * prm.groups, (rows_max + 3) / 4);
     if (prm.dtype == MLA_FP16)
-        mla_combine_kernel<true><<<cgrid, 256, 0, st>>>(prm);
+        mla_combine_kernel<true><<<cgrid, 128, 0, st>>>(prm);
     else
-        mla_combine_kernel<false><<<cgrid, 256, 0, st>>>(prm);
+        mla_combine_kernel<false><<<cgrid, 128, 0, st>>>(prm);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

@@ -1,5 +1,5 @@
 // Tile scheduler: splits the decode work of a batch into `num_parts` contiguous
-// ranges of nearly equal cost, one per two-SM cluster of the split-KV kernel.
+// ranges of equal cost, one per two-SM cluster of the split-KV kernel.
 //
 // "FlashMLA" usage page (deepep.org): get_mla_metadata analyses the sequence
 // lengths once per decoding step and returns tile_scheduler_metadata and
@@ -9,13 +9,16 @@
 // print the algorithm or the metadata format; this one is our own.
 //
 // Work units.  A "virtual batch" vb = b * row_groups + g is request b restricted
-// to query rows [128 g, 128 g + 128) of its s_q * h_q rows.  Its cost is its
-// page count ceil(L_b / 64) plus kFixedCost pages of per-chunk overhead (Q load,
-// epilogue).  Walking the virtual batches in order, each partition takes
-// budget T = ceil(W / num_parts) + kFixedCost of cost (the extra kFixedCost pays
-// for the chunk a split adds, so the budgets cover the total); a virtual batch
-// that does not fit whole is cut at a page boundary and continues in the next
-// partition (a split).  The last partition takes whatever remains.
+// to query rows [128 g, 128 g + 128) of its s_q * h_q rows.  Lay the virtual
+// batches on a line of cost units: vb takes kFixedCost units of per-chunk
+// overhead (Q load, epilogue) followed by one unit per 64-token page, starting
+// at C[vb] = sum of the costs before it; W is the total.  Partition p takes the
+// units [p T, (p + 1) T) with T = ceil(W / num_parts).  A unit position x maps to
+// the page position (vb, blk) with vb the virtual batch whose span holds x and
+// blk = clamp(x - C[vb] - kFixedCost, 0, pages(vb)); partition p covers the page
+// positions from map(p T) up to map((p + 1) T).  A virtual batch whose pages are
+// cut by partition starts is split; every partition computes its range on its
+// own, so the device version is one thread per partition.
 //
 // Output:
 //   md[p * 8 + 0..4] = begin_vb, begin_blk, end_vb, end_blk, begin_split
@@ -48,46 +51,84 @@ MLA_HD inline int row_groups(int heads_per_kv) { return (heads_per_kv + kRowsPer
 
 MLA_HD inline int pages_of(int seqlen) { return seqlen <= 0 ? 0 : (seqlen + kPage - 1) / kPage; }
 
-// seqlens: [batch]; md: [num_parts * 8]; num_splits: [batch * groups + 1].
-MLA_HD inline void schedule(const int32_t* seqlens, int batch, int groups, int num_parts, int32_t* md,
-                            int32_t* num_splits)
+// Position on the page line of cost unit x.  C: exclusive prefix of the costs,
+// nv entries; total: W.  Returns (vb, blk) through the references.
+MLA_HD inline void unit_to_page(long long x, const long long* C, const int32_t* pages, int nv, long long total,
+                                int& vb, int& blk)
+{
+    if (x >= total) {
+        vb = nv;
+        blk = 0;
+        return;
+    }
+    int lo = 0, hi = nv - 1;  // largest v with C[v] <= x
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (C[mid] <= x)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    long long b = x - C[lo] - kFixedCost;
+    if (b < 0) b = 0;
+    vb = lo;
+    blk = static_cast<int>(b);  // < pages[lo]: positions at or past the span's end belong to lo + 1
+    (void)pages;
+}
+
+// Range of partition p: md row.  C / pages: per virtual batch.
+MLA_HD inline void partition_range(int p, int num_parts, const long long* C, const int32_t* pages, int nv,
+                                   long long total, int32_t* m)
+{
+    const long long T = (total + num_parts - 1) / num_parts;
+    int bv, bb, ev, eb;
+    unit_to_page(static_cast<long long>(p) * T, C, pages, nv, total, bv, bb);
+    if (p == num_parts - 1) {
+        ev = nv;
+        eb = 0;
+    } else {
+        unit_to_page(static_cast<long long>(p + 1) * T, C, pages, nv, total, ev, eb);
+    }
+    m[0] = bv;
+    m[1] = bb;
+    m[2] = ev;
+    m[3] = eb;
+    m[4] = 0;
+    m[5] = m[6] = m[7] = 0;
+}
+
+// Host reference of the whole schedule (the device kernel computes the same
+// values in parallel).  Scratch: C [nv] and pages [nv].
+inline void schedule_host(const int32_t* seqlens, int batch, int groups, int num_parts, int32_t* md,
+                          int32_t* num_splits, long long* C, int32_t* pages)
 {
     const int nv = batch * groups;
-    long long W = 0;
-    for (int b = 0; b < batch; ++b) W += static_cast<long long>(pages_of(seqlens[b]) + kFixedCost) * groups;
-    const long long T = (W + num_parts - 1) / num_parts + kFixedCost;
-
-    num_splits[0] = 0;
-    int vb = 0, blk = 0, cur_split = 0;
+    long long total = 0;
+    for (int v = 0; v < nv; ++v) {
+        pages[v] = pages_of(seqlens[v / groups]);
+        C[v] = total;
+        total += pages[v] + kFixedCost;
+    }
+    for (int p = 0; p < num_parts; ++p) partition_range(p, num_parts, C, pages, nv, total, md + p * kMdInts);
+    // split counts: 1 + number of partitions that start inside a virtual batch's pages
+    for (int v = 0; v <= nv; ++v) num_splits[v] = 0;
     for (int p = 0; p < num_parts; ++p) {
         int32_t* m = md + p * kMdInts;
-        m[0] = vb;
-        m[1] = blk;
-        m[4] = cur_split;
-        m[5] = m[6] = m[7] = 0;
-        const bool last = (p == num_parts - 1);
-        long long budget = T;
-        while (vb < nv) {
-            const int n = pages_of(seqlens[vb / groups]);
-            const int rest = n - blk;
-            if (rest + kFixedCost <= budget || last) {
-                budget -= rest + kFixedCost;
-                num_splits[vb + 1] = num_splits[vb] + cur_split + 1;
-                ++vb;
-                blk = 0;
-                cur_split = 0;
-                if (budget <= 0 && !last) break;
-            } else {
-                const long long take = budget - kFixedCost;
-                if (take <= 0) break;
-                blk += static_cast<int>(take);
-                ++cur_split;
-                break;
-            }
+        if (m[1] > 0) {
+            // index of this split = 1 + number of earlier mid-batch starts in the same vb
+            int idx = 1;
+            for (int q = p - 1; q >= 0 && md[q * kMdInts + 0] == m[0] && md[q * kMdInts + 1] > 0; --q) ++idx;
+            m[4] = idx;
+            num_splits[m[0] + 1] += 1;  // extra splits, accumulated below
         }
-        m[2] = vb;
-        m[3] = blk;
     }
+    int acc = 0;
+    for (int v = 0; v < nv; ++v) {
+        const int extra = num_splits[v + 1];
+        num_splits[v] = acc;
+        acc += 1 + extra;
+    }
+    num_splits[nv] = acc;
 }
 
 }  // namespace mla
