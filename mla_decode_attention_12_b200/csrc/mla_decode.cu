@@ -56,14 +56,17 @@
 
 namespace mla {
 
-constexpr int kThreads = 224;          // 4 softmax warps + Q/K loader + MMA issuer + V loader
+constexpr int kThreads = 256;          // 4 softmax warps + K loader + MMA issuer + V loader + Q loader
 constexpr int kKWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kVWarp = 6;
+constexpr int kQWarp = 7;
 constexpr int kDv = 512;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;         // O: columns [0, 256)
 constexpr uint32_t kTmemS = 256;       // S buffers: [256, 288), [288, 320)
+constexpr uint32_t kTmemQ = 320;       // Q columns [0, 384) as the A operand: [320, 512)
+constexpr int kQTmemBoxes = 6;         // 64-column boxes of Q kept in tensor memory
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 constexpr int kWorkspaceHeader = 256;
@@ -72,14 +75,16 @@ constexpr int kWorkspaceHeader = 256;
 template <bool kRope>
 struct Layout {
     static constexpr int kBoxes = kRope ? 9 : 8;               // 64-column boxes in a d_qk row
-    static constexpr int kQBytes = kBoxes * 8192;              // Q: 64 rows x d_qk, one SW128 box per 64 columns
+    static constexpr int kQSmemBoxes = kBoxes - kQTmemBoxes;   // Q boxes kept in shared memory
+    static constexpr int kQBytes = kQSmemBoxes * 8192;         // 64 rows, one SW128 box per 64 columns
     static constexpr int kKBytes = kBoxes * 4096;              // K: this CTA's 32 tokens of a page x d_qk
+    static constexpr int kKStages = 3;
     static constexpr int kVBytes = 4 * 8192;                   // V: 64 tokens x this CTA's 256 d_v columns
     static constexpr int kPBytes = 8192;                       // P: 64 rows x 64 tokens, 16-bit
     static constexpr int kKSteps = kBoxes * 4;                 // K=16 MMA steps of Q K^T
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kQBytes;              // 2 stages
-    static constexpr int kOffV = kOffK + 2 * kKBytes;          // 2 stages
+    static constexpr int kOffK = kOffQ + kQBytes;              // kKStages stages
+    static constexpr int kOffV = kOffK + kKStages * kKBytes;   // 2 stages
     static constexpr int kOffP = kOffV + 2 * kVBytes;          // 2 buffers
     static constexpr int kOffRed = kOffP + 2 * kPBytes;        // 3 x 128 floats: 2 page row-max halves, row sums
     static constexpr int kRedBytes = 3 * 128 * 4;
@@ -89,25 +94,40 @@ struct Layout {
 };
 
 enum BarSlot : int {
-    kBarQFull = 0,    // leader: Q of both CTAs landed (transaction bytes)
+    kBarQFull = 0,    // leader: Q of both CTAs in place (TMA bytes + 8 softmax warps' TMEM stores)
     kBarQFree = 1,    // both: the chunk's Q K^T MMAs completed
-    kBarKFull = 2,    // leader, 2 stages
-    kBarKEmpty = 4,   // both, 2 stages
-    kBarVFull = 6,    // leader, 2 stages
-    kBarVEmpty = 8,   // both, 2 stages
-    kBarSFull = 10,   // both, 2 S buffers
-    kBarPFull = 12,   // leader, 2 P buffers, 8 warps (4 per CTA)
-    kBarPvDone = 14,  // both, 2 P buffers
-    kBarOFull = 16,   // both
-    kBarOFree = 17,   // leader, 8 warps
-    kBarDrain = 18,   // leader
-    kBarTail = 19,    // both: V load of a sequence's last page (local)
-    kBarPair = 20,    // both: 2 slots, rendezvous of softmax warps {w, w ^ 2} (64 threads)
-    kBarCount = 22
+    kBarKFull = 2,    // leader, 3 stages
+    kBarKEmpty = 5,   // both, 3 stages
+    kBarVFull = 8,    // leader, 2 stages
+    kBarVEmpty = 10,  // both, 2 stages
+    kBarSFull = 12,   // both, 2 S buffers
+    kBarPFull = 14,   // leader, 2 P buffers, 8 warps (4 per CTA)
+    kBarPvDone = 16,  // both, 2 P buffers
+    kBarOFull = 18,   // both
+    kBarOFree = 19,   // leader, 8 warps
+    kBarDrain = 20,   // leader
+    kBarTail = 21,    // both: V load of a sequence's last page (local)
+    kBarPair = 22,    // both: 2 slots, rendezvous of softmax warps {w, w ^ 2} (one arrive per warp)
+    kBarCount = 24
+};
+
+// Position in a ring of kN stages: stage index and the parity of its current use.
+template <int kN>
+struct Ring {
+    uint32_t stage = 0, phase = 0;
+    __device__ void advance()
+    {
+        if (++stage == kN) {
+            stage = 0;
+            phase ^= 1u;
+        }
+    }
 };
 constexpr int kOffTmemSlot = kBarCount * 8;  // uint32 written by tcgen05.alloc
 constexpr int kOffAbort = kOffTmemSlot + 4;  // int abort flag
 static_assert(kOffAbort + 4 <= Layout<true>::kBarBytes, "barrier area too small");
+static_assert(2 * Layout<true>::kPBytes >= 4 * 32 * 32 * 4, "epilogue staging must fit in the P buffers");
+static_assert(kTmemQ + 8 * 4 * kQTmemBoxes == kTmemCols, "tensor memory plan");
 static_assert(Layout<true>::kSmemBytes <= 232448 && Layout<false>::kSmemBytes <= 232448,
               "shared memory plan exceeds 227 KB");
 static_assert(Layout<true>::kOffQ % 1024 == 0 && Layout<true>::kOffK % 1024 == 0 && Layout<true>::kOffV % 1024 == 0 &&
@@ -120,6 +140,8 @@ struct DecodeParams {
     const int32_t* seqlens;
     const int32_t* md;
     const int32_t* num_splits;
+    const void* q;
+    const void* kvcache;
     void* o;
     float* lse;
     float* o_accum;     // [slots, 128, 512]
@@ -153,6 +175,7 @@ struct Sync {
     // Bounded wait for phase `parity` of `bar`.  Returns false on abort / timeout.
     __device__ bool wait(uint32_t bar, uint32_t parity) const
     {
+        if (mbar_test_wait(bar, parity)) return true;
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         const uint64_t t0 = global_timer_ns();
@@ -246,11 +269,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     // ---------------- set-up
     if (threadIdx.x == 0) {
-        mbar_init(bar(kBarQFull), 1);
+        mbar_init(bar(kBarQFull), 1 + 8);
         mbar_init(bar(kBarQFree), 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < L::kKStages; ++s) {
             mbar_init(bar(kBarKFull + s), 1);
             mbar_init(bar(kBarKEmpty + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(bar(kBarVFull + s), 1);
             mbar_init(bar(kBarVEmpty + s), 1);
             mbar_init(bar(kBarSFull + s), 1);
@@ -261,8 +286,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_init(bar(kBarOFree), 8);
         mbar_init(bar(kBarDrain), 1);
         mbar_init(bar(kBarTail), 1);
-        mbar_init(bar(kBarPair + 0), 64);
-        mbar_init(bar(kBarPair + 1), 64);
+        mbar_init(bar(kBarPair + 0), 2);
+        mbar_init(bar(kBarPair + 1), 2);
         *reinterpret_cast<volatile int*>(smem + L::kOffBar + kOffAbort) = 0;
         fence_mbar_init();
     }
@@ -276,7 +301,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_alloc_pair(s_bar + kOffTmemSlot, kTmemCols);
         tmem_relinquish_pair();
     }
-    if (warp == kKWarp && lane == 0) {
+    if (warp == kQWarp && lane == 0) {
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
@@ -293,11 +318,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int begin_vb = md[0];
     const int begin_split = md[4];
 
-    if (warp == kKWarp) {
-        // ============================ Q and K producer ============================
+    if (warp == kQWarp) {
+        // ============================ Q producer ============================
+        // Loads the shared-memory part of each chunk's 64 query rows (columns
+        // 384 and up) once the previous chunk's Q K^T MMAs are done; the softmax
+        // warps store columns [0, 384) into tensor memory.
         if (lane == 0) {
-            const uint32_t q_tx = L::kBoxes * p.box_rows * 128;
-            uint32_t g = 0, k = 0;
+            const uint32_t q_tx = L::kQSmemBoxes * p.box_rows * 128;
+            const int y_off = 64 * static_cast<int>(cta);
+            uint32_t k = 0;
             int vb, lo, hi;
             bool ok = true;
             while (ok && chunks.next(vb, lo, hi)) {
@@ -305,13 +334,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int b = vb / p.groups, rg = vb % p.groups;
                 if (!(ok = sync.wait(bar(kBarQFree), (k & 1) ^ 1))) break;
                 if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * q_tx);
-                for (int i = 0; i < L::kBoxes; ++i)
-                    tma_load_3d_pair(s_q + i * 8192, &tm_q, lead_bar(kBarQFull), 64 * i,
-                                     rg * kRowsPerGroup + 64 * static_cast<int>(cta), b);
+                for (int i = 0; i < L::kQSmemBoxes; ++i)
+                    tma_load_3d_pair(s_q + i * 8192, &tm_q, lead_bar(kBarQFull), 64 * (kQTmemBoxes + i),
+                                     rg * kRowsPerGroup + y_off, b);
+                ++k;
+            }
+            if (!ok) {
+                const uint64_t t0 = global_timer_ns();  // let issued loads land (see the V producer)
+                while (global_timer_ns() - t0 < 50000000ull) {
+                }
+            }
+        }
+    } else if (warp == kKWarp) {
+        // ============================ K producer ============================
+        if (lane == 0) {
+            Ring<L::kKStages> ring;
+            int vb, lo, hi;
+            bool ok = true;
+            while (ok && chunks.next(vb, lo, hi)) {
+                if (hi <= lo) continue;
+                const int b = vb / p.groups;
                 const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-                for (int blk = lo; blk < hi; ++blk, ++g) {
-                    const uint32_t st = g & 1;
-                    if (!(ok = sync.wait(bar(kBarKEmpty + st), ((g >> 1) & 1) ^ 1))) break;
+                for (int blk = lo; blk < hi; ++blk, ring.advance()) {
+                    const uint32_t st = ring.stage;
+                    if (!(ok = sync.wait(bar(kBarKEmpty + st), ring.phase ^ 1))) break;
                     const int page = page_of(p, table, blk);
                     if (leader) mbar_arrive_expect_tx(bar(kBarKFull + st), 2 * L::kKBytes);
                     const uint32_t dst = s_k + st * L::kKBytes;
@@ -319,7 +365,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         tma_load_2d_pair(dst + i * 4096, &tm_k, lead_bar(kBarKFull + st), 64 * i,
                                          page * kPage + 32 * static_cast<int>(cta));
                 }
-                ++k;
             }
             if (!ok) {
                 const uint64_t t0 = global_timer_ns();  // let issued loads land (see the V producer)
@@ -350,11 +395,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const bool is_tail = (blk == last_page) && tail != 0;
                 if (lane == 0 && leader) mbar_arrive_expect_tx(bar(kBarVFull + st), 2 * L::kVBytes);
                 if (!is_tail) {
-                    if (lane == 0)
+                    if (lane == 0) {
                         for (int i = 0; i < 4; ++i) {
                             const int box = 4 * (i >> 1) + 2 * static_cast<int>(cta) + (i & 1);
                             tma_load_2d_pair(dst + i * 8192, &tm_v, lead_bar(kBarVFull + st), 64 * box, page * kPage);
                         }
+                    }
                 } else {
                     if (lane == 0) {
                         mbar_arrive_expect_tx(bar(kBarTail), L::kVBytes);
@@ -433,25 +479,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 return true;
             };
+            Ring<L::kKStages> kring;
             while (ok && chunks.next(vb, lo, hi)) {
                 const int n = hi - lo;
                 if (n <= 0) continue;
                 if (!(ok = wwait(bar(kBarQFull), k & 1))) break;
-                for (int j = 0; j < n && ok; ++j) {
+                for (int j = 0; j < n && ok; ++j, kring.advance()) {
                     const uint32_t gp = g + j;
-                    const uint32_t st = gp & 1;
-                    if (!(ok = wwait(bar(kBarKFull + st), (gp >> 1) & 1))) break;
+                    const uint32_t sb = gp & 1;
+                    const uint32_t st = kring.stage;
+                    if (!(ok = wwait(bar(kBarKFull + st), kring.phase))) break;
                     tc_fence_after();
                     if (issuer) {
                         const uint64_t kd0 = k_desc + ((st * L::kKBytes) >> 4);
+                        // Q columns [0, 384) from tensor memory (8 columns per K=16 step) ...
 #pragma unroll
-                        for (int ks = 0; ks < L::kKSteps; ++ks) {
+                        for (int ks = 0; ks < 4 * kQTmemBoxes; ++ks)
+                            mma_ts_pair(tmem + kTmemS + 32 * sb, tmem + kTmemQ + 8 * ks,
+                                        kd0 + (((ks >> 2) * 4096 + (ks & 3) * 32) >> 4), idesc_qk, ks > 0 ? 1u : 0u);
+                        // ... and the remaining columns from shared memory.
+#pragma unroll
+                        for (int ks = 4 * kQTmemBoxes; ks < L::kKSteps; ++ks) {
                             const int box = ks >> 2, sub = ks & 3;
-                            mma_ss_pair(tmem + kTmemS + 32 * st, q_desc + ((box * 8192 + sub * 32) >> 4),
-                                        kd0 + ((box * 4096 + sub * 32) >> 4), idesc_qk, ks > 0 ? 1u : 0u);
+                            mma_ss_pair(tmem + kTmemS + 32 * sb, q_desc + (((box - kQTmemBoxes) * 8192 + sub * 32) >> 4),
+                                        kd0 + ((box * 4096 + sub * 32) >> 4), idesc_qk, 1u);
                         }
                         mma_commit_pair(bar(kBarKEmpty + st), both);
-                        mma_commit_pair(bar(kBarSFull + st), both);
+                        mma_commit_pair(bar(kBarSFull + sb), both);
                         if (j == n - 1) mma_commit_pair(bar(kBarQFree), both);
                     }
                     __syncwarp();
@@ -482,11 +536,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t pair_phase = 0;
         const uint32_t p_full_lead[2] = {lead_bar(kBarPFull), lead_bar(kBarPFull + 1)};
         const uint32_t o_free_lead = lead_bar(kBarOFree);
+        const uint32_t q_full_lead = lead_bar(kBarQFull);
         auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
+        // Q columns [0, 384) of this thread's row of chunk `kq` into tensor memory, the A
+        // operand of Q K^T.  Threads t and t ^ 64 hold the same row and write the same
+        // values: the pair MMA reads A duplicated in lane quadrants {0,2} and {1,3}.
+        auto store_q = [&](int qvb, uint32_t kq) -> bool {
+            const int qb = qvb / p.groups;
+            const int qrow_idx = (qvb % p.groups) * kRowsPerGroup + 64 * static_cast<int>(cta) + r;
+            if (!wwait(bar(kBarQFree), (kq & 1) ^ 1)) return false;
+            tc_fence_after();
+            const bool valid = qrow_idx < p.rows;
+            const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
+                                                               (static_cast<size_t>(qb) * p.rows + qrow_idx) * p.d_qk * 2);
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                uint4 v[24];
+#pragma unroll
+                for (int i = 0; i < 24; ++i) v[i] = valid ? __ldg(qrow + 24 * half + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int c = 0; c < 3; ++c) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        w[4 * i] = v[8 * c + i].x;
+                        w[4 * i + 1] = v[8 * c + i].y;
+                        w[4 * i + 2] = v[8 * c + i].z;
+                        w[4 * i + 3] = v[8 * c + i].w;
+                    }
+                    tmem_st32(tmem + kTmemQ + lane_base + 96 * half + 32 * c, w);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader)
+                    mbar_arrive(bar(kBarQFull));
+                else
+                    mbar_arrive_remote(q_full_lead);
+            }
+            return true;
+        };
         uint32_t g = 0, k = 0;
         int vb, lo, hi;
         bool ok = true;
-        while (ok && chunks.next(vb, lo, hi)) {
+        bool have = chunks.next(vb, lo, hi);
+        bool q_ready = false;  // this chunk's Q already stored (ahead of the previous epilogue)
+        while (ok && have) {
             const int b = vb / p.groups, rg = vb % p.groups;
             const int Lb = p.seqlens[b];
             const int row = rg * kRowsPerGroup + 64 * static_cast<int>(cta) + r;
@@ -499,11 +596,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int n = hi - lo;
             float m_ref = -INFINITY, l_half = 0.f;
 
+            if (n > 0 && !q_ready && !(ok = store_q(vb, k))) break;
+            q_ready = false;
+
             for (int j = 0; j < n; ++j) {
                 const uint32_t gp = g + j;
                 const uint32_t sb = gp & 1;
                 if (!(ok = wwait(bar(kBarSFull + sb), (gp >> 1) & 1))) break;
                 tc_fence_after();
+                // Logits stay unscaled until the exponent: scale > 0 keeps the maximum, and
+                // scale * s - ref is one FFMA.  Only a page the row does not fully see
+                // (the sequence's last page, the causal diagonal) needs the mask.
                 float x[32];
                 {
                     uint32_t a[32];
@@ -511,14 +614,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     tmem_wait_ld();
                     reg_fence(a);
                     const int lim = n_vis - (lo + j) * kPage - 32 * h;  // columns >= lim are not visible
+                    if (__all_sync(0xffffffffu, lim >= 32)) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) x[c] = (c < lim) ? __uint_as_float(a[c]) * p.scale_log2 : -INFINITY;
+                        for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(a[c]);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) x[c] = (c < lim) ? __uint_as_float(a[c]) : -INFINITY;
+                    }
                 }
-                float mx = x[0];
+                float mx;
+                {
+                    float m16[16];
 #pragma unroll
-                for (int c = 1; c < 32; ++c) mx = fmaxf(mx, x[c]);
+                    for (int c = 0; c < 16; ++c) m16[c] = fmaxf(x[c], x[c + 16]);
+#pragma unroll
+                    for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                        for (int c = 0; c < w; ++c) m16[c] = fmaxf(m16[c], m16[c + w]);
+                    mx = m16[0] * p.scale_log2;  // log2-domain maximum (-inf stays -inf)
+                }
                 red[sb * 128 + t] = mx;
-                mbar_arrive(pair_bar);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(pair_bar);
                 if (!(ok = wwait(pair_bar, pair_phase++ & 1))) break;
                 mx = fmaxf(mx, red[sb * 128 + (t ^ 64)]);
                 // the same decision in both halves of the row
@@ -532,15 +649,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     m_ref = mx;
                 }
                 const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
-                float rs = 0.f;
                 uint32_t pk[16];
+                float s16[16];
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
-                    const float p0 = fast_exp2(x[2 * c] - ref);
-                    const float p1 = fast_exp2(x[2 * c + 1] - ref);
-                    rs += p0 + p1;
+                    const float p0 = fast_exp2(fmaf(x[2 * c], p.scale_log2, -ref));
+                    const float p1 = fast_exp2(fmaf(x[2 * c + 1], p.scale_log2, -ref));
+                    s16[c] = p0 + p1;
                     pk[c] = pack2(p0, p1, kFp16);
                 }
+#pragma unroll
+                for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int c = 0; c < w; ++c) s16[c] += s16[c + w];
+                const float rs = s16[0];
                 l_half = l_half * alpha + rs;
 
                 if (__any_sync(0xffffffffu, rescale)) {
@@ -561,8 +683,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     tmem_wait_st();
                 }
-                // P buffer gp&1 was last read by the PV of page gp-2
-                if (gp >= 2 && !(ok = wwait(bar(kBarPvDone + sb), ((gp - 2) >> 1) & 1))) break;
+                // P buffer gp&1 was last read by the PV of page gp-2.  That PV was issued
+                // before the Q K^T of page gp, tcgen05 MMAs of one thread complete in
+                // issue order, and the S_full commit of page gp covers every earlier MMA:
+                // having waited for S_full, the buffer is free.
                 {
                     uint8_t* prow = smem + L::kOffP + sb * L::kPBytes + r * 128;
 #pragma unroll
@@ -584,14 +708,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
 
+            // The next chunk's Q goes into tensor memory now (its region is free once this
+            // chunk's last Q K^T is done, which S_full of the last page implies), so the MMA
+            // can start the next chunk while this epilogue drains O.
+            int nvb = 0, nlo = 0, nhi = 0;
+            const bool have_next = chunks.next(nvb, nlo, nhi);
+            if (have_next && nhi > nlo && n > 0) {
+                if (!(ok = store_q(nvb, k + 1))) break;
+                q_ready = true;
+            }
+
             // ---- epilogue: full row sum from both halves, O / l, LSE
             const bool empty = (n <= 0);
             red[256 + t] = l_half;
-            mbar_arrive(pair_bar);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pair_bar);
             if (!(ok = wwait(pair_bar, pair_phase++ & 1))) break;
             const float l_other = red[256 + (t ^ 64)];
             const float l_sum = (h == 0) ? (l_half + l_other) : (l_other + l_half);
-            mbar_arrive(pair_bar);  // red[256..] free for the next chunk once both have read it
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pair_bar);  // red[256..] free for the next chunk once both have read it
             if (!(ok = wwait(pair_bar, pair_phase++ & 1))) break;
             const float inv_l = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
             const float lse_v = (l_sum > 0.f) ? (m_ref + log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
@@ -599,11 +735,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (!(ok = wwait(bar(kBarOFull), k & 1))) break;
                 tc_fence_after();
             }
+            // O leaves tensor memory one 32-column block at a time: each thread holds 32
+            // values of its own row; the warp transposes the 32 x 32 block through shared
+            // memory (the P buffers are idle now) so that global stores write whole
+            // 128-byte row segments instead of one 16-byte piece per row.
+            {
+                // 4 KB per warp (the two P buffers hold the four warps' tiles); element
+                // (row, col) sits at row * 32 + (col ^ row): conflict-free in both directions.
+                float* stage = reinterpret_cast<float*>(smem + L::kOffP) + warp * (32 * 32);
+                const int row_base = rg * kRowsPerGroup + 64 * static_cast<int>(cta) + (t & 32);  // warp's first row
+                const size_t slot = static_cast<size_t>(p.num_splits[vb]) + split_idx;
 #pragma unroll 1
-            for (int i = 0; i < 2; ++i) {
-                const int col0 = 256 * i + 128 * h;  // first d_v column this thread holds in chunk i
-#pragma unroll 1
-                for (int cb = 0; cb < 4; ++cb) {
+                for (int blk = 0; blk < 8; ++blk) {
+                    const int i = blk >> 2, cb = blk & 3;
+                    const int colw = 256 * i + 128 * h + 32 * cb;  // first d_v column of the block
                     uint32_t v[32];
                     if (!empty) {
                         tmem_ld32(tmem + kTmemO + 128 * i + lane_base + 32 * cb, v);
@@ -613,28 +758,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 32; ++e) v[e] = 0;
                     }
-                    if (!row_valid) continue;
-                    if (nsplit == 1) {
-                        uint4* dst = reinterpret_cast<uint4*>(
-                            static_cast<uint8_t*>(p.o) +
-                            ((static_cast<size_t>(b) * p.rows + row) * kDv + col0 + 32 * cb) * 2);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(
-                                pack2(__uint_as_float(v[8 * e + 0]) * inv_l, __uint_as_float(v[8 * e + 1]) * inv_l, kFp16),
-                                pack2(__uint_as_float(v[8 * e + 2]) * inv_l, __uint_as_float(v[8 * e + 3]) * inv_l, kFp16),
-                                pack2(__uint_as_float(v[8 * e + 4]) * inv_l, __uint_as_float(v[8 * e + 5]) * inv_l, kFp16),
-                                pack2(__uint_as_float(v[8 * e + 6]) * inv_l, __uint_as_float(v[8 * e + 7]) * inv_l, kFp16));
-                    } else {
-                        const size_t slot = static_cast<size_t>(p.num_splits[vb]) + split_idx;
-                        float4* dst = reinterpret_cast<float4*>(
-                            p.o_accum + (slot * kRowsPerGroup + 64 * cta + r) * kDv + col0 + 32 * cb);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv_l, __uint_as_float(v[4 * e + 1]) * inv_l,
-                                                 __uint_as_float(v[4 * e + 2]) * inv_l,
-                                                 __uint_as_float(v[4 * e + 3]) * inv_l);
+                    for (int e = 0; e < 32; ++e) stage[lane * 32 + (e ^ lane)] = __uint_as_float(v[e]) * inv_l;
+                    __syncwarp();
+                    // lane = (row offset within a group of 4 rows) * 8 + (4-column group)
+                    const int cg = lane & 7, rsub = lane >> 3;
+#pragma unroll 2
+                    for (int rr = 0; rr < 32; rr += 4) {
+                        const int lr = rr + rsub;  // row within the warp's 32
+                        const int grow = row_base + lr;
+                        const float* src = stage + lr * 32;
+                        const float a0 = src[(4 * cg + 0) ^ lr], a1 = src[(4 * cg + 1) ^ lr];
+                        const float a2 = src[(4 * cg + 2) ^ lr], a3 = src[(4 * cg + 3) ^ lr];
+                        if (grow < p.rows) {
+                            if (nsplit == 1) {
+                                uint2* dst = reinterpret_cast<uint2*>(
+                                    static_cast<uint8_t*>(p.o) + ((static_cast<size_t>(b) * p.rows + grow) * kDv + colw + 4 * cg) * 2);
+                                *dst = make_uint2(pack2(a0, a1, kFp16), pack2(a2, a3, kFp16));
+                            } else {
+                                float4* dst = reinterpret_cast<float4*>(
+                                    p.o_accum + (slot * kRowsPerGroup + (grow - rg * kRowsPerGroup)) * kDv + colw + 4 * cg);
+                                *dst = make_float4(a0, a1, a2, a3);
+                            }
+                        }
                     }
+                    __syncwarp();
                 }
             }
             if (h == 0) {
@@ -657,6 +805,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 ++k;
             }
             g += (n > 0 ? n : 0);
+            have = have_next;
+            vb = nvb;
+            lo = nlo;
+            hi = nhi;
         }
     }
 
@@ -1020,6 +1172,8 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     prm.seqlens = cache_seqlens;
     prm.md = tile_md;
     prm.num_splits = num_splits;
+    prm.q = q;
+    prm.kvcache = kvcache;
     prm.o = o;
     prm.lse = lse;
     prm.batch = batch;
