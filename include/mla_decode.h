@@ -196,6 +196,42 @@ MLA_API mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int
  */
 MLA_API mla_status mla_read_device_status(void* workspace, int clear, int* device_status, void* stream);
 
+/*
+ * Allocation-free variant of mla_decode_with_kvcache (the pages describe no
+ * counterpart: it exists for callers that cannot allocate device memory).
+ *
+ * Some callers cannot call cudaMalloc or any allocator at decode time: runtimes
+ * that plan all device memory ahead and forbid later allocations, plugins that
+ * are handed only tensor pointers by a host framework that owns every buffer,
+ * and latency-critical paths where an allocation could block.  This entry point
+ * takes the same arguments as mla_decode_with_kvcache minus the workspace; it
+ * uses instead a fixed scratch array of MLA_NOALLOC_SCRATCH_BYTES compiled into
+ * the library, which every GPU that loads the library holds until the process
+ * exits.  The caller still provides q, kvcache, block_table, cache_seqlens, the
+ * scheduler outputs, o and lse.
+ *
+ *   - Problems needing more than MLA_NOALLOC_SCRATCH_BYTES of workspace
+ *     (mla_decode_workspace_bytes) are rejected with MLA_ERR_WORKSPACE.
+ *   - The first call on a device looks up the device address of the scratch
+ *     array (once per device, with that device current); make that first call
+ *     before capturing any stream on that device.
+ *   - No memory is allocated or freed; each call clears the scratch status word
+ *     with an asynchronous memset on `stream` and then enqueues the same kernels
+ *     as mla_decode_with_kvcache.
+ *   - All calls on a device share one scratch array, which keeps the last
+ *     call's contents: calls whose execution overlaps on the GPU (different
+ *     streams without ordering between them) race on it and give wrong results.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+MLA_API mla_status mla_decode_with_kvcache_noalloc(const void* q, int batch, int s_q, int h_q, int d_qk,
+                                                   const void* kvcache, int num_blocks, int page_size,
+                                                   int h_kv, const int32_t* block_table,
+                                                   int max_blocks_per_seq, const int32_t* cache_seqlens,
+                                                   int dv, int dtype, const int32_t* tile_md,
+                                                   int num_parts, const int32_t* num_splits, int causal,
+                                                   float softmax_scale, void* o, float* lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

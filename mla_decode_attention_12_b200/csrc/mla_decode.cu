@@ -1314,3 +1314,62 @@ mla_status mla_read_device_status(void* workspace, int clear, int* device_status
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free decode
+// Scratch of mla_decode_with_kvcache_noalloc: the same layout as a caller-provided
+// workspace (status header, split LSEs, split partial outputs), held in a
+// file-scope device array of MLA_NOALLOC_SCRATCH_BYTES on every GPU that loads
+// this library, for the life of the process.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};  // device address of the array, per device
+
+// Device address of the scratch array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address comes from the
+// runtime, once per device, with that device current.
+mla_status noalloc_scratch(void** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return MLA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+            cudaGetLastError();
+            return MLA_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return MLA_OK;
+}
+}  // namespace
+
+extern "C" mla_status mla_decode_with_kvcache_noalloc(const void* q, int batch, int s_q, int h_q, int d_qk,
+                                                      const void* kvcache, int num_blocks, int page_size, int h_kv,
+                                                      const int32_t* block_table, int max_blocks_per_seq,
+                                                      const int32_t* cache_seqlens, int dv, int dtype,
+                                                      const int32_t* tile_md, int num_parts,
+                                                      const int32_t* num_splits, int causal, float softmax_scale,
+                                                      void* o, float* lse, void* stream)
+{
+    if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_parts <= 0) return MLA_ERR_INVALID_ARG;
+    if (batch == 0) return MLA_OK;
+    const size_t need = mla_decode_workspace_bytes(batch, s_q, h_q, h_kv, num_parts);
+    if (need == 0) return MLA_ERR_INVALID_ARG;
+    if (need > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;  // problem too large for the fixed scratch
+    void* scratch = nullptr;
+    mla_status st = noalloc_scratch(&scratch);
+    if (st != MLA_OK) return st;
+    // The status word must start at zero; the split partials are always written
+    // before they are read, so the rest of the scratch needs no clearing.
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(scratch, 0, sizeof(int), cs) != cudaSuccess) return MLA_ERR_CUDA;
+    return mla_decode_with_kvcache(q, batch, s_q, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, block_table,
+                                   max_blocks_per_seq, cache_seqlens, dv, dtype, tile_md, num_parts, num_splits,
+                                   causal, softmax_scale, o, lse, scratch, MLA_NOALLOC_SCRATCH_BYTES, stream);
+}
