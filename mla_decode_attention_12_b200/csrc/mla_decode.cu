@@ -267,6 +267,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int part = blockIdx.x >> 1;
     auto lead_bar = [&](int slot) { return map_to_cta(bar(slot), 0); };  // leader's barrier, cluster address
 
+    // The first chunk's query rows start moving into L2 before the set-up.
+    if (warp < 4) {
+        const int32_t* md0 = p.md + part * kMdInts;
+        ChunkIter first{md0[0], md0[1], md0[2], md0[3], p.groups, p.seqlens};
+        int fvb, flo, fhi;
+        while (first.next(fvb, flo, fhi))
+            if (fhi > flo) {
+                const int qrow_idx = (fvb % p.groups) * kRowsPerGroup + 64 * static_cast<int>(cta) + (threadIdx.x & 63);
+                if (qrow_idx < p.rows) {
+                    const uint8_t* a = static_cast<const uint8_t*>(p.q) +
+                                       (static_cast<size_t>(fvb / p.groups) * p.rows + qrow_idx) * p.d_qk * 2;
+                    for (int i = 0; i < 6; ++i) prefetch_l2(a + 128 * i);
+                }
+                break;
+            }
+    }
+
     // ---------------- set-up
     if (threadIdx.x == 0) {
         mbar_init(bar(kBarQFull), 1 + 8);
@@ -538,17 +555,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t o_free_lead = lead_bar(kBarOFree);
         const uint32_t q_full_lead = lead_bar(kBarQFull);
         auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
+        auto q_row_ptr = [&](int qvb, bool& valid) {
+            const int qrow_idx = (qvb % p.groups) * kRowsPerGroup + 64 * static_cast<int>(cta) + r;
+            valid = qrow_idx < p.rows;
+            return reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
+                                                  (static_cast<size_t>(qvb / p.groups) * p.rows + qrow_idx) * p.d_qk * 2);
+        };
+        auto prefetch_q_row = [&](int qvb) {
+            bool valid;
+            const uint8_t* a = reinterpret_cast<const uint8_t*>(q_row_ptr(qvb, valid));
+            if (valid)
+                for (int i = 0; i < 6; ++i) prefetch_l2(a + 128 * i);
+        };
         // Q columns [0, 384) of this thread's row of chunk `kq` into tensor memory, the A
         // operand of Q K^T.  Threads t and t ^ 64 hold the same row and write the same
         // values: the pair MMA reads A duplicated in lane quadrants {0,2} and {1,3}.
         auto store_q = [&](int qvb, uint32_t kq) -> bool {
-            const int qb = qvb / p.groups;
-            const int qrow_idx = (qvb % p.groups) * kRowsPerGroup + 64 * static_cast<int>(cta) + r;
+            bool valid;
+            const uint4* qrow = q_row_ptr(qvb, valid);
             if (!wwait(bar(kBarQFree), (kq & 1) ^ 1)) return false;
             tc_fence_after();
-            const bool valid = qrow_idx < p.rows;
-            const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
-                                                               (static_cast<size_t>(qb) * p.rows + qrow_idx) * p.d_qk * 2);
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 uint4 v[24];
@@ -593,10 +619,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (p.causal) n_vis = min(max(Lb - p.s_q + 1 + s_tok, 0), Lb);
             const int nsplit = p.num_splits[vb + 1] - p.num_splits[vb];
             const int split_idx = (vb == begin_vb) ? begin_split : 0;
+            const size_t slot = static_cast<size_t>(p.num_splits[vb]) + split_idx;  // split partial's workspace slot
             const int n = hi - lo;
             float m_ref = -INFINITY, l_half = 0.f;
 
             if (n > 0 && !q_ready && !(ok = store_q(vb, k))) break;
+            {
+                // The next chunk's Q row goes to L2 now, so storing it later hits L2.
+                ChunkIter peek = chunks;
+                int pvb, plo, phi;
+                while (peek.next(pvb, plo, phi))
+                    if (phi > plo) {
+                        prefetch_q_row(pvb);
+                        break;
+                    }
+            }
             q_ready = false;
 
             for (int j = 0; j < n; ++j) {
@@ -744,20 +781,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // (row, col) sits at row * 32 + (col ^ row): conflict-free in both directions.
                 float* stage = reinterpret_cast<float*>(smem + L::kOffP) + warp * (32 * 32);
                 const int row_base = rg * kRowsPerGroup + 64 * static_cast<int>(cta) + (t & 32);  // warp's first row
-                const size_t slot = static_cast<size_t>(p.num_splits[vb]) + split_idx;
 #pragma unroll 1
-                for (int blk = 0; blk < 8; ++blk) {
-                    const int i = blk >> 2, cb = blk & 3;
-                    const int colw = 256 * i + 128 * h + 32 * cb;  // first d_v column of the block
-                    uint32_t v[32];
+                for (int blk2 = 0; blk2 < 4; ++blk2) {
+                    // two 32-column TMEM loads in flight per wait
+                    uint32_t v2[2][32];
                     if (!empty) {
-                        tmem_ld32(tmem + kTmemO + 128 * i + lane_base + 32 * cb, v);
+                        tmem_ld32(tmem + kTmemO + 64 * blk2 + lane_base, v2[0]);
+                        tmem_ld32(tmem + kTmemO + 64 * blk2 + 32 + lane_base, v2[1]);
                         tmem_wait_ld();
-                        reg_fence(v);
+                        reg_fence(v2[0]);
+                        reg_fence(v2[1]);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = 0;
+                        for (int e = 0; e < 32; ++e) v2[0][e] = v2[1][e] = 0;
                     }
+#pragma unroll
+                for (int half_blk = 0; half_blk < 2; ++half_blk) {
+                    const int blk = 2 * blk2 + half_blk;
+                    const int i = blk >> 2, cb = blk & 3;
+                    const int colw = 256 * i + 128 * h + 32 * cb;  // first d_v column of the block
+                    const uint32_t* v = v2[half_blk];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) stage[lane * 32 + (e ^ lane)] = __uint_as_float(v[e]) * inv_l;
                     __syncwarp();
@@ -784,12 +827,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     __syncwarp();
                 }
+                }
             }
             if (h == 0) {
                 if (nsplit == 1) {
                     if (row_valid) p.lse[static_cast<size_t>(b) * p.rows + row] = lse_v;
                 } else {
-                    const size_t slot = static_cast<size_t>(p.num_splits[vb]) + split_idx;
                     p.lse_accum[slot * kRowsPerGroup + 64 * cta + r] = lse_v;
                 }
             }

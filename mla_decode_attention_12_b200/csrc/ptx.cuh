@@ -146,6 +146,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint3
         : "memory");
 }
 
+// Hint: bring the 128-byte line holding `gaddr` into L2.
+__device__ __forceinline__ void prefetch_l2(const void* gaddr)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(gaddr));
+}
+
 // Asynchronous 16-byte store into another CTA's shared memory; completion is
 // signalled as 16 transaction bytes on that CTA's mbarrier.
 __device__ __forceinline__ void st_async_v4(uint32_t cluster_dst, float a, float b, float c, float d,
