@@ -44,7 +44,7 @@ namespace mla {
 
 constexpr int kPage = 64;
 constexpr int kRowsPerGroup = 128;
-constexpr int kFixedCost = 4;
+constexpr int kFixedCost = 24;  // per-chunk overhead in page units (Q load, epilogue, pipeline refill), tuned on B200
 constexpr int kMdInts = 8;
 
 MLA_HD inline int row_groups(int heads_per_kv) { return (heads_per_kv + kRowsPerGroup - 1) / kRowsPerGroup; }

@@ -6,12 +6,17 @@ sequences still get one (empty) chunk, the split counts in num_splits match the
 chunks, split indices count up from 0 in partition order, and the work is
 balanced.
 """
+import os
+import re
+
 import numpy as np
 import pytest
 
 import mla_decode_attention_12_b200 as mla
 
-FIXED = 4
+_SRC = os.path.join(os.path.dirname(os.path.dirname(__file__)), "mla_decode_attention_12_b200", "csrc",
+                    "scheduler.cuh")
+FIXED = int(re.search(r"constexpr int kFixedCost = (\d+);", open(_SRC).read()).group(1))
 
 
 def pages(L):
