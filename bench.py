@@ -257,6 +257,23 @@ class _Null:
         return False
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """Maximum of a per-rank number over all ranks (the job is as slow as its slowest replica)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_replica: float, world: int, step_ms: float) -> float:
+    """Throughput of N independent replicas, each doing one decode step per step time."""
+    return world * flops_per_replica / (step_ms * 1e-3) / 1e12
+
+
 def roofline(p: W.Problem, t_splitkv_ms: float, peaks, src: str, traffic):
     flops, nbytes = p.flops(), p.io_bytes()
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
@@ -388,11 +405,7 @@ def run_ours(args):
     sampler = ClockSampler(local, getattr(props, "uuid", None) and str(props.uuid))
     t = time_steps(torch, runner, flush, args.steps, args.warmup, barrier, sampler)
     status = runner.status()
-    step_ms = float(t[:, 0].mean())
-    if world > 1:
-        x = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(x, op=dist.ReduceOp.MAX)
-        step_ms = float(x.item())
+    step_ms = max_over_ranks(float(t[:, 0].mean()), device=dev)
     main = workload_line(p, t, peaks, src)
 
     extra = {}
@@ -413,7 +426,7 @@ def run_ours(args):
     base = cpu_baseline(p, args.cpu_seconds) if (rank == 0 and world == 1 and args.cpu_seconds > 0) else None
 
     if rank == 0:
-        value = world * p.flops() / (step_ms * 1e-3) / 1e12
+        value = whole_job_tflops(p.flops(), world, step_ms)
         line = {
             "metric": METRIC,
             "value": round(value, 2),
