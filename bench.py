@@ -9,9 +9,9 @@ pages, shuffled block table, bf16 N(0,1), scale 1/sqrt(576)).  The other four
 decode workloads are timed in the same run and reported under "workloads".
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
-device synchronisation; each step is timed on the launching stream with CUDA
-events around each kernel (each kernel replays its own captured CUDA graph);
-L2 is flushed between steps (a write of 2 x L2), outside the events.  For N > 1 GPUs each rank runs an independent replica
+device synchronisation; each step replays one captured CUDA graph holding the
+three kernels with timing events between them (on the launching stream); L2
+is flushed between steps (a write of 2 x L2), outside the events.  For N > 1 GPUs each rank runs an independent replica
 (the path needs no collective) and rank 0 reports the maximum step time over
 ranks.
 
@@ -208,23 +208,25 @@ class Runner:
                     f()
         torch.cuda.current_stream(dev).wait_stream(s)
         torch.cuda.synchronize(dev)
-        self.graphs = []
-        for f in stages:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
+        # One graph per step: the three kernels with timing events between them (event
+        # record nodes), so a replay costs one launch and the breakdown is exact.
+        self.events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.events[0].record()
+            for i, f in enumerate(stages):
                 f()
-            self.graphs.append(g)
+                self.events[i + 1].record()
         torch.cuda.synchronize(dev)
 
-    def step(self, ev=None):
-        if ev is None:
-            for g in self.graphs:
-                g.replay()
-            return
-        ev[0].record()
-        for i, g in enumerate(self.graphs):
-            g.replay()
-            ev[i + 1].record()
+    def step(self):
+        self.graph.replay()
+
+    def times_ms(self):
+        """(step, metadata, split-KV, combine) of the last replay; call after synchronising."""
+        e = self.events
+        return (e[0].elapsed_time(e[3]), e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
+                e[2].elapsed_time(e[3]))
 
     def status(self):
         return self.mla.read_device_status(self.call.workspace, clear=True)
@@ -234,19 +236,19 @@ def time_steps(torch, runner, flush, steps, warmup, barrier, sampler=None):
     for _ in range(warmup):
         flush.zero_()
         runner.step()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
+    t = []
     ctx = sampler if sampler is not None else _Null()
     with ctx:
-        for i in range(steps):
+        for _ in range(steps):
             flush.zero_()  # L2 flush between steps, outside the events
-            runner.step(evs[i])
-        torch.cuda.synchronize()
+            runner.step()
+            torch.cuda.synchronize()
+            t.append(runner.times_ms())
     barrier()
-    t = np.array([[e[0].elapsed_time(e[3]), e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
-                   e[2].elapsed_time(e[3])] for e in evs])  # ms: step, metadata, splitkv, combine
-    return t
+    return np.array(t)  # ms: step, metadata, splitkv, combine
 
 
 class _Null:
