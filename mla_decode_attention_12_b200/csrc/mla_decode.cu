@@ -70,6 +70,7 @@ constexpr int kQTmemBoxes = 6;         // 64-column boxes of Q kept in tensor me
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 constexpr int kWorkspaceHeader = 256;
+constexpr int kNumMaps = 5;  // tensor maps of the split-KV kernel: Q, K, V, O, split partials
 
 // Shared-memory plan of one CTA (each CTA of the pair owns 64 query rows).
 template <bool kRope>
@@ -126,7 +127,8 @@ struct Ring {
 constexpr int kOffTmemSlot = kBarCount * 8;  // uint32 written by tcgen05.alloc
 constexpr int kOffAbort = kOffTmemSlot + 4;  // int abort flag
 static_assert(kOffAbort + 4 <= Layout<true>::kBarBytes, "barrier area too small");
-static_assert(2 * Layout<true>::kPBytes >= 4 * 32 * 32 * 4, "epilogue staging must fit in the P buffers");
+static_assert(2 * Layout<true>::kPBytes >= 4 * 4096 && 2 * Layout<false>::kPBytes >= 4 * 4096,
+              "epilogue staging (4 KB per softmax warp) must fit in the P buffers");
 static_assert(kTmemQ + 8 * 4 * kQTmemBoxes == kTmemCols, "tensor memory plan");
 static_assert(Layout<true>::kSmemBytes <= 232448 && Layout<false>::kSmemBytes <= 232448,
               "shared memory plan exceeds 227 KB");
@@ -246,7 +248,8 @@ __device__ __forceinline__ int page_of(const DecodeParams& p, const int32_t* tab
 template <bool kRope, bool kFp16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mla_splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const DecodeParams p)
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                       const __grid_constant__ CUtensorMap tm_oacc, const DecodeParams p)
 {
     using L = Layout<kRope>;
     extern __shared__ uint8_t smem_raw[];
@@ -575,23 +578,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint4* qrow = q_row_ptr(qvb, valid);
             if (!wwait(bar(kBarQFree), (kq & 1) ^ 1)) return false;
             tc_fence_after();
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                uint4 v[24];
+            // all 48 loads in flight at once: one memory round trip
+            uint4 v[48];
 #pragma unroll
-                for (int i = 0; i < 24; ++i) v[i] = valid ? __ldg(qrow + 24 * half + i) : make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < 48; ++i) v[i] = valid ? __ldg(qrow + i) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-                for (int c = 0; c < 3; ++c) {
-                    uint32_t w[32];
+            for (int c = 0; c < 6; ++c) {
+                uint32_t w[32];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        w[4 * i] = v[8 * c + i].x;
-                        w[4 * i + 1] = v[8 * c + i].y;
-                        w[4 * i + 2] = v[8 * c + i].z;
-                        w[4 * i + 3] = v[8 * c + i].w;
-                    }
-                    tmem_st32(tmem + kTmemQ + lane_base + 96 * half + 32 * c, w);
+                for (int i = 0; i < 8; ++i) {
+                    w[4 * i] = v[8 * c + i].x;
+                    w[4 * i + 1] = v[8 * c + i].y;
+                    w[4 * i + 2] = v[8 * c + i].z;
+                    w[4 * i + 3] = v[8 * c + i].w;
                 }
+                tmem_st32(tmem + kTmemQ + lane_base + 32 * c, w);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -772,15 +773,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (!(ok = wwait(bar(kBarOFull), k & 1))) break;
                 tc_fence_after();
             }
-            // O leaves tensor memory one 32-column block at a time: each thread holds 32
-            // values of its own row; the warp transposes the 32 x 32 block through shared
-            // memory (the P buffers are idle now) so that global stores write whole
-            // 128-byte row segments instead of one 16-byte piece per row.
+            // O leaves tensor memory 64 columns at a time.  Each warp writes its 32 rows
+            // into a 4 KB tile of shared memory (the P buffers are idle now) in the
+            // 128-byte-swizzled layout of the output tensor maps, and lane 0 hands the
+            // tile to the TMA unit: the global writes proceed asynchronously while the
+            // warp moves on.  A tile is rewritten only after the TMA unit has read it.
             {
-                // 4 KB per warp (the two P buffers hold the four warps' tiles); element
-                // (row, col) sits at row * 32 + (col ^ row): conflict-free in both directions.
-                float* stage = reinterpret_cast<float*>(smem + L::kOffP) + warp * (32 * 32);
-                const int row_base = rg * kRowsPerGroup + 64 * static_cast<int>(cta) + (t & 32);  // warp's first row
+                const uint32_t stage = s_p + warp * 4096;
+                uint8_t* stage_row = smem + L::kOffP + warp * 4096 + lane * 128;
+                const int row_in_group = 64 * static_cast<int>(cta) + (t & 32);  // warp's first row
+                const bool tile_live = rg * kRowsPerGroup + row_in_group < p.rows;
+                auto stage_free = [&]() {
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                };
+                auto stage_issue = [&](const CUtensorMap* map, int x, int y, int z) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && tile_live) {
+                        tma_store_3d(map, stage, x, y, z);
+                        bulk_commit_group();
+                    }
+                };
 #pragma unroll 1
                 for (int blk2 = 0; blk2 < 4; ++blk2) {
                     // two 32-column TMEM loads in flight per wait
@@ -791,43 +805,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         tmem_wait_ld();
                         reg_fence(v2[0]);
                         reg_fence(v2[1]);
+                        if (blk2 == 3) {
+                            // O has left tensor memory: the next chunk's P V may start
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) {
+                                if (leader)
+                                    mbar_arrive(bar(kBarOFree));
+                                else
+                                    mbar_arrive_remote(o_free_lead);
+                            }
+                        }
                     } else {
 #pragma unroll
                         for (int e = 0; e < 32; ++e) v2[0][e] = v2[1][e] = 0;
                     }
+                    const int col0 = 256 * (blk2 >> 1) + 128 * h + 64 * (blk2 & 1);  // first d_v column
+                    if (nsplit == 1) {
+                        // 64 16-bit values of the row: eight 16-byte chunks
+                        stage_free();
 #pragma unroll
-                for (int half_blk = 0; half_blk < 2; ++half_blk) {
-                    const int blk = 2 * blk2 + half_blk;
-                    const int i = blk >> 2, cb = blk & 3;
-                    const int colw = 256 * i + 128 * h + 32 * cb;  // first d_v column of the block
-                    const uint32_t* v = v2[half_blk];
+                        for (int c = 0; c < 8; ++c) {
+                            const uint32_t* v = v2[c >> 2] + 8 * (c & 3);
+                            uint4 w;
+                            w.x = pack2(__uint_as_float(v[0]) * inv_l, __uint_as_float(v[1]) * inv_l, kFp16);
+                            w.y = pack2(__uint_as_float(v[2]) * inv_l, __uint_as_float(v[3]) * inv_l, kFp16);
+                            w.z = pack2(__uint_as_float(v[4]) * inv_l, __uint_as_float(v[5]) * inv_l, kFp16);
+                            w.w = pack2(__uint_as_float(v[6]) * inv_l, __uint_as_float(v[7]) * inv_l, kFp16);
+                            *reinterpret_cast<uint4*>(stage_row + ((c ^ (lane & 7)) << 4)) = w;
+                        }
+                        stage_issue(&tm_o, col0, rg * kRowsPerGroup + row_in_group, b);
+                    } else {
+                        // fp32 partial: two tiles of 32 columns
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) stage[lane * 32 + (e ^ lane)] = __uint_as_float(v[e]) * inv_l;
-                    __syncwarp();
-                    // lane = (row offset within a group of 4 rows) * 8 + (4-column group)
-                    const int cg = lane & 7, rsub = lane >> 3;
-#pragma unroll 2
-                    for (int rr = 0; rr < 32; rr += 4) {
-                        const int lr = rr + rsub;  // row within the warp's 32
-                        const int grow = row_base + lr;
-                        const float* src = stage + lr * 32;
-                        const float a0 = src[(4 * cg + 0) ^ lr], a1 = src[(4 * cg + 1) ^ lr];
-                        const float a2 = src[(4 * cg + 2) ^ lr], a3 = src[(4 * cg + 3) ^ lr];
-                        if (grow < p.rows) {
-                            if (nsplit == 1) {
-                                uint2* dst = reinterpret_cast<uint2*>(
-                                    static_cast<uint8_t*>(p.o) + ((static_cast<size_t>(b) * p.rows + grow) * kDv + colw + 4 * cg) * 2);
-                                *dst = make_uint2(pack2(a0, a1, kFp16), pack2(a2, a3, kFp16));
-                            } else {
-                                float4* dst = reinterpret_cast<float4*>(
-                                    p.o_accum + (slot * kRowsPerGroup + (grow - rg * kRowsPerGroup)) * kDv + colw + 4 * cg);
-                                *dst = make_float4(a0, a1, a2, a3);
+                        for (int hb = 0; hb < 2; ++hb) {
+                            stage_free();
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const uint32_t* v = v2[hb] + 4 * c;
+                                *reinterpret_cast<float4*>(stage_row + ((c ^ (lane & 7)) << 4)) =
+                                    make_float4(__uint_as_float(v[0]) * inv_l, __uint_as_float(v[1]) * inv_l,
+                                                __uint_as_float(v[2]) * inv_l, __uint_as_float(v[3]) * inv_l);
                             }
+                            stage_issue(&tm_oacc, col0 + 32 * hb, row_in_group, static_cast<int>(slot));
                         }
                     }
-                    __syncwarp();
                 }
-                }
+                stage_free();  // the tiles are P buffers again for the next chunk
             }
             if (h == 0) {
                 if (nsplit == 1) {
@@ -836,23 +860,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     p.lse_accum[slot * kRowsPerGroup + 64 * cta + r] = lse_v;
                 }
             }
-            if (!empty) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    if (leader)
-                        mbar_arrive(bar(kBarOFree));
-                    else
-                        mbar_arrive_remote(o_free_lead);
-                }
-                ++k;
-            }
+            if (!empty) ++k;
             g += (n > 0 ? n : 0);
             have = have_next;
             vb = nvb;
             lo = nlo;
             hi = nhi;
         }
+        if (lane == 0) bulk_wait_all();  // output writes complete before the CTA exits
+        __syncwarp();
     }
 
     // ---------------- teardown
@@ -1085,7 +1101,7 @@ static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorM
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    kern<<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], prm);
+    kern<<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], prm);
     return cudaGetLastError();
 }
 
@@ -1251,7 +1267,14 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
         encode_3d(&maps[0], q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 64, prm.box_rows,
                   CU_TENSOR_MAP_SWIZZLE_128B) &&
         encode_2d(&maps[1], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage / 2, CU_TENSOR_MAP_SWIZZLE_128B) &&
-        encode_2d(&maps[2], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B);
+        encode_2d(&maps[2], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B) &&
+        // O: [batch][rows][512] 16-bit, stored in tiles of 64 columns x 32 rows (rows past
+        // the end are clipped by the TMA unit); split partials: [slots][128][512] fp32,
+        // tiles of 32 columns x 32 rows.
+        encode_3d(&maps[3], o, dt, kDv, rows, batch, kDv * 2, static_cast<uint64_t>(kDv) * 2 * rows, 64,
+                  rows < 32 ? rows : 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+        encode_3d(&maps[4], prm.o_accum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kDv, kRowsPerGroup, slots, kDv * 4,
+                  static_cast<uint64_t>(kDv) * 4 * kRowsPerGroup, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
     return ok ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -1292,7 +1315,7 @@ mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, int h_q, i
                                    size_t workspace_bytes, void* stream)
 {
     DecodeParams prm;
-    CUtensorMap maps[3];
+    CUtensorMap maps[kNumMaps];
     mla_status s = prepare_decode(MLA_DECODE_ARGS, prm, maps);
     if (s != MLA_OK || batch == 0) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1309,7 +1332,7 @@ mla_status mla_decode_splitkv(const void* q, int batch, int s_q, int h_q, int d_
                               void* stream)
 {
     DecodeParams prm;
-    CUtensorMap maps[3];
+    CUtensorMap maps[kNumMaps];
     mla_status s = prepare_decode(MLA_DECODE_ARGS, prm, maps);
     if (s != MLA_OK || batch == 0) return s;
     return launch_splitkv_stage(prm, maps, static_cast<cudaStream_t>(stream));
