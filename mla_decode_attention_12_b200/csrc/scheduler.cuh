@@ -9,16 +9,21 @@
 // print the algorithm or the metadata format; this one is our own.
 //
 // Work units.  A "virtual batch" vb = b * row_groups + g is request b restricted
-// to query rows [128 g, 128 g + 128) of its s_q * h_q rows.  Lay the virtual
-// batches on a line of cost units: vb takes kFixedCost units of per-chunk
-// overhead (Q load, epilogue) followed by one unit per 64-token page, starting
-// at C[vb] = sum of the costs before it; W is the total.  Partition p takes the
-// units [p T, (p + 1) T) with T = ceil(W / num_parts).  A unit position x maps to
-// the page position (vb, blk) with vb the virtual batch whose span holds x and
-// blk = clamp(x - C[vb] - kFixedCost, 0, pages(vb)); partition p covers the page
-// positions from map(p T) up to map((p + 1) T).  A virtual batch whose pages are
-// cut by partition starts is split; every partition computes its range on its
-// own, so the device version is one thread per partition.
+// to query rows [128 g, 128 g + 128) of its s_q * h_q rows.  Every chunk (one
+// partition's share of one virtual batch) costs F = kFixedCost units of
+// overhead (Q load, pipeline refill, epilogue) plus one unit per 64-token page.
+// Lay the virtual batches on a line: vb takes F units followed by its pages,
+// starting at C[vb] = sum of the costs before it; W is the total.  A partition
+// that starts inside a virtual batch's pages opens one more chunk than the line
+// shows, so it gets F units fewer of the line: with D = ceil((W - F) / num_parts),
+// partition 0 takes the line units [0, F + D) and partition p >= 1 the units
+// [F + p D, F + (p + 1) D); each partition's cost (pages + F per chunk) is then
+// at most F + D.  A unit position x maps to the page position (vb, blk) with vb
+// the virtual batch whose span holds x and blk = clamp(x - C[vb] - F, 0,
+// pages(vb)); partition p covers the page positions from map(start p) up to
+// map(start p+1).  A virtual batch whose pages are cut by partition starts is
+// split; every partition computes its range on its own, so the device version
+// is one thread per partition.
 //
 // Output:
 //   md[p * 8 + 0..4] = begin_vb, begin_blk, end_vb, end_blk, begin_split
@@ -44,7 +49,7 @@ namespace mla {
 
 constexpr int kPage = 64;
 constexpr int kRowsPerGroup = 128;
-constexpr int kFixedCost = 24;  // per-chunk overhead in page units (Q load, epilogue, pipeline refill), tuned on B200
+constexpr int kFixedCost = 16;  // per-chunk overhead in page units (Q load, epilogue, pipeline refill), tuned on B200
 constexpr int kMdInts = 8;
 
 MLA_HD inline int row_groups(int heads_per_kv) { return (heads_per_kv + kRowsPerGroup - 1) / kRowsPerGroup; }
@@ -56,11 +61,12 @@ MLA_HD inline int pages_of(int seqlen) { return seqlen <= 0 ? 0 : (seqlen + kPag
 MLA_HD inline void unit_to_page(long long x, const long long* C, const int32_t* pages, int nv, long long total,
                                 int& vb, int& blk)
 {
-    if (x >= total) {
+    if (x >= total || nv == 0) {
         vb = nv;
         blk = 0;
         return;
     }
+    if (x < 0) x = 0;
     int lo = 0, hi = nv - 1;  // largest v with C[v] <= x
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -80,14 +86,16 @@ MLA_HD inline void unit_to_page(long long x, const long long* C, const int32_t* 
 MLA_HD inline void partition_range(int p, int num_parts, const long long* C, const int32_t* pages, int nv,
                                    long long total, int32_t* m)
 {
-    const long long T = (total + num_parts - 1) / num_parts;
+    long long D = (total - kFixedCost + num_parts - 1) / num_parts;  // line units of a partition after its first F
+    if (D < 0) D = 0;
+    auto start = [&](int q) -> long long { return q == 0 ? 0 : kFixedCost + static_cast<long long>(q) * D; };
     int bv, bb, ev, eb;
-    unit_to_page(static_cast<long long>(p) * T, C, pages, nv, total, bv, bb);
+    unit_to_page(start(p), C, pages, nv, total, bv, bb);
     if (p == num_parts - 1) {
         ev = nv;
         eb = 0;
     } else {
-        unit_to_page(static_cast<long long>(p + 1) * T, C, pages, nv, total, ev, eb);
+        unit_to_page(start(p + 1), C, pages, nv, total, ev, eb);
     }
     m[0] = bv;
     m[1] = bb;

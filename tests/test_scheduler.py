@@ -63,13 +63,14 @@ def check_schedule(seqlens, heads_per_kv, num_parts):
         assert len(lst) == ns[vb + 1] - ns[vb] >= 1
         assert [s for _, _, s in lst] == list(range(len(lst)))
         assert [lo for _, lo, _ in lst] == sorted(lo for _, lo, _ in lst)
-    # balance: every partition but the last stays within its budget T
+    # balance: every partition's cost, pages plus the fixed cost of each of its
+    # chunks, stays within the budget F + ceil((W - F) / num_parts)
     W = sum((pages(L) + FIXED) * groups for L in seqlens)
-    T = -(-W // num_parts) + FIXED
+    T = max(-(-(W - FIXED) // num_parts), 0) + FIXED
     cost = np.zeros(num_parts, np.int64)
     for p, vb, lo, hi, _ in ch:
         cost[p] += (hi - lo) + FIXED
-    assert cost[:-1].max(initial=0) <= T
+    assert cost.max(initial=0) <= T
     return md, ns, cost, T
 
 
