@@ -208,34 +208,55 @@ class Runner:
                     f()
         torch.cuda.current_stream(dev).wait_stream(s)
         torch.cuda.synchronize(dev)
-        # One graph per step: the three kernels with timing events between them (event
-        # record nodes), so a replay costs one launch and the breakdown is exact.
-        self.events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        # Two graphs of one step each, so a replay costs one launch.  The step graph has
+        # timing events only around the three kernels: consecutive kernels keep their
+        # programmatic launch edges, so each one's set-up overlaps the previous one's end.
+        # The staged graph has an event between kernels (event record nodes serialise
+        # them) and gives each kernel's own duration.
+        self.events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph):
             self.events[0].record()
+            for f in stages:
+                f()
+            self.events[1].record()
+        self.stage_events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        self.stage_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.stage_graph):
+            self.stage_events[0].record()
             for i, f in enumerate(stages):
                 f()
-                self.events[i + 1].record()
+                self.stage_events[i + 1].record()
         torch.cuda.synchronize(dev)
 
     def step(self):
         self.graph.replay()
 
+    def step_staged(self):
+        self.stage_graph.replay()
+
     def times_ms(self):
-        """(step, metadata, split-KV, combine) of the last replay; call after synchronising."""
-        e = self.events
-        return (e[0].elapsed_time(e[3]), e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
-                e[2].elapsed_time(e[3]))
+        """Duration of the last step replay; call after synchronising."""
+        return self.events[0].elapsed_time(self.events[1])
+
+    def stage_times_ms(self):
+        """(metadata, split-KV, combine) of the last staged replay; call after synchronising."""
+        e = self.stage_events
+        return (e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]))
 
     def status(self):
         return self.mla.read_device_status(self.call.workspace, clear=True)
 
 
-def time_steps(torch, runner, flush, steps, warmup, barrier, sampler=None):
+def time_steps(torch, runner, flush, steps, warmup, barrier, sampler=None, staged_steps=None):
+    """Times `steps` step replays (after `warmup`), then `staged_steps` staged replays for
+    the per-kernel breakdown.  Returns ms rows: step, metadata, split-KV, combine (the
+    breakdown columns come from the staged replays, cycled over the step rows)."""
     for _ in range(warmup):
         flush.zero_()
         runner.step()
+        flush.zero_()
+        runner.step_staged()
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -248,7 +269,17 @@ def time_steps(torch, runner, flush, steps, warmup, barrier, sampler=None):
             torch.cuda.synchronize()
             t.append(runner.times_ms())
     barrier()
-    return np.array(t)  # ms: step, metadata, splitkv, combine
+    st = []
+    for _ in range(min(steps, 100) if staged_steps is None else staged_steps):
+        flush.zero_()
+        runner.step_staged()
+        torch.cuda.synchronize()
+        st.append(runner.stage_times_ms())
+    st = np.array(st)
+    rows = np.zeros((len(t), 4))
+    rows[:, 0] = t
+    rows[:, 1:] = st[np.arange(len(t)) % len(st)]
+    return rows  # ms: step, metadata, splitkv, combine
 
 
 class _Null:
@@ -450,7 +481,9 @@ def run_ours(args):
             "kv_gbs": main["kv_gbs"],
             "tflops": main["tflops"],
             "breakdown_us": {"metadata": main["us_metadata"], "splitkv": main["us_splitkv"],
-                             "combine": main["us_combine"]},
+                             "combine": main["us_combine"],
+                             "note": "each kernel alone: replays with an event between kernels, "
+                                     "which removes the launch overlap the timed steps have"},
             "roofline": main["roofline"],
             "cpu_baseline": base,
             "e2e": e2e_line,

@@ -270,23 +270,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int part = blockIdx.x >> 1;
     auto lead_bar = [&](int slot) { return map_to_cta(bar(slot), 0); };  // leader's barrier, cluster address
 
-    // The first chunk's query rows start moving into L2 before the set-up.
-    if (warp < 4) {
-        const int32_t* md0 = p.md + part * kMdInts;
-        ChunkIter first{md0[0], md0[1], md0[2], md0[3], p.groups, p.seqlens};
-        int fvb, flo, fhi;
-        while (first.next(fvb, flo, fhi))
-            if (fhi > flo) {
-                const int qrow_idx = (fvb % p.groups) * kRowsPerGroup + 64 * static_cast<int>(cta) + (threadIdx.x & 63);
-                if (qrow_idx < p.rows) {
-                    const uint8_t* a = static_cast<const uint8_t*>(p.q) +
-                                       (static_cast<size_t>(fvb / p.groups) * p.rows + qrow_idx) * p.d_qk * 2;
-                    for (int i = 0; i < 6; ++i) prefetch_l2(a + 128 * i);
-                }
-                break;
-            }
-    }
-
     // ---------------- set-up
     if (threadIdx.x == 0) {
         mbar_init(bar(kBarQFull), 1 + 8);
@@ -331,6 +314,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     cluster_sync();  // both CTAs' barriers initialised before any remote arrive / transaction
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kOffBar + kOffTmemSlot);
+    // The set-up above touched no global memory, so it may overlap the grid before this
+    // one (the metadata kernel); everything below may read what that grid wrote.
+    grid_dependency_wait();
+    grid_launch_dependents();
 
     Sync sync{s_bar + kOffAbort, map_to_cta(s_bar + kOffAbort, cta ^ 1u), p.status};
     const int32_t* md = p.md + part * kMdInts;
@@ -890,6 +877,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 template <bool kFp16>
 __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
 {
+    grid_dependency_wait();  // the split partials of the split-KV grid
     const int vb = blockIdx.x;
     const int slot0 = p.num_splits[vb];
     const int nsplit = p.num_splits[vb + 1] - slot0;
@@ -988,6 +976,8 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
                                                                     int num_parts, int32_t* md, int32_t* num_splits)
 {
     extern __shared__ __align__(16) uint8_t meta_smem[];
+    grid_dependency_wait();
+    grid_launch_dependents();  // the split-KV grid sets up while the schedule is computed
     __shared__ long long warp_tot_ll[32];
     __shared__ int warp_tot_i[32];
     const int nv = batch * groups;
@@ -1080,6 +1070,22 @@ static bool encode_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dt
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch configuration with programmatic stream serialization: the grid may start
+// while the previous one in the stream finishes; each kernel calls
+// grid_dependency_wait() before it reads global memory that grid could have written.
+static void programmatic_launch(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, dim3 grid, dim3 block,
+                                size_t smem, cudaStream_t stream)
+{
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+}
+
 static size_t workspace_slots(int batch, int groups, int num_parts)
 {
     return static_cast<size_t>(batch) * groups + static_cast<size_t>(num_parts);
@@ -1101,8 +1107,10 @@ static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorM
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    kern<<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], prm);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    programmatic_launch(cfg, attr, dim3(grid), dim3(kThreads), smem, stream);
+    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], prm);
 }
 
 }  // namespace mla
@@ -1185,9 +1193,12 @@ mla_status mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_p
             configured_device = dev;
         }
     }
-    mla_metadata_kernel<<<1, kMetaThreads, smem, static_cast<cudaStream_t>(stream)>>>(
-        cache_seqlens, batch, row_groups(heads_per_kv), num_parts, tile_md, num_splits);
-    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    programmatic_launch(cfg, attr, dim3(1), dim3(kMetaThreads), smem, static_cast<cudaStream_t>(stream));
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, mla_metadata_kernel, cache_seqlens, batch, row_groups(heads_per_kv),
+                                             num_parts, tile_md, num_splits);
+    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 size_t mla_decode_workspace_bytes(int batch, int s_q, int h_q, int h_kv, int num_parts)
@@ -1295,11 +1306,12 @@ static mla_status launch_combine_stage(const DecodeParams& prm, cudaStream_t st)
 {
     const int rows_max = prm.rows < kRowsPerGroup ? prm.rows : kRowsPerGroup;
     dim3 cgrid(prm.batch * prm.groups, (rows_max + 3) / 4);
-    if (prm.dtype == MLA_FP16)
-        mla_combine_kernel<true><<<cgrid, 128, 0, st>>>(prm);
-    else
-        mla_combine_kernel<false><<<cgrid, 128, 0, st>>>(prm);
-    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    programmatic_launch(cfg, attr, cgrid, dim3(128), 0, st);
+    const cudaError_t e = prm.dtype == MLA_FP16 ? cudaLaunchKernelEx(&cfg, mla_combine_kernel<true>, prm)
+                                                : cudaLaunchKernelEx(&cfg, mla_combine_kernel<false>, prm);
+    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 #define MLA_DECODE_ARGS                                                                                          \

@@ -162,6 +162,13 @@ __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bu
 // Wait until the bulk stores of this thread are complete.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Programmatic dependent launch.  wait: block until the grid launched before this one
+// in the stream has completed and its memory writes are visible (returns at once when
+// this grid was not launched with programmatic serialization).  launch_dependents:
+// let the next grid in the stream, if it opted in, start launching now.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Hint: bring the 128-byte line holding `gaddr` into L2.
 __device__ __forceinline__ void prefetch_l2(const void* gaddr)
 {

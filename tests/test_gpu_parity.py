@@ -71,6 +71,16 @@ def test_parity_few_partitions(oracle_mod, parts):
     print(compare(o, lse, o_ref, lse_ref, p.dtype, f"parts={parts}"))
 
 
+@pytest.mark.parametrize("parts", [1, 2])
+def test_parity_leading_empty_chunks(oracle_mod, parts):
+    # A partition whose first chunks are empty sequences: the first non-empty
+    # chunk's Q, loaded while the kernel sets up, must reach that chunk.
+    p = W.make_problem([0, 0, 700, 0, 130, 0], s_q=1, h_q=32, causal=False, seed=130 + parts)
+    o, lse, md, ns = run_gpu(p, num_parts=parts)
+    o_ref, lse_ref = oracle_full(oracle_mod, p)
+    print(compare(o, lse, o_ref, lse_ref, p.dtype, f"leading empty, parts={parts}"))
+
+
 def test_metadata_kernel_matches_host_schedule():
     rng = np.random.default_rng(7)
     for hpk in (16, 128, 256):
