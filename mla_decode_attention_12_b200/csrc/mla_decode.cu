@@ -871,10 +871,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------ combine kernel
 // Merges the split partial results of every virtual batch with more than one
 // split: lse = log sum_k exp(lse_k), o = sum_k exp(lse_k - lse) o_k (the exact
-// identity behind split-KV).  One warp per query row, 4 rows per CTA; lane i
-// owns 16 of the 512 output columns; the split weights are computed 32 at a
-// time (one per lane) and broadcast with shuffles.
-template <bool kFp16>
+// identity behind split-KV).  Two layouts of the same sum, chosen on the host:
+//  * few splits per virtual batch: one warp per query row, 4 rows per CTA; lane i
+//    owns 16 of the 512 output columns and walks the splits in order;
+//  * many splits (few virtual batches, long sequences): one CTA per row, warp w
+//    sums splits w, w + 4, ... and the four partial sums are added through shared
+//    memory, so a row's splits are read four at a time.
+template <bool kFp16, bool kSplitParallel>
 __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
 {
     grid_dependency_wait();  // the split partials of the split-KV grid
@@ -884,9 +887,9 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
     if (nsplit <= 1) return;
     const int b = vb / p.groups, rg = vb % p.groups;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = blockIdx.y * 4 + warp;
+    const int r = kSplitParallel ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y) * 4 + warp;
     const int rows_here = min(kRowsPerGroup, p.rows - rg * kRowsPerGroup);
-    if (r >= rows_here) return;
+    if (r >= rows_here) return;  // uniform over the CTA in the split-parallel layout
     const float* lse_k = p.lse_accum + static_cast<size_t>(slot0) * kRowsPerGroup + r;
     float mx = -INFINITY;
     for (int k = lane; k < nsplit; k += 32) mx = fmaxf(mx, lse_k[static_cast<size_t>(k) * kRowsPerGroup]);
@@ -898,33 +901,54 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
 #pragma unroll
     for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float lse = (mx == -INFINITY) ? -INFINITY : mx + logf(sum);
-    float acc[16];
+    float4 acc[4];  // float4 columns lane, lane + 32, lane + 64, lane + 96
 #pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto add_split = [&](const float4* s4, float w) {
+        const float4 v0 = s4[0], v1 = s4[32], v2 = s4[64], v3 = s4[96];
+        acc[0].x += w * v0.x; acc[0].y += w * v0.y; acc[0].z += w * v0.z; acc[0].w += w * v0.w;
+        acc[1].x += w * v1.x; acc[1].y += w * v1.y; acc[1].z += w * v1.z; acc[1].w += w * v1.w;
+        acc[2].x += w * v2.x; acc[2].y += w * v2.y; acc[2].z += w * v2.z; acc[2].w += w * v2.w;
+        acc[3].x += w * v3.x; acc[3].y += w * v3.y; acc[3].z += w * v3.z; acc[3].w += w * v3.w;
+    };
     if (mx != -INFINITY) {
         const float4* src = reinterpret_cast<const float4*>(p.o_accum + (static_cast<size_t>(slot0) * kRowsPerGroup + r) * kDv) + lane;
         const size_t stride4 = static_cast<size_t>(kRowsPerGroup) * kDv / 4;  // float4s between splits
-        for (int kb = 0; kb < nsplit; kb += 32) {
-            const int k = kb + lane;
-            const float w_mine = (k < nsplit) ? expf(lse_k[static_cast<size_t>(k) * kRowsPerGroup] - lse) : 0.f;
-            const int cnt = min(32, nsplit - kb);
+        if (kSplitParallel) {
+#pragma unroll 2
+            for (int k = warp; k < nsplit; k += 4)
+                add_split(src + static_cast<size_t>(k) * stride4, expf(lse_k[static_cast<size_t>(k) * kRowsPerGroup] - lse));
+        } else {
+            for (int kb = 0; kb < nsplit; kb += 32) {
+                const int k = kb + lane;
+                const float w_mine = (k < nsplit) ? expf(lse_k[static_cast<size_t>(k) * kRowsPerGroup] - lse) : 0.f;
+                const int cnt = min(32, nsplit - kb);
 #pragma unroll 4
-            for (int kk = 0; kk < cnt; ++kk) {
-                const float w = __shfl_sync(0xffffffffu, w_mine, kk);
-                const float4* s4 = src + static_cast<size_t>(kb + kk) * stride4;
-                const float4 v0 = s4[0], v1 = s4[32], v2 = s4[64], v3 = s4[96];
-                acc[0] += w * v0.x; acc[1] += w * v0.y; acc[2] += w * v0.z; acc[3] += w * v0.w;
-                acc[4] += w * v1.x; acc[5] += w * v1.y; acc[6] += w * v1.z; acc[7] += w * v1.w;
-                acc[8] += w * v2.x; acc[9] += w * v2.y; acc[10] += w * v2.z; acc[11] += w * v2.w;
-                acc[12] += w * v3.x; acc[13] += w * v3.y; acc[14] += w * v3.z; acc[15] += w * v3.w;
+                for (int kk = 0; kk < cnt; ++kk)
+                    add_split(src + static_cast<size_t>(kb + kk) * stride4, __shfl_sync(0xffffffffu, w_mine, kk));
             }
         }
+    }
+    if (kSplitParallel) {
+        __shared__ float4 part[3][128];  // warps 1-3's sums
+        if (warp > 0)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) part[warp - 1][lane + 32 * i] = acc[i];
+        __syncthreads();
+        if (warp != 0) return;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int w = 0; w < 3; ++w) {
+                const float4 o = part[w][lane + 32 * i];
+                acc[i].x += o.x; acc[i].y += o.y; acc[i].z += o.z; acc[i].w += o.w;
+            }
     }
     const int row = rg * kRowsPerGroup + r;
     uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.o) + (static_cast<size_t>(b) * p.rows + row) * kDv * 2);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        dst[lane + 32 * i] = make_uint2(pack2(acc[4 * i], acc[4 * i + 1], kFp16), pack2(acc[4 * i + 2], acc[4 * i + 3], kFp16));
+        dst[lane + 32 * i] = make_uint2(pack2(acc[i].x, acc[i].y, kFp16), pack2(acc[i].z, acc[i].w, kFp16));
     if (lane == 0) p.lse[static_cast<size_t>(b) * p.rows + row] = lse;
 }
 
@@ -1305,12 +1329,21 @@ static mla_status launch_splitkv_stage(const DecodeParams& prm, const CUtensorMa
 static mla_status launch_combine_stage(const DecodeParams& prm, cudaStream_t st)
 {
     const int rows_max = prm.rows < kRowsPerGroup ? prm.rows : kRowsPerGroup;
-    dim3 cgrid(prm.batch * prm.groups, (rows_max + 3) / 4);
+    // Fewer than one virtual batch per 4 partitions means many splits per virtual batch
+    // (long sequences): read each row's splits in parallel.
+    const long long nv = static_cast<long long>(prm.batch) * prm.groups;
+    const bool split_parallel = 4 * nv < prm.num_parts;
+    dim3 cgrid(static_cast<unsigned>(nv), split_parallel ? rows_max : (rows_max + 3) / 4);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     programmatic_launch(cfg, attr, cgrid, dim3(128), 0, st);
-    const cudaError_t e = prm.dtype == MLA_FP16 ? cudaLaunchKernelEx(&cfg, mla_combine_kernel<true>, prm)
-                                                : cudaLaunchKernelEx(&cfg, mla_combine_kernel<false>, prm);
+    cudaError_t e;
+    if (prm.dtype == MLA_FP16)
+        e = split_parallel ? cudaLaunchKernelEx(&cfg, mla_combine_kernel<true, true>, prm)
+                           : cudaLaunchKernelEx(&cfg, mla_combine_kernel<true, false>, prm);
+    else
+        e = split_parallel ? cudaLaunchKernelEx(&cfg, mla_combine_kernel<false, true>, prm)
+                           : cudaLaunchKernelEx(&cfg, mla_combine_kernel<false, false>, prm);
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -1372,6 +1405,7 @@ mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int
     prm.groups = groups;
     prm.batch = batch;
     prm.dtype = dtype;
+    prm.num_parts = num_parts;
     prm.lse_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader);
     prm.o_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader +
                                            align_up(slots * kRowsPerGroup * sizeof(float), 256));
