@@ -994,7 +994,7 @@ __device__ void block_exclusive_scan(T* data, int n, T* warp_tot, T& total)
 
 // One CTA of kMetaThreads threads.  Dynamic shared memory: C [nv] int64,
 // pages [nv] int32, extra-split counts [nv] int32, begins [num_parts] int32 x 2.
-constexpr int kMetaThreads = 1024;
+constexpr int kMetaThreads = 256;
 
 __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_t* seqlens, int batch, int groups,
                                                                     int num_parts, int32_t* md, int32_t* num_splits)
