@@ -854,7 +854,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             lo = nlo;
             hi = nhi;
         }
-        if (lane == 0) bulk_wait_all();  // output writes complete before the CTA exits
+        // Shared memory must outlive the TMA unit's reads of the output tiles; the writes
+        // themselves are complete, and visible to the next grid, when the grid completes.
+        if (lane == 0) bulk_wait_read_all();
         __syncwarp();
     }
 
