@@ -81,6 +81,23 @@ def test_parity_leading_empty_chunks(oracle_mod, parts):
     print(compare(o, lse, o_ref, lse_ref, p.dtype, f"leading empty, parts={parts}"))
 
 
+@pytest.mark.parametrize("name,parts", [("long_split_like", None), ("compute_like", None), ("few_parts", 3)])
+def test_two_stage_calls_match_single_call(name, parts):
+    # mla_decode_splitkv followed by mla_decode_combine is the same computation as
+    # mla_decode_with_kvcache: bit-identical O and LSE.  The cases cover both combine
+    # layouts (many splits per virtual batch, and few).
+    p = (W.make_problem([2500, 64, 0, 700, 1, 130], s_q=2, h_q=64, causal=True, seed=140)
+         if name == "few_parts" else SMALL[name]())
+    o1, lse1, md, ns = run_gpu(p, num_parts=parts)
+    q, kv, bt, sl = to_device(p)
+    call = mla.DecodeCall(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale)
+    call.splitkv()
+    call.combine()
+    torch.cuda.synchronize()
+    assert int(ns[-1].item()) > ns.numel() - 1, "the case must split some sequence"
+    assert torch.equal(call.out, o1) and torch.equal(call.lse, lse1)
+
+
 def test_metadata_kernel_matches_host_schedule():
     rng = np.random.default_rng(7)
     for hpk in (16, 128, 256):
