@@ -195,8 +195,9 @@ class Runner:
         self.ns = torch.zeros(n_ns, dtype=torch.int32, device=dev)
         mla.get_mla_metadata(self.sl, self.rows, 1, out=(self.md, self.ns))
         ws = torch.zeros(mla.workspace_bytes(p.batch, p.s_q, p.h_q, 1, parts), dtype=torch.uint8, device=dev)
+        # padding heads (the spec_padded workload) are declared, so their outputs are skipped
         self.call = mla.DecodeCall(self.q, self.kv, self.bt, self.sl, p.dv, self.md, self.ns, causal=p.causal,
-                                   softmax_scale=p.scale, workspace=ws)
+                                   softmax_scale=p.scale, workspace=ws, active_heads=p.active_heads)
         self.launches_per_step = 3
         stages = [lambda: mla.get_mla_metadata(self.sl, self.rows, 1, out=(self.md, self.ns)),
                   self.call.splitkv, self.call.combine]

@@ -145,8 +145,17 @@ MLA_API size_t mla_decode_workspace_bytes(int batch, int s_q, int h_q, int h_kv,
  *   tile_md, num_splits, num_parts   from mla_get_metadata for this batch
  *   causal          0 or 1
  *   softmax_scale   > 0, or <= 0 for 1/sqrt(d_qk)
+ *   active_heads    heads [0, active_heads) are real, heads [active_heads, h_q) are
+ *                   padding ("FlashMLA vLLM Optimization" page, active-head switch: a
+ *                   tensor-parallel rank's query is padded to h_q heads of which it
+ *                   consumes only a few).  Padding heads are still computed inside the
+ *                   MMA tiles, but their o and lse are left as they were and the
+ *                   combine skips them.  A value that is not a multiple of 8 in
+ *                   (0, h_q] (0 included), or an h_q that is not a multiple of 8,
+ *                   means every head is real.
  *   o               device [batch, s_q, h_q, 512], dtype `dtype`, 16-byte aligned, written
- *   lse             device float32 [batch, s_q, h_q], written
+ *                   (real heads)
+ *   lse             device float32 [batch, s_q, h_q], written (real heads)
  *   workspace       device, >= mla_decode_workspace_bytes(...), 256-byte aligned
  * Enqueues the split-KV kernel and the combine kernel on `stream`.  Calls
  * sharing one workspace must not run concurrently.
@@ -157,8 +166,8 @@ MLA_API mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, in
                                    const int32_t* cache_seqlens, int dv, int dtype,
                                    const int32_t* tile_md, int num_parts,
                                    const int32_t* num_splits, int causal, float softmax_scale,
-                                   void* o, float* lse, void* workspace, size_t workspace_bytes,
-                                   void* stream);
+                                   int active_heads, void* o, float* lse, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /*
  * The two stages of mla_decode_with_kvcache, for callers that schedule or time
@@ -173,8 +182,8 @@ MLA_API mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, in
  *   in the workspace.
  * mla_decode_combine: merges those partial results into o / lse
  *   (lse = log sum_k exp(lse_k), o = sum_k exp(lse_k - lse) o_k); batch, s_q,
- *   h_q, h_kv, dv, dtype, num_splits, num_parts, o, lse and workspace must be
- *   the ones given to mla_decode_splitkv.
+ *   h_q, h_kv, dv, dtype, num_splits, num_parts, active_heads, o, lse and
+ *   workspace must be the ones given to mla_decode_splitkv.
  */
 MLA_API mla_status mla_decode_splitkv(const void* q, int batch, int s_q, int h_q, int d_qk,
                                       const void* kvcache, int num_blocks, int page_size, int h_kv,
@@ -182,12 +191,13 @@ MLA_API mla_status mla_decode_splitkv(const void* q, int batch, int s_q, int h_q
                                       const int32_t* cache_seqlens, int dv, int dtype,
                                       const int32_t* tile_md, int num_parts,
                                       const int32_t* num_splits, int causal, float softmax_scale,
-                                      void* o, float* lse, void* workspace, size_t workspace_bytes,
-                                      void* stream);
+                                      int active_heads, void* o, float* lse, void* workspace,
+                                      size_t workspace_bytes, void* stream);
 
 MLA_API mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int dtype,
-                                      const int32_t* num_splits, int num_parts, void* o, float* lse,
-                                      void* workspace, size_t workspace_bytes, void* stream);
+                                      const int32_t* num_splits, int num_parts, int active_heads,
+                                      void* o, float* lse, void* workspace, size_t workspace_bytes,
+                                      void* stream);
 
 /*
  * Reads the device status word of a workspace (synchronises `stream`).
@@ -230,7 +240,8 @@ MLA_API mla_status mla_decode_with_kvcache_noalloc(const void* q, int batch, int
                                                    int max_blocks_per_seq, const int32_t* cache_seqlens,
                                                    int dv, int dtype, const int32_t* tile_md,
                                                    int num_parts, const int32_t* num_splits, int causal,
-                                                   float softmax_scale, void* o, float* lse, void* stream);
+                                                   float softmax_scale, int active_heads, void* o, float* lse,
+                                                   void* stream);
 
 #ifdef __cplusplus
 }

@@ -37,13 +37,14 @@ SIGNATURES = {
                                  _P, _I, _I, _I,              # kvcache, num_blocks, page_size, h_kv
                                  _P, _I, _P, _I, _I,          # block_table, max_blocks, seqlens, dv, dtype
                                  _P, _I, _P, _I, _F,          # tile_md, num_parts, num_splits, causal, scale
+                                 _I,                          # active_heads
                                  _P, _P, _P, _SZ, _P], _I),   # o, lse, workspace, ws_bytes, stream
     "mla_decode_splitkv": ([_P, _I, _I, _I, _I, _P, _I, _I, _I, _P, _I, _P, _I, _I,
-                            _P, _I, _P, _I, _F, _P, _P, _P, _SZ, _P], _I),
-    "mla_decode_combine": ([_I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _SZ, _P], _I),
+                            _P, _I, _P, _I, _F, _I, _P, _P, _P, _SZ, _P], _I),
+    "mla_decode_combine": ([_I, _I, _I, _I, _I, _I, _P, _I, _I, _P, _P, _P, _SZ, _P], _I),
     "mla_read_device_status": ([_P, _I, ctypes.POINTER(_I), _P], _I),
     "mla_decode_with_kvcache_noalloc": ([_P, _I, _I, _I, _I, _P, _I, _I, _I, _P, _I, _P, _I, _I,
-                                         _P, _I, _P, _I, _F, _P, _P, _P], _I),
+                                         _P, _I, _P, _I, _F, _I, _P, _P, _P], _I),
 }
 
 _lock = threading.Lock()

@@ -111,7 +111,7 @@ class DecodeCall:
     """Marshalled arguments of one decode call (device tensors), reusable across stages."""
 
     def __init__(self, q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata, num_splits,
-                 causal=False, softmax_scale=None, workspace=None, out=None, lse=None):
+                 causal=False, softmax_scale=None, workspace=None, out=None, lse=None, active_heads=None):
         dev = q.device
         if q.dtype not in _DTYPES or kvcache.dtype != q.dtype:
             raise ValueError("q and kvcache must both be bfloat16 or both float16")
@@ -137,12 +137,13 @@ class DecodeCall:
         self.device = dev
         self.out, self.lse, self.workspace = out, lse, workspace
         self._keep = (q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits)
+        active = 0 if active_heads is None else int(active_heads)  # 0: every head is real
         self.args = (_ptr(q), b, s_q, h_q, d_qk, _ptr(kvcache), num_blocks, page, h_kv, _ptr(block_table),
                      block_table.shape[1], _ptr(cache_seqlens), dv, _DTYPES[q.dtype],
                      _ptr(tile_scheduler_metadata), num_parts, _ptr(num_splits), int(bool(causal)), scale,
-                     _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel())
-        self.combine_args = (b, s_q, h_q, h_kv, dv, _DTYPES[q.dtype], _ptr(num_splits), num_parts, _ptr(out),
-                             _ptr(lse), _ptr(workspace), workspace.numel())
+                     active, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel())
+        self.combine_args = (b, s_q, h_q, h_kv, dv, _DTYPES[q.dtype], _ptr(num_splits), num_parts, active,
+                             _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel())
 
     def run(self):
         """Split-KV kernel then combine kernel (mla_decode_with_kvcache)."""
@@ -165,8 +166,11 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
                            cache_seqlens: torch.Tensor, dv: int, tile_scheduler_metadata: torch.Tensor,
                            num_splits: torch.Tensor, causal: bool = False, softmax_scale: float | None = None,
                            workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
-                           lse: torch.Tensor | None = None):
+                           lse: torch.Tensor | None = None, active_heads: int | None = None):
     """MLA decode over a paged cache; returns ``(o [b, s_q, h_q, dv], lse [b, s_q, h_q] float32)``.
+
+    ``active_heads``: heads ``[active_heads, h_q)`` are padding whose outputs are not
+    written (a multiple of 8 no larger than ``h_q``; anything else means all heads).
 
     ``q`` [b, s_q, h_q, d_qk] and ``kvcache`` [num_blocks, 64, h_kv, d_qk] are bf16 or
     fp16; ``block_table`` [b, max_blocks] and ``cache_seqlens`` [b] are int32.  With
@@ -181,7 +185,8 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
             t.to(dev, non_blocking=nb) for t in
             (q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits))
     call = DecodeCall(q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata, num_splits,
-                      causal=causal, softmax_scale=softmax_scale, workspace=workspace, out=out, lse=lse)
+                      causal=causal, softmax_scale=softmax_scale, workspace=workspace, out=out, lse=lse,
+                      active_heads=active_heads)
     out, lse = call.run()
     if host:
         return out.cpu(), lse.cpu()

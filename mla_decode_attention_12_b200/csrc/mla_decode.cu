@@ -70,7 +70,8 @@ constexpr int kQTmemBoxes = 6;         // 64-column boxes of Q kept in tensor me
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 constexpr int kWorkspaceHeader = 256;
-constexpr int kNumMaps = 5;  // tensor maps of the split-KV kernel: Q, K, V, O, split partials
+constexpr int kNumMaps = 7;  // tensor maps of the split-KV kernel: Q, K, V, O, split partials, and O and
+                             // split partials with 8-row boxes
 
 // Shared-memory plan of one CTA (each CTA of the pair owns 64 query rows).
 template <bool kRope>
@@ -150,6 +151,7 @@ struct DecodeParams {
     float* lse_accum;   // [slots, 128]
     int* status;
     int batch, s_q, h_q, rows, groups, max_blocks, num_blocks, causal, box_rows;
+    int active_heads;  // heads >= active_heads are padding: not written, not combined
     float scale_log2;
     int dtype, d_qk, num_parts;  // host-side dispatch only
 };
@@ -245,11 +247,12 @@ __device__ __forceinline__ int page_of(const DecodeParams& p, const int32_t* tab
 //   O   columns [0, 256):  d_v chunk i (256 wide) at [128 i, 128 i + 128)
 //   S   columns [256, 288) and [288, 320): two page buffers
 // Thread t of the softmax warps owns row t % 64 and token / d_v half t / 64.
-template <bool kRope, bool kFp16>
+template <bool kRope, bool kFp16, bool kPadHeads>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mla_splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                       const __grid_constant__ CUtensorMap tm_oacc, const DecodeParams p)
+                       const __grid_constant__ CUtensorMap tm_oacc, const __grid_constant__ CUtensorMap tm_o8,
+                       const __grid_constant__ CUtensorMap tm_oacc8, const DecodeParams p)
 {
     using L = Layout<kRope>;
     extern __shared__ uint8_t smem_raw[];
@@ -769,16 +772,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint32_t stage = s_p + warp * 4096;
                 uint8_t* stage_row = smem + L::kOffP + warp * 4096 + lane * 128;
                 const int row_in_group = 64 * static_cast<int>(cta) + (t & 32);  // warp's first row
-                const bool tile_live = rg * kRowsPerGroup + row_in_group < p.rows;
+                // Rows past the end are clipped by the tensor maps.  A tile whose rows are all
+                // real heads is stored whole; one that also holds padding heads is stored in
+                // 8-row groups (each all real or all padding: h_q and active_heads are
+                // multiples of 8 then), skipping the padding ones.
+                // (Without padding heads, kPadHeads = false, every tile that starts before
+                // the last row is stored whole.)
+                bool tile_live, tile_whole = true;
+                uint32_t real_rows = 0xffffffffu;
+                if constexpr (kPadHeads) {
+                    const int lane_row = rg * kRowsPerGroup + row_in_group + lane;
+                    const bool lane_padding = lane_row < p.rows && lane_row % p.h_q >= p.active_heads;
+                    real_rows = __ballot_sync(0xffffffffu, lane_row < p.rows && !lane_padding);
+                    tile_live = real_rows != 0u;
+                    tile_whole = !__any_sync(0xffffffffu, lane_padding);
+                } else {
+                    tile_live = rg * kRowsPerGroup + row_in_group < p.rows;
+                }
                 auto stage_free = [&]() {
                     if (lane == 0) bulk_wait_read_all();
                     __syncwarp();
                 };
-                auto stage_issue = [&](const CUtensorMap* map, int x, int y, int z) {
+                auto stage_issue = [&](const CUtensorMap* map, const CUtensorMap* map8, int x, int y, int z) {
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0 && tile_live) {
-                        tma_store_3d(map, stage, x, y, z);
+                        if (tile_whole) {
+                            tma_store_3d(map, stage, x, y, z);
+                        } else {
+#pragma unroll
+                            for (int g8 = 0; g8 < 4; ++g8)
+                                if ((real_rows >> (8 * g8)) & 0xffu) tma_store_3d(map8, stage + 1024 * g8, x, y + 8 * g8, z);
+                        }
                         bulk_commit_group();
                     }
                 };
@@ -821,7 +846,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             w.w = pack2(__uint_as_float(v[6]) * inv_l, __uint_as_float(v[7]) * inv_l, kFp16);
                             *reinterpret_cast<uint4*>(stage_row + ((c ^ (lane & 7)) << 4)) = w;
                         }
-                        stage_issue(&tm_o, col0, rg * kRowsPerGroup + row_in_group, b);
+                        stage_issue(&tm_o, &tm_o8, col0, rg * kRowsPerGroup + row_in_group, b);
                     } else {
                         // fp32 partial: two tiles of 32 columns
 #pragma unroll
@@ -834,18 +859,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                     make_float4(__uint_as_float(v[0]) * inv_l, __uint_as_float(v[1]) * inv_l,
                                                 __uint_as_float(v[2]) * inv_l, __uint_as_float(v[3]) * inv_l);
                             }
-                            stage_issue(&tm_oacc, col0 + 32 * hb, row_in_group, static_cast<int>(slot));
+                            stage_issue(&tm_oacc, &tm_oacc8, col0 + 32 * hb, row_in_group, static_cast<int>(slot));
                         }
                     }
                 }
                 stage_free();  // the tiles are P buffers again for the next chunk
             }
-            if (h == 0) {
-                if (nsplit == 1) {
-                    if (row_valid) p.lse[static_cast<size_t>(b) * p.rows + row] = lse_v;
-                } else {
+            if (h == 0 && row_valid && (!kPadHeads || row % p.h_q < p.active_heads)) {
+                if (nsplit == 1)
+                    p.lse[static_cast<size_t>(b) * p.rows + row] = lse_v;
+                else
                     p.lse_accum[slot * kRowsPerGroup + 64 * cta + r] = lse_v;
-                }
             }
             if (!empty) ++k;
             g += (n > 0 ? n : 0);
@@ -891,7 +915,8 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = kSplitParallel ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y) * 4 + warp;
     const int rows_here = min(kRowsPerGroup, p.rows - rg * kRowsPerGroup);
-    if (r >= rows_here) return;  // uniform over the CTA in the split-parallel layout
+    // uniform over the CTA in the split-parallel layout; padding heads are not combined
+    if (r >= rows_here || (rg * kRowsPerGroup + r) % p.h_q >= p.active_heads) return;
     const float* lse_k = p.lse_accum + static_cast<size_t>(slot0) * kRowsPerGroup + r;
     float mx = -INFINITY;
     for (int k = lane; k < nsplit; k += 32) mx = fmaxf(mx, lse_k[static_cast<size_t>(k) * kRowsPerGroup]);
@@ -1112,6 +1137,15 @@ static void programmatic_launch(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* at
     cfg.numAttrs = 1;
 }
 
+// Heads [active_heads, h_q) are padding whose outputs nobody reads: a count that is not a
+// multiple of 8 in (0, h_q], or an h_q that is not a multiple of 8, means every head (fail
+// closed to the full computation, as the "FlashMLA vLLM Optimization" page's active-head
+// switch does).
+static int effective_active_heads(int active_heads, int h_q)
+{
+    return (active_heads > 0 && active_heads <= h_q && active_heads % 8 == 0 && h_q % 8 == 0) ? active_heads : h_q;
+}
+
 static size_t workspace_slots(int batch, int groups, int num_parts)
 {
     return static_cast<size_t>(batch) * groups + static_cast<size_t>(num_parts);
@@ -1119,10 +1153,10 @@ static size_t workspace_slots(int batch, int groups, int num_parts)
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-template <bool kRope, bool kFp16>
+template <bool kRope, bool kFp16, bool kPadHeads>
 static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorMap* maps, const DecodeParams& prm)
 {
-    auto kern = mla_splitkv_kernel<kRope, kFp16>;
+    auto kern = mla_splitkv_kernel<kRope, kFp16, kPadHeads>;
     const int smem = Layout<kRope>::kSmemBytes;
     static int configured_device = -1;  // the attribute is per device; set it once per device in use
     int dev = 0;
@@ -1136,7 +1170,15 @@ static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorM
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     programmatic_launch(cfg, attr, dim3(grid), dim3(kThreads), smem, stream);
-    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], prm);
+    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], prm);
+}
+
+// The kernel variant with padding-head logic runs only when some heads are padding.
+template <bool kRope, bool kFp16>
+static cudaError_t launch_splitkv_heads(int grid, cudaStream_t st, const CUtensorMap* maps, const DecodeParams& prm)
+{
+    return prm.active_heads < prm.h_q ? launch_splitkv<kRope, kFp16, true>(grid, st, maps, prm)
+                                      : launch_splitkv<kRope, kFp16, false>(grid, st, maps, prm);
 }
 
 }  // namespace mla
@@ -1243,8 +1285,8 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
                                  int num_blocks, int page_size, int h_kv, const int32_t* block_table,
                                  int max_blocks_per_seq, const int32_t* cache_seqlens, int dv, int dtype,
                                  const int32_t* tile_md, int num_parts, const int32_t* num_splits, int causal,
-                                 float softmax_scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
-                                 DecodeParams& prm, CUtensorMap* maps)
+                                 float softmax_scale, int active_heads, void* o, float* lse, void* workspace,
+                                 size_t workspace_bytes, DecodeParams& prm, CUtensorMap* maps)
 {
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
         num_parts <= 0 || (causal != 0 && causal != 1))
@@ -1282,6 +1324,7 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     prm.causal = causal;
     prm.box_rows = rows < 64 ? rows : 64;  // query rows per CTA of the pair
     prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+    prm.active_heads = effective_active_heads(active_heads, h_q);
     prm.dtype = dtype;
     prm.d_qk = d_qk;
     prm.num_parts = num_parts;
@@ -1311,7 +1354,13 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
         encode_3d(&maps[3], o, dt, kDv, rows, batch, kDv * 2, static_cast<uint64_t>(kDv) * 2 * rows, 64,
                   rows < 32 ? rows : 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
         encode_3d(&maps[4], prm.o_accum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kDv, kRowsPerGroup, slots, kDv * 4,
-                  static_cast<uint64_t>(kDv) * 4 * kRowsPerGroup, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+                  static_cast<uint64_t>(kDv) * 4 * kRowsPerGroup, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+        // the same with 8-row boxes: tiles that mix real and padding heads are stored
+        // 8 rows at a time (one 1 KB swizzle atom each), skipping the padding groups
+        encode_3d(&maps[5], o, dt, kDv, rows, batch, kDv * 2, static_cast<uint64_t>(kDv) * 2 * rows, 64,
+                  rows < 8 ? rows : 8, CU_TENSOR_MAP_SWIZZLE_128B) &&
+        encode_3d(&maps[6], prm.o_accum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kDv, kRowsPerGroup, slots, kDv * 4,
+                  static_cast<uint64_t>(kDv) * 4 * kRowsPerGroup, 32, 8, CU_TENSOR_MAP_SWIZZLE_128B);
     return ok ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -1320,11 +1369,11 @@ static mla_status launch_splitkv_stage(const DecodeParams& prm, const CUtensorMa
     const int grid = 2 * prm.num_parts;
     cudaError_t e;
     if (prm.d_qk == 576)
-        e = prm.dtype == MLA_FP16 ? launch_splitkv<true, true>(grid, st, maps, prm)
-                                  : launch_splitkv<true, false>(grid, st, maps, prm);
+        e = prm.dtype == MLA_FP16 ? launch_splitkv_heads<true, true>(grid, st, maps, prm)
+                                  : launch_splitkv_heads<true, false>(grid, st, maps, prm);
     else
-        e = prm.dtype == MLA_FP16 ? launch_splitkv<false, true>(grid, st, maps, prm)
-                                  : launch_splitkv<false, false>(grid, st, maps, prm);
+        e = prm.dtype == MLA_FP16 ? launch_splitkv_heads<false, true>(grid, st, maps, prm)
+                                  : launch_splitkv_heads<false, false>(grid, st, maps, prm);
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -1351,14 +1400,14 @@ static mla_status launch_combine_stage(const DecodeParams& prm, cudaStream_t st)
 
 #define MLA_DECODE_ARGS                                                                                          \
     q, batch, s_q, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, block_table, max_blocks_per_seq,            \
-        cache_seqlens, dv, dtype, tile_md, num_parts, num_splits, causal, softmax_scale, o, lse, workspace,      \
-        workspace_bytes
+        cache_seqlens, dv, dtype, tile_md, num_parts, num_splits, causal, softmax_scale, active_heads, o, lse,   \
+        workspace, workspace_bytes
 
 mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache,
                                    int num_blocks, int page_size, int h_kv, const int32_t* block_table,
                                    int max_blocks_per_seq, const int32_t* cache_seqlens, int dv, int dtype,
                                    const int32_t* tile_md, int num_parts, const int32_t* num_splits, int causal,
-                                   float softmax_scale, void* o, float* lse, void* workspace,
+                                   float softmax_scale, int active_heads, void* o, float* lse, void* workspace,
                                    size_t workspace_bytes, void* stream)
 {
     DecodeParams prm;
@@ -1375,8 +1424,8 @@ mla_status mla_decode_splitkv(const void* q, int batch, int s_q, int h_q, int d_
                               int num_blocks, int page_size, int h_kv, const int32_t* block_table,
                               int max_blocks_per_seq, const int32_t* cache_seqlens, int dv, int dtype,
                               const int32_t* tile_md, int num_parts, const int32_t* num_splits, int causal,
-                              float softmax_scale, void* o, float* lse, void* workspace, size_t workspace_bytes,
-                              void* stream)
+                              float softmax_scale, int active_heads, void* o, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream)
 {
     DecodeParams prm;
     CUtensorMap maps[kNumMaps];
@@ -1386,8 +1435,8 @@ mla_status mla_decode_splitkv(const void* q, int batch, int s_q, int h_q, int d_
 }
 
 mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int dtype, const int32_t* num_splits,
-                              int num_parts, void* o, float* lse, void* workspace, size_t workspace_bytes,
-                              void* stream)
+                              int num_parts, int active_heads, void* o, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream)
 {
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_parts <= 0) return MLA_ERR_INVALID_ARG;
     if (dtype != MLA_BF16 && dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
@@ -1408,6 +1457,8 @@ mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int
     prm.batch = batch;
     prm.dtype = dtype;
     prm.num_parts = num_parts;
+    prm.h_q = h_q;
+    prm.active_heads = effective_active_heads(active_heads, h_q);
     prm.lse_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader);
     prm.o_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader +
                                            align_up(slots * kRowsPerGroup * sizeof(float), 256));
@@ -1469,7 +1520,7 @@ extern "C" mla_status mla_decode_with_kvcache_noalloc(const void* q, int batch, 
                                                       const int32_t* cache_seqlens, int dv, int dtype,
                                                       const int32_t* tile_md, int num_parts,
                                                       const int32_t* num_splits, int causal, float softmax_scale,
-                                                      void* o, float* lse, void* stream)
+                                                      int active_heads, void* o, float* lse, void* stream)
 {
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_parts <= 0) return MLA_ERR_INVALID_ARG;
     if (batch == 0) return MLA_OK;
@@ -1485,5 +1536,6 @@ extern "C" mla_status mla_decode_with_kvcache_noalloc(const void* q, int batch, 
     if (cudaMemsetAsync(scratch, 0, sizeof(int), cs) != cudaSuccess) return MLA_ERR_CUDA;
     return mla_decode_with_kvcache(q, batch, s_q, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, block_table,
                                    max_blocks_per_seq, cache_seqlens, dv, dtype, tile_md, num_parts, num_splits,
-                                   causal, softmax_scale, o, lse, scratch, MLA_NOALLOC_SCRATCH_BYTES, stream);
+                                   causal, softmax_scale, active_heads, o, lse, scratch, MLA_NOALLOC_SCRATCH_BYTES,
+                                   stream);
 }

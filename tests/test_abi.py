@@ -59,7 +59,7 @@ def _decode(lib, **over):
     fake = 1 << 20  # aligned non-null "device" pointers: validation must reject before any use
     args = dict(q=fake, batch=2, s_q=1, h_q=16, d_qk=576, kvcache=fake, num_blocks=8, page_size=64, h_kv=1,
                 block_table=fake, max_blocks=4, seqlens=fake, dv=512, dtype=0, md=fake, num_parts=74,
-                num_splits=fake, causal=0, scale=0.0, o=fake, lse=fake, ws=fake,
+                num_splits=fake, causal=0, scale=0.0, active_heads=0, o=fake, lse=fake, ws=fake,
                 ws_bytes=1 << 40, stream=None)
     args.update(over)
     return lib.mla_decode_with_kvcache(*args.values())

@@ -98,6 +98,36 @@ def test_two_stage_calls_match_single_call(name, parts):
     assert torch.equal(call.out, o1) and torch.equal(call.lse, lse1)
 
 
+@pytest.mark.parametrize("case", ["few_splits", "many_splits", "not_a_multiple_of_8"])
+def test_active_heads(oracle_mod, case):
+    # Padding heads (queries zero, as a tensor-parallel rank pads its heads) are neither
+    # written nor combined; the real heads match the oracle.  A count that is not a
+    # multiple of 8 falls back to every head.
+    if case == "many_splits":
+        p = W.make_problem([20000, 7000], s_q=2, h_q=64, causal=True, active_heads=16, seed=150)
+    else:
+        p = W.make_workload("spec_padded", seqlens=[300, 420, 511, 129, 64, 2])
+    active = 12 if case == "not_a_multiple_of_8" else 16
+    q, kv, bt, sl = to_device(p)
+    md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q, 1)
+    o = torch.full((p.batch, p.s_q, p.h_q, 512), 7.0, dtype=q.dtype, device="cuda")
+    lse = torch.full((p.batch, p.s_q, p.h_q), 7.0, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(mla.workspace_bytes(p.batch, p.s_q, p.h_q, 1, md.shape[0]), dtype=torch.uint8, device="cuda")
+    mla.flash_mla_with_kvcache(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale,
+                               workspace=ws, out=o, lse=lse, active_heads=active)
+    torch.cuda.synchronize()
+    assert mla.read_device_status(ws) == 0
+    if case == "many_splits":
+        assert int(ns[-1].item()) >= 4 * p.batch, "the case must split each sequence several times"
+    o_ref, lse_ref = oracle_full(oracle_mod, p)
+    real = p.h_q if active % 8 else active
+    print(compare(o[:, :, :real].contiguous(), lse[:, :, :real].contiguous(), o_ref[:, :, :real], lse_ref[:, :, :real],
+                  p.dtype, f"active heads {active} ({case})"))
+    if real < p.h_q:
+        assert bool((o[:, :, real:] == 7.0).all()), "padding heads' O was written"
+        assert bool((lse[:, :, real:] == 7.0).all()), "padding heads' LSE was written"
+
+
 def test_metadata_kernel_matches_host_schedule():
     rng = np.random.default_rng(7)
     for hpk in (16, 128, 256):

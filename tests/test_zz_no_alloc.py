@@ -50,7 +50,7 @@ def _device_problem(p):
 def _args(p, q, kv, bt, sl, md, ns, o, lse):
     return (q.data_ptr(), p.batch, p.s_q, p.h_q, p.d_qk, kv.data_ptr(), p.num_blocks, 64, 1, bt.data_ptr(),
             bt.shape[1], sl.data_ptr(), 512, p.dtype, md.data_ptr(), md.shape[0], ns.data_ptr(), int(p.causal),
-            p.scale, o.data_ptr(), lse.data_ptr())
+            p.scale, 0, o.data_ptr(), lse.data_ptr())
 
 
 def _regular(lib, p, t):
@@ -97,5 +97,5 @@ def test_noalloc_rejects_problems_beyond_its_scratch(lib):
     # host with MLA_ERR_WORKSPACE before anything is enqueued.
     fake = 1 << 20
     rc = lib.mla_decode_with_kvcache_noalloc(fake, 4096, 1, 128, 576, fake, 4096, 64, 1, fake, 1, fake, 512, 0,
-                                             fake, 74, fake, 0, 0.0, fake, fake, None)
+                                             fake, 74, fake, 0, 0.0, 0, fake, fake, None)
     assert rc == 3
