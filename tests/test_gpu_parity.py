@@ -98,16 +98,18 @@ def test_two_stage_calls_match_single_call(name, parts):
     assert torch.equal(call.out, o1) and torch.equal(call.lse, lse1)
 
 
-@pytest.mark.parametrize("case", ["few_splits", "many_splits", "not_a_multiple_of_8"])
+@pytest.mark.parametrize("case", ["few_splits", "many_splits", "not_a_multiple_of_8", "h_q_not_a_multiple_of_8"])
 def test_active_heads(oracle_mod, case):
     # Padding heads (queries zero, as a tensor-parallel rank pads its heads) are neither
     # written nor combined; the real heads match the oracle.  A count that is not a
     # multiple of 8 falls back to every head.
     if case == "many_splits":
         p = W.make_problem([20000, 7000], s_q=2, h_q=64, causal=True, active_heads=16, seed=150)
+    elif case == "h_q_not_a_multiple_of_8":
+        p = W.make_problem([900, 77], s_q=2, h_q=100, causal=True, active_heads=96, seed=151)
     else:
         p = W.make_workload("spec_padded", seqlens=[300, 420, 511, 129, 64, 2])
-    active = 12 if case == "not_a_multiple_of_8" else 16
+    active = {"not_a_multiple_of_8": 12, "h_q_not_a_multiple_of_8": 96}.get(case, 16)
     q, kv, bt, sl = to_device(p)
     md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q, 1)
     o = torch.full((p.batch, p.s_q, p.h_q, 512), 7.0, dtype=q.dtype, device="cuda")
@@ -120,7 +122,7 @@ def test_active_heads(oracle_mod, case):
     if case == "many_splits":
         assert int(ns[-1].item()) >= 4 * p.batch, "the case must split each sequence several times"
     o_ref, lse_ref = oracle_full(oracle_mod, p)
-    real = p.h_q if active % 8 else active
+    real = p.h_q if (active % 8 or p.h_q % 8) else active
     print(compare(o[:, :, :real].contiguous(), lse[:, :, :real].contiguous(), o_ref[:, :, :real], lse_ref[:, :, :real],
                   p.dtype, f"active heads {active} ({case})"))
     if real < p.h_q:
