@@ -118,12 +118,18 @@ MLA_API mla_status mla_get_metadata_host(const int32_t* cache_seqlens, int batch
                                  int h_kv, int num_parts, int32_t* tile_md, int32_t* num_splits);
 
 /*
- * Bytes of device workspace mla_decode_with_kvcache needs: a 256-byte status
- * header plus float32 partial outputs and LSEs for up to
- * batch * row_groups + num_parts splits of 128 rows each.
- * Returns 0 for invalid sizes.
+ * Bytes of device workspace mla_decode_with_kvcache needs: a control block
+ * (the status word and two int32 counters per (request, row group)), then
+ * float32 partial outputs and LSEs for up to batch * row_groups + num_parts
+ * splits of 128 rows each.  Returns 0 for invalid sizes.
+ *
+ * The first mla_decode_workspace_zero_bytes(...) bytes (the control block) must
+ * be zero before a workspace is first used; every call that completes without
+ * a device error leaves them zero again.  After a device error (see
+ * mla_read_device_status) zero them before reusing the workspace.
  */
 MLA_API size_t mla_decode_workspace_bytes(int batch, int s_q, int h_q, int h_kv, int num_parts);
+MLA_API size_t mla_decode_workspace_zero_bytes(int batch, int s_q, int h_q, int h_kv);
 
 /*
  * Dense MLA decoding with a paged KV cache ("FlashMLA" usage page:

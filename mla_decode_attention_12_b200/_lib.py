@@ -33,6 +33,7 @@ SIGNATURES = {
     "mla_get_metadata": ([_P, _I, _I, _I, _I, _P, _P, _P], _I),
     "mla_get_metadata_host": ([_P, _I, _I, _I, _I, _P, _P], _I),
     "mla_decode_workspace_bytes": ([_I, _I, _I, _I, _I], _SZ),
+    "mla_decode_workspace_zero_bytes": ([_I, _I, _I, _I], _SZ),
     "mla_decode_with_kvcache": ([_P, _I, _I, _I, _I,          # q, batch, s_q, h_q, d_qk
                                  _P, _I, _I, _I,              # kvcache, num_blocks, page_size, h_kv
                                  _P, _I, _P, _I, _I,          # block_table, max_blocks, seqlens, dv, dtype

@@ -96,14 +96,25 @@ def workspace_bytes(batch: int, s_q: int, h_q: int, h_kv: int, num_parts: int) -
     return n
 
 
-def get_workspace(nbytes: int, device: torch.device) -> torch.Tensor:
-    """A cached, grow-only workspace per (device, stream); its status header starts zeroed."""
+def workspace_zero_bytes(batch: int, s_q: int, h_q: int, h_kv: int) -> int:
+    """Leading workspace bytes (status word and counters) that must be zero before first use."""
+    return _lib.load().mla_decode_workspace_zero_bytes(batch, s_q, h_q, h_kv)
+
+
+def get_workspace(nbytes: int, device: torch.device, zero_bytes: int = 256) -> torch.Tensor:
+    """A cached, grow-only workspace per (device, stream) whose first ``zero_bytes`` are zero.
+
+    Calls leave the control block zero; it is cleared again only when a call needs a
+    larger one than any before (its counters then reach into bytes used for other data).
+    """
     key = (device.index, _stream(device))
-    ws = _workspaces.get(key)
+    ws, zeroed = _workspaces.get(key, (None, 0))
     if ws is None or ws.numel() < nbytes:
-        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
-        ws[:256].zero_()
-        _workspaces[key] = ws
+        ws, zeroed = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device), 0
+    if zeroed < zero_bytes:
+        ws[:zero_bytes].zero_()
+        zeroed = zero_bytes
+    _workspaces[key] = (ws, zeroed)
     return ws
 
 
@@ -132,7 +143,8 @@ class DecodeCall:
         if lse is None:
             lse = torch.empty(b, s_q, h_q, dtype=torch.float32, device=dev)
         if workspace is None:
-            workspace = get_workspace(workspace_bytes(b, s_q, h_q, h_kv, num_parts), dev)
+            workspace = get_workspace(workspace_bytes(b, s_q, h_q, h_kv, num_parts), dev,
+                                      workspace_zero_bytes(b, s_q, h_q, h_kv))
         scale = float(softmax_scale) if softmax_scale is not None else 1.0 / math.sqrt(d_qk)
         self.device = dev
         self.out, self.lse, self.workspace = out, lse, workspace

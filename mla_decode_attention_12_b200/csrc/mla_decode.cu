@@ -150,6 +150,8 @@ struct DecodeParams {
     float* o_accum;     // [slots, 128, 512]
     float* lse_accum;   // [slots, 128]
     int* status;
+    int* split_done;      // [NV]: split-KV warps that announced their partials (8 per split)
+    int* combine_passed;  // [NV]: combine CTAs past their wait
     int batch, s_q, h_q, rows, groups, max_blocks, num_blocks, causal, box_rows;
     int active_heads;  // heads >= active_heads are padding: not written, not combined
     float scale_log2;
@@ -598,6 +600,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t g = 0, k = 0;
         int vb, lo, hi;
         bool ok = true;
+        // The combine of a virtual batch starts once the 8 warps of each of its splits (4 per
+        // CTA of the pair) have announced their partial results.  A warp announces a split
+        // at the start of its next epilogue, or at the end, when its stores have long
+        // completed, so the wait for completion costs nothing.
+        int announce_vb = -1;
+        auto announce = [&]() {
+            if (announce_vb >= 0) {
+                __syncwarp();
+                if (lane == 0) {
+                    bulk_wait_all();             // this warp's tile stores of that split are complete
+                    fence_proxy_async_global();  // ... and ordered before the counter update
+                    __threadfence();             // (with the LSE stores of the warp)
+                    atomicAdd(p.split_done + announce_vb, 1);
+                }
+                __syncwarp();
+                announce_vb = -1;
+            }
+        };
         bool have = chunks.next(vb, lo, hi);
         bool q_ready = false;  // this chunk's Q already stored (ahead of the previous epilogue)
         while (ok && have) {
@@ -763,6 +783,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (!(ok = wwait(bar(kBarOFull), k & 1))) break;
                 tc_fence_after();
             }
+            announce();
             // O leaves tensor memory 64 columns at a time.  Each warp writes its 32 rows
             // into a 4 KB tile of shared memory (the P buffers are idle now) in the
             // 128-byte-swizzled layout of the output tensor maps, and lane 0 hands the
@@ -871,6 +892,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 else
                     p.lse_accum[slot * kRowsPerGroup + 64 * cta + r] = lse_v;
             }
+            if (nsplit > 1) announce_vb = vb;
             if (!empty) ++k;
             g += (n > 0 ? n : 0);
             have = have_next;
@@ -878,6 +900,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             lo = nlo;
             hi = nhi;
         }
+        if (ok) announce();
         // Shared memory must outlive the TMA unit's reads of the output tiles; the writes
         // themselves are complete, and visible to the next grid, when the grid completes.
         if (lane == 0) bulk_wait_read_all();
@@ -906,11 +929,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 template <bool kFp16, bool kSplitParallel>
 __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
 {
-    grid_dependency_wait();  // the split partials of the split-KV grid
+    // No wait for the whole split-KV grid: the CTAs of a virtual batch start combining once
+    // its splits are announced (8 warps per split), while other partitions still run.  This
+    // grid is launched only after every split-KV CTA is resident (programmatic launch), so
+    // the wait below cannot starve its producers; it is bounded all the same.  The last
+    // combine CTA of the virtual batch past the wait clears both counters for the next call.
+    // (The schedule was written by the metadata grid, complete before the split-KV grid
+    // allowed this one to launch.)
     const int vb = blockIdx.x;
     const int slot0 = p.num_splits[vb];
     const int nsplit = p.num_splits[vb + 1] - slot0;
     if (nsplit <= 1) return;
+    __shared__ int go;
+    if (threadIdx.x == 0) {
+        const int want = 8 * nsplit;
+        bool ready = ld_acquire_gpu(p.split_done + vb) >= want;
+        const uint64_t t0 = global_timer_ns();
+        while (!ready) {
+            __nanosleep(200);
+            ready = ld_acquire_gpu(p.split_done + vb) >= want;
+            if (!ready && global_timer_ns() - t0 > kWaitTimeoutNs) {
+                atomicCAS(p.status, 0, MLA_ERR_TIMEOUT);
+                break;
+            }
+        }
+        if (ready && atomicAdd(p.combine_passed + vb, 1) == static_cast<int>(gridDim.y) - 1) {
+            p.combine_passed[vb] = 0;
+            p.split_done[vb] = 0;
+        }
+        go = ready;
+    }
+    __syncthreads();
+    if (!go) return;
     const int b = vb / p.groups, rg = vb % p.groups;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = kSplitParallel ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y) * 4 + warp;
@@ -919,12 +969,12 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
     if (r >= rows_here || (rg * kRowsPerGroup + r) % p.h_q >= p.active_heads) return;
     const float* lse_k = p.lse_accum + static_cast<size_t>(slot0) * kRowsPerGroup + r;
     float mx = -INFINITY;
-    for (int k = lane; k < nsplit; k += 32) mx = fmaxf(mx, lse_k[static_cast<size_t>(k) * kRowsPerGroup]);
+    for (int k = lane; k < nsplit; k += 32) mx = fmaxf(mx, __ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup));
 #pragma unroll
     for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float sum = 0.f;
     if (mx != -INFINITY)
-        for (int k = lane; k < nsplit; k += 32) sum += expf(lse_k[static_cast<size_t>(k) * kRowsPerGroup] - mx);
+        for (int k = lane; k < nsplit; k += 32) sum += expf(__ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup) - mx);
 #pragma unroll
     for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float lse = (mx == -INFINITY) ? -INFINITY : mx + logf(sum);
@@ -932,7 +982,7 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     auto add_split = [&](const float4* s4, float w) {
-        const float4 v0 = s4[0], v1 = s4[32], v2 = s4[64], v3 = s4[96];
+        const float4 v0 = __ldcg(s4), v1 = __ldcg(s4 + 32), v2 = __ldcg(s4 + 64), v3 = __ldcg(s4 + 96);
         acc[0].x += w * v0.x; acc[0].y += w * v0.y; acc[0].z += w * v0.z; acc[0].w += w * v0.w;
         acc[1].x += w * v1.x; acc[1].y += w * v1.y; acc[1].z += w * v1.z; acc[1].w += w * v1.w;
         acc[2].x += w * v2.x; acc[2].y += w * v2.y; acc[2].z += w * v2.z; acc[2].w += w * v2.w;
@@ -944,11 +994,12 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
         if (kSplitParallel) {
 #pragma unroll 2
             for (int k = warp; k < nsplit; k += 4)
-                add_split(src + static_cast<size_t>(k) * stride4, expf(lse_k[static_cast<size_t>(k) * kRowsPerGroup] - lse));
+                add_split(src + static_cast<size_t>(k) * stride4,
+                          expf(__ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup) - lse));
         } else {
             for (int kb = 0; kb < nsplit; kb += 32) {
                 const int k = kb + lane;
-                const float w_mine = (k < nsplit) ? expf(lse_k[static_cast<size_t>(k) * kRowsPerGroup] - lse) : 0.f;
+                const float w_mine = (k < nsplit) ? expf(__ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup) - lse) : 0.f;
                 const int cnt = min(32, nsplit - kb);
 #pragma unroll 4
                 for (int kk = 0; kk < cnt; ++kk)
@@ -1153,6 +1204,24 @@ static size_t workspace_slots(int batch, int groups, int num_parts)
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Workspace layout: a control block (the status word, then two int32 counters per virtual
+// batch: split partials announced, combine CTAs past their wait), which must be zero before
+// the first call and is left zero by every call that completes without a device error; then
+// the split LSEs and the split partial outputs.
+static size_t control_bytes(size_t nv) { return align_up(kWorkspaceHeader + 2 * nv * sizeof(int32_t), 256); }
+
+static void workspace_pointers(void* workspace, int batch, int groups, int num_parts, DecodeParams& prm)
+{
+    const size_t nv = static_cast<size_t>(batch) * groups;
+    const size_t slots = workspace_slots(batch, groups, num_parts);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    prm.status = reinterpret_cast<int*>(ws);
+    prm.split_done = reinterpret_cast<int*>(ws + kWorkspaceHeader);
+    prm.combine_passed = prm.split_done + nv;
+    prm.lse_accum = reinterpret_cast<float*>(ws + control_bytes(nv));
+    prm.o_accum = reinterpret_cast<float*>(ws + control_bytes(nv) + align_up(slots * kRowsPerGroup * sizeof(float), 256));
+}
+
 template <bool kRope, bool kFp16, bool kPadHeads>
 static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorMap* maps, const DecodeParams& prm)
 {
@@ -1269,12 +1338,18 @@ mla_status mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_p
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+size_t mla_decode_workspace_zero_bytes(int batch, int s_q, int h_q, int h_kv)
+{
+    if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || h_q % h_kv) return 0;
+    return control_bytes(static_cast<size_t>(batch) * row_groups(s_q * h_q / h_kv));
+}
+
 size_t mla_decode_workspace_bytes(int batch, int s_q, int h_q, int h_kv, int num_parts)
 {
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_parts <= 0 || h_q % h_kv) return 0;
     const int groups = row_groups(s_q * h_q / h_kv);
     const size_t slots = workspace_slots(batch, groups, num_parts);
-    size_t bytes = kWorkspaceHeader;
+    size_t bytes = control_bytes(static_cast<size_t>(batch) * groups);
     bytes += align_up(slots * kRowsPerGroup * sizeof(float), 256);
     bytes += slots * kRowsPerGroup * kDv * sizeof(float);
     return bytes;
@@ -1330,10 +1405,7 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     prm.num_parts = num_parts;
     if (batch == 0) return MLA_OK;
     const size_t slots = workspace_slots(batch, groups, num_parts);
-    prm.status = static_cast<int*>(workspace);
-    prm.lse_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader);
-    prm.o_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader +
-                                           align_up(slots * kRowsPerGroup * sizeof(float), 256));
+    workspace_pointers(workspace, batch, groups, num_parts, prm);
     if (!maps) return MLA_OK;
 
     const CUtensorMapDataType dt =
@@ -1447,7 +1519,6 @@ mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int
     if (workspace_bytes < mla_decode_workspace_bytes(batch, s_q, h_q, h_kv, num_parts)) return MLA_ERR_WORKSPACE;
     const int rows = s_q * h_q;
     const int groups = row_groups(rows);
-    const size_t slots = workspace_slots(batch, groups, num_parts);
     DecodeParams prm{};
     prm.num_splits = num_splits;
     prm.o = o;
@@ -1459,9 +1530,7 @@ mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int
     prm.num_parts = num_parts;
     prm.h_q = h_q;
     prm.active_heads = effective_active_heads(active_heads, h_q);
-    prm.lse_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader);
-    prm.o_accum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeader +
-                                           align_up(slots * kRowsPerGroup * sizeof(float), 256));
+    workspace_pointers(workspace, batch, groups, num_parts, prm);
     return launch_combine_stage(prm, static_cast<cudaStream_t>(stream));
 }
 
@@ -1530,10 +1599,12 @@ extern "C" mla_status mla_decode_with_kvcache_noalloc(const void* q, int batch, 
     void* scratch = nullptr;
     mla_status st = noalloc_scratch(&scratch);
     if (st != MLA_OK) return st;
-    // The status word must start at zero; the split partials are always written
-    // before they are read, so the rest of the scratch needs no clearing.
+    // The control block (status word and split / combine counters) must start at zero;
+    // the split partials are always written before they are read, so the rest of the
+    // scratch needs no clearing.
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(scratch, 0, sizeof(int), cs) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaMemsetAsync(scratch, 0, mla_decode_workspace_zero_bytes(batch, s_q, h_q, h_kv), cs) != cudaSuccess)
+        return MLA_ERR_CUDA;
     return mla_decode_with_kvcache(q, batch, s_q, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, block_table,
                                    max_blocks_per_seq, cache_seqlens, dv, dtype, tile_md, num_parts, num_splits,
                                    causal, softmax_scale, active_heads, o, lse, scratch, MLA_NOALLOC_SCRATCH_BYTES,

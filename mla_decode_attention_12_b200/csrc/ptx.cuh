@@ -169,6 +169,18 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Orders this thread's async-proxy accesses to global memory (completed TMA stores) with its
+// later generic-proxy operations.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Load with acquire semantics at GPU scope (pairs with a release by another CTA).
+__device__ __forceinline__ int ld_acquire_gpu(const int* ptr)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
 // Hint: bring the 128-byte line holding `gaddr` into L2.
 __device__ __forceinline__ void prefetch_l2(const void* gaddr)
 {

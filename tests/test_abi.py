@@ -48,10 +48,13 @@ def test_sizes(lib):
     assert lib.mla_metadata_sizes(32, 256, 1, 74, ctypes.byref(a), ctypes.byref(b)) == 0
     assert b.value == 32 * 2 + 1
     assert lib.mla_metadata_sizes(-1, 128, 1, 74, ctypes.byref(a), ctypes.byref(b)) == 1
-    # workspace: header + (NV + parts) * 128 * (1 + 512) floats
+    # workspace: control block (status word + 2 int32 counters per virtual batch, 256-byte
+    # aligned), then (NV + parts) * 128 * (1 + 512) floats
     nv, parts = 64, 74
-    want = 256 + ((nv + parts) * 128 * 4 + 255) // 256 * 256 + (nv + parts) * 128 * 512 * 4
+    control = (256 + 2 * nv * 4 + 255) // 256 * 256
+    want = control + ((nv + parts) * 128 * 4 + 255) // 256 * 256 + (nv + parts) * 128 * 512 * 4
     assert lib.mla_decode_workspace_bytes(64, 1, 128, 1, 74) == want
+    assert lib.mla_decode_workspace_zero_bytes(64, 1, 128, 1) == control == 768
     assert lib.mla_decode_workspace_bytes(64, 0, 128, 1, 74) == 0
 
 
