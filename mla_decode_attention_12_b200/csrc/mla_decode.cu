@@ -12,28 +12,27 @@
 //
 // Design for sm_100a (ours; the pages' kernels target Hopper):
 //
-// * One two-CTA cluster (two SMs) per scheduler partition.  The 128 query rows
-//   of a row group are the MMA M dimension in both CTAs.  The d_qk columns are
-//   split between the CTAs: CTA c owns latent columns [256c, 256c+256) and
-//   RoPE columns [512 + 32c, 512 + 32c + 32).  Each CTA loads only its columns
-//   of Q and of every cached page (every KV byte is read from HBM once, by one
-//   CTA), computes the partial logits S_c = Q_c K_c^T with tcgen05 into tensor
-//   memory, and the two partials are summed by exchanging them through
-//   distributed shared memory (st.async into the peer's buffer).  Both CTAs
-//   then hold the same logits and run the same online softmax, so each can
-//   accumulate its half of O = P V (V columns [256c, 256c+256)) in its own
-//   tensor memory: O half (256 columns) + two S/P buffers (2 x 64) = 384 of
-//   the 512 TMEM columns.
-// * Warp roles per CTA: warps 0-3 softmax / correction / epilogue (thread =
-//   query row = TMEM lane), warp 4 TMA producer (Q per chunk, one 64-token page
-//   per pipeline stage, pages found through the block table), warp 5 MMA issuer.
-// * P is written back into the S buffer in tensor memory (16-bit, two per
-//   column) and is the A operand of the PV MMA; V is read from the same shared
-//   memory stage as K (MN-major descriptor), never loaded twice.
-// * Online softmax in base 2 with a lazily moved reference maximum: O is only
-//   rescaled when the running maximum grows by more than 2^8.
-// * Split chunks write fp32 partial O and LSE to the workspace; the combine
-//   kernel merges them.
+// * One two-CTA cluster (an SM pair) per scheduler partition; the even CTA issues
+//   two-SM tcgen05 MMAs (cta_group::2, M = 128 query rows, 64 per CTA).
+//   S = Q K^T: N = 64 tokens of a page, each CTA supplying its 32 tokens (K stage of
+//   32 tokens x 576 columns); O += P V: N = 256 d_v columns per MMA, each CTA supplying
+//   128 of them (V stage of 64 tokens x its 256 d_v columns, read from L2 again: every
+//   HBM byte is read once, every L2 byte twice).  Each CTA receives the full-width
+//   results for its own 64 rows in tensor memory (the 2x2 layout of pair MMAs).
+// * Tensor memory per CTA: O 256 columns, two S buffers 2 x 32, Q columns [0, 384) as
+//   the A operand of Q K^T 192; shared memory: Q columns 384+, a 3-stage K ring, a
+//   2-stage V ring, two P buffers (P is the A operand of P V), barriers.
+// * Warp roles: 4 softmax warps (thread = TMEM lane: row t % 64, token / d_v half
+//   t / 64), a K loader, the MMA issuer, a V loader (zeroes page tails), a Q loader.
+//   Pages are gathered through the block table by TMA.
+// * Online softmax in base 2 with a lazily moved reference maximum: O is rescaled in
+//   tensor memory only when the running maximum grows by more than 2^8.
+// * Epilogue: the softmax warps store the next chunk's Q into tensor memory, then drain
+//   O 64 columns at a time into swizzled tiles handed to TMA bulk stores: 16-bit O for
+//   unsplit chunks, fp32 partials and LSEs for split ones, which the combine kernel
+//   merges as soon as each virtual batch's splits are announced.
+// * The metadata, split-KV and combine kernels are launched with programmatic launch
+//   overlap.
 //
 // Every mbarrier wait is bounded: after kWaitTimeoutNs the waiting thread sets
 // an abort flag (seen by both CTAs of the cluster) and MLA_ERR_TIMEOUT in the
