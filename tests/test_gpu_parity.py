@@ -130,6 +130,29 @@ def test_active_heads(oracle_mod, case):
         assert bool((lse[:, :, real:] == 7.0).all()), "padding heads' LSE was written"
 
 
+def test_cached_workspace_across_growing_problems():
+    # The API's cached workspace grows with the problem; its control block (status word and
+    # split / combine counters) must be zero for every call, including after a larger
+    # problem has reused bytes that held split partials before.  Each call must equal the
+    # same call on a freshly zeroed workspace.
+    probs = [W.make_problem([3000, 900, 4100], s_q=1, h_q=128, seed=160),
+             W.make_problem([2500, 64, 700, 1, 130, 5000, 3100, 2000], s_q=2, h_q=64, causal=True, seed=161),
+             W.make_problem([3000, 900, 4100], s_q=1, h_q=128, seed=160)]
+    for p in probs:
+        q, kv, bt, sl = to_device(p)
+        md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q, 1)
+        assert int(ns[-1].item()) > ns.numel() - 1, "the case must split some sequence"
+        o_c, lse_c = mla.flash_mla_with_kvcache(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale)
+        ws = torch.zeros(mla.workspace_bytes(p.batch, p.s_q, p.h_q, 1, md.shape[0]), dtype=torch.uint8, device="cuda")
+        o_f, lse_f = mla.flash_mla_with_kvcache(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale,
+                                                workspace=ws)
+        torch.cuda.synchronize()
+        assert mla.read_device_status(ws) == 0
+        assert torch.equal(o_c, o_f) and torch.equal(lse_c, lse_f)
+        zb = mla.workspace_zero_bytes(p.batch, p.s_q, p.h_q, 1)
+        assert int(ws[:zb].count_nonzero().item()) == 0, "a call must leave the control block zero"
+
+
 def test_metadata_kernel_matches_host_schedule():
     rng = np.random.default_rng(7)
     for hpk in (16, 128, 256):
