@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for MLA decoding: the five decode workloads and generic problems.
+"""Seeded synthetic inputs for MLA decoding: the decode workloads and generic problems.
 
 This module draws random numbers and lays them out; it holds none of the
 attention arithmetic, so both the CUDA path and the FP64 oracle can take their
@@ -13,6 +13,11 @@ Layouts (the ones the library's C ABI takes):
 * ``block_table``  ``[batch, max_blocks_per_seq]`` int32 physical page ids, a seeded
                    Fisher-Yates permutation of the pages; unused slots are -1.
 * ``cache_seqlens`` ``[batch]`` int32.
+* FP8 cache (``Problem.fp8_kv``): ``kvcache`` is ``[num_blocks, page_size, h_kv, 656]``
+  uint8 in the "FP8 with scale" layout of the upstream FlashMLA documentation
+  ("FP8 KV Cache"): 512 float8_e4m3 latent bytes, 4 little-endian float32 scales
+  (one per 128 latent values), 64 bfloat16 RoPE values.  The generator draws the
+  e4m3 bit fields and the scales directly (it does not quantize anything).
 
 The workloads follow the decode configurations the pages benchmark (paged
 cache with 64-token pages, MQA mode d_qk = 576 / d_v = 512, variable sequence
@@ -29,6 +34,7 @@ import numpy as np
 PAGE = 64
 BF16 = 0
 FP16 = 1
+FP8_ROW_BYTES = 656
 
 
 @dataclasses.dataclass
@@ -47,6 +53,7 @@ class Problem:
     page_size: int = PAGE
     active_heads: int | None = None  # heads >= this are zero-filled (padded heads)
     seed: int = 0
+    fp8_kv: bool = False     # kvcache holds 656-byte "FP8 with scale" rows (uint8)
 
     @property
     def batch(self) -> int:
@@ -84,9 +91,13 @@ class Problem:
         """2 * (d_qk + d_v) per visible (query row, key) pair, all heads."""
         return 2.0 * (self.d_qk + self.dv) * float(self.visible().sum()) * self.h_q
 
+    def kv_row_bytes(self) -> int:
+        """Bytes of one cached token row: d_qk 16-bit values, or 656 for the FP8 cache."""
+        return FP8_ROW_BYTES if self.fp8_kv else self.d_qk * 2
+
     def kv_bytes(self) -> int:
-        """Cached rows read once: sum_b L_b * h_kv * d_qk * 2 bytes."""
-        return int(self.cache_seqlens.astype(np.int64).sum()) * self.h_kv * self.d_qk * 2
+        """Cached rows read once: sum_b L_b * h_kv * row bytes."""
+        return int(self.cache_seqlens.astype(np.int64).sum()) * self.h_kv * self.kv_row_bytes()
 
     def io_bytes(self) -> int:
         """Algorithmic bytes: KV once + Q + O (16-bit) + LSE (fp32)."""
@@ -121,6 +132,31 @@ def _normal_bits(rng: np.random.Generator, shape, std: float, dtype: int) -> np.
     return out
 
 
+def _fp8_rows(rng: np.random.Generator, n: int) -> np.ndarray:
+    """n random "FP8 with scale" token rows, uint8 [n, 656].
+
+    Latent bytes: random sign, exponent field ~ round(N(12.5, 1.5)) clipped to
+    [0, 15], uniform 3-bit fraction (the NaN pattern S.1111.111 is replaced by
+    S.1111.110); at the drawn scales (1 + U[0, 1)) * 2^-7 the values have roughly
+    unit magnitude, like a per-128-block quantized N(0, 1) latent.  RoPE: bfloat16
+    N(0, 1).
+    """
+    rows = np.empty((n, FP8_ROW_BYTES), np.uint8)
+    chunk = 1 << 16
+    for i in range(0, n, chunk):
+        m = min(chunk, n - i)
+        sign = rng.integers(0, 2, size=(m, 512), dtype=np.uint8) << np.uint8(7)
+        e = np.clip(np.rint(rng.normal(12.5, 1.5, size=(m, 512))), 0, 15).astype(np.uint8)
+        f = rng.integers(0, 8, size=(m, 512), dtype=np.uint8)
+        f[(e == 15) & (f == 7)] = 6
+        rows[i:i + m, :512] = sign | (e << np.uint8(3)) | f
+        scales = ((1.0 + rng.random((m, 4), dtype=np.float32)) * np.float32(2.0 ** -7)).astype("<f4")
+        rows[i:i + m, 512:528] = scales.view(np.uint8)
+        rope = _normal_bits(rng, (m, 64), 1.0, BF16).astype("<u2")
+        rows[i:i + m, 528:] = rope.view(np.uint8)
+    return rows
+
+
 def make_problem(
     seqlens,
     *,
@@ -138,13 +174,18 @@ def make_problem(
     extra_pages: int = 0,
     extra_table_cols: int = 0,
     name: str = "problem",
+    fp8_kv: bool = False,
 ) -> Problem:
     """Seeded problem with the given sequence lengths.
 
     ``poison`` fills what a correct kernel must never use with NaN: the tail
     rows of each sequence's last page and every page no sequence owns
     (``extra_pages`` of them).  Unused block-table slots are always -1.
+    ``fp8_kv`` draws an "FP8 with scale" cache (bfloat16 q, d_qk = 576); its
+    poison is all-ones bytes (NaN latent values, scales and RoPE values).
     """
+    if fp8_kv and (dtype != BF16 or d_qk != 576):
+        raise ValueError("the FP8 cache goes with bfloat16 queries and d_qk = 576")
     rng = np.random.Generator(np.random.PCG64(seed))
     seqlens = np.asarray(seqlens, dtype=np.int32)
     b = seqlens.size
@@ -156,7 +197,10 @@ def make_problem(
     q = _normal_bits(rng, (b, s_q, h_q, d_qk), std, dtype)
     if active_heads is not None and active_heads < h_q:
         q[:, :, active_heads:, :] = 0
-    kv = _normal_bits(rng, (num_blocks, PAGE, h_kv, d_qk), std, dtype)
+    if fp8_kv:
+        kv = _fp8_rows(rng, num_blocks * PAGE * h_kv).reshape(num_blocks, PAGE, h_kv, FP8_ROW_BYTES)
+    else:
+        kv = _normal_bits(rng, (num_blocks, PAGE, h_kv, d_qk), std, dtype)
 
     perm = rng.permutation(num_blocks).astype(np.int32)
     table = np.full((b, max_blocks), -1, np.int32)
@@ -166,7 +210,7 @@ def make_problem(
         pos += n
 
     if poison:
-        nan_bits = np.uint16(0x7FC0) if dtype == BF16 else np.uint16(0x7E00)
+        nan_bits = np.uint8(0xFF) if fp8_kv else np.uint16(0x7FC0) if dtype == BF16 else np.uint16(0x7E00)
         for i, L in enumerate(seqlens):
             n = nblk[i]
             if n and int(L) % PAGE:
@@ -178,20 +222,21 @@ def make_problem(
         scale = 1.0 / math.sqrt(d_qk)
     return Problem(name=name, q=q, kvcache=kv, block_table=table, cache_seqlens=seqlens,
                    dtype=dtype, causal=causal, scale=float(scale), active_heads=active_heads,
-                   seed=seed)
+                   seed=seed, fp8_kv=fp8_kv)
 
 
 # ----------------------------------------------------------------------------
-# The five decode workloads.  Workload k draws from seed 1000 + k.
+# The decode workloads: the five decode configurations, and the compute one over an
+# FP8 cache.  Workload k (1-based position in WORKLOADS) draws from seed 1000 + k.
 # ----------------------------------------------------------------------------
 
-WORKLOADS = ("tiny", "compute", "spec_padded", "long_split", "fp16_norope")
+WORKLOADS = ("tiny", "compute", "spec_padded", "long_split", "fp16_norope", "fp8_compute")
 
 
 def workload_seqlens(name: str, rng: np.random.Generator) -> np.ndarray:
     if name == "tiny":
         return np.array([256, 193], np.int32)
-    if name == "compute":
+    if name in ("compute", "fp8_compute"):
         return rng.integers(1024, 8192, size=64, endpoint=True).astype(np.int32)
     if name == "spec_padded":
         return rng.integers(4096 - 512, 4096 + 512, size=128, endpoint=True).astype(np.int32)
@@ -204,7 +249,7 @@ def workload_seqlens(name: str, rng: np.random.Generator) -> np.ndarray:
 
 
 def make_workload(name: str, *, poison: bool = False, seqlens=None) -> Problem:
-    """One of the five decode workloads (synthetic data, fixed seed 1000 + index).
+    """One of the decode workloads (synthetic data, fixed seed 1000 + index).
 
     ``seqlens`` overrides the sequence lengths (for scaled-down parity cases with
     the same head / dtype / mask structure).
@@ -225,4 +270,6 @@ def make_workload(name: str, *, poison: bool = False, seqlens=None) -> Problem:
     if name == "fp16_norope":
         return make_problem(L, s_q=4, h_q=64, d_qk=512, causal=True, dtype=FP16, std=0.5,
                             **common)
+    if name == "fp8_compute":
+        return make_problem(L, s_q=1, h_q=128, d_qk=576, fp8_kv=True, **common)
     raise KeyError(name)

@@ -21,6 +21,14 @@ Functions and the passages they follow (page title, section):
 * :func:`combine` -- the log-sum-exp merge of such partials.
 * :func:`decode_rows` -- :func:`decode` for selected rows of a large problem.
 * :func:`half_bits_to_float64` -- exact decoding of bfloat16 / float16 bits.
+* :func:`e4m3_to_float64`, :func:`dequant_fp8` -- the "FP8 with scale" KV cache
+  of the upstream FlashMLA documentation ("FP8 KV Cache" section, reproduced on
+  the "FlashMLA vLLM Optimization" page): 656-byte token rows of 512
+  float8_e4m3 latent values, 4 float32 scales and 64 bfloat16 RoPE values,
+  dequantized to bfloat16.
+* :func:`decode_fp8`, :func:`decode_rows_fp8` -- attention over such a cache:
+  the page says the kernel dequantizes the cache to bfloat16 and computes in
+  bfloat16, so this is :func:`decode` of the dequantized rows.
 
 Every function here is pinned by tests in ``tests/test_oracle_pins.py`` against
 closed forms, brute force through an independent library path, invariants and
@@ -92,6 +100,10 @@ def _load():
             lib.mla_oracle_combine.restype = None
             lib.mla_oracle_half_to_double.argtypes = [ctypes.c_uint16, ctypes.c_int]
             lib.mla_oracle_half_to_double.restype = ctypes.c_double
+            lib.mla_oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+            lib.mla_oracle_e4m3_to_double.restype = ctypes.c_double
+            lib.mla_oracle_dequant_fp8_rows.argtypes = [P, ctypes.c_long, P]
+            lib.mla_oracle_dequant_fp8_rows.restype = None
             lib.mla_oracle_num_threads.argtypes = []
             lib.mla_oracle_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -111,7 +123,8 @@ class use_library:
         self._saved = _lib
         lib = ctypes.CDLL(self.path)
         for name in ("mla_oracle_decode", "mla_oracle_decode_range", "mla_oracle_decode_rows",
-                     "mla_oracle_combine", "mla_oracle_half_to_double", "mla_oracle_num_threads"):
+                     "mla_oracle_combine", "mla_oracle_half_to_double", "mla_oracle_num_threads",
+                     "mla_oracle_e4m3_to_double", "mla_oracle_dequant_fp8_rows"):
             src = getattr(self._saved, name)
             dst = getattr(lib, name)
             dst.argtypes, dst.restype = src.argtypes, src.restype
@@ -220,3 +233,36 @@ def half_bits_to_float64(bits, dtype=BF16) -> np.ndarray:
     f = _load().mla_oracle_half_to_double
     flat = [f(int(x), dtype) for x in bits.ravel()]
     return np.array(flat, dtype=np.float64).reshape(bits.shape)
+
+
+FP8_ROW_BYTES = 656  # bytes per token of the "FP8 with scale" cache
+
+
+def e4m3_to_float64(codes) -> np.ndarray:
+    """Decode float8_e4m3 bytes exactly (NaN for S.1111.111)."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    f = _load().mla_oracle_e4m3_to_double
+    return np.array([f(int(x)) for x in codes.ravel()], dtype=np.float64).reshape(codes.shape)
+
+
+def dequant_fp8(kv_u8) -> np.ndarray:
+    """Dequantize an "FP8 with scale" cache [..., 656] uint8 into bfloat16 bits [..., 576]."""
+    kv_u8 = np.ascontiguousarray(kv_u8, dtype=np.uint8)
+    if kv_u8.shape[-1] != FP8_ROW_BYTES:
+        raise ValueError("an FP8 cache row is 656 bytes")
+    n = kv_u8.size // FP8_ROW_BYTES
+    out = np.empty(kv_u8.shape[:-1] + (576,), np.uint16)
+    _load().mla_oracle_dequant_fp8_rows(_ptr(kv_u8), n, _ptr(out))
+    return out
+
+
+def decode_fp8(q_bits, kv_u8, block_table, seqlens, dv=512, causal=False, scale=None, page_size=64):
+    """Attention over an "FP8 with scale" cache: bfloat16 q, out; d_qk = 576."""
+    return decode(q_bits, dequant_fp8(kv_u8), block_table, seqlens, dv, BF16, causal, scale, page_size)
+
+
+def decode_rows_fp8(q_bits, kv_u8, block_table, seqlens, row_ids, dv=512, causal=False, scale=None,
+                    page_size=64):
+    """:func:`decode_rows` over an "FP8 with scale" cache."""
+    return decode_rows(q_bits, dequant_fp8(kv_u8), block_table, seqlens, row_ids, dv, BF16, causal,
+                       scale, page_size)

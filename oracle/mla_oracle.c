@@ -29,6 +29,10 @@
  *   - Upstream FlashMLA documentation, FP8 KV cache format: a token row is the
  *     512-wide NoPE (latent) part followed by the 64-wide RoPE part, so V is the
  *     leading 512 columns of the row.
+ *   - Upstream FlashMLA documentation, "FP8 KV Cache": the "FP8 with scale" row of
+ *     656 bytes (512 float8_e4m3 latent values, 4 float32 scales, one per 128
+ *     values, 64 bfloat16 RoPE values), dequantized to bfloat16 before the
+ *     attention, which then runs as for a bfloat16 cache.
  *   - Upstream FlashMLA documentation, "Sparse MLA Prefill / Equivalent PyTorch
  *     code": the softmax written out (max, log-sum-exp, weights exp(P - lse)).
  * Readings where the pages are silent (each is listed in the design notes):
@@ -76,6 +80,70 @@ static double oracle_fp16_to_double(uint16_t h)
 double mla_oracle_half_to_double(uint16_t h, int dtype)
 {
     return dtype == 0 ? oracle_bf16_to_double(h) : oracle_fp16_to_double(h);
+}
+
+/* ------------------------------------------------------------------ */
+/* "FP8 with scale" KV cache rows.                                      */
+/* ------------------------------------------------------------------ */
+
+/*
+ * One 8-bit float in the E4M3 encoding (the "float8_e4m3" of the FP8 cache
+ * format; the OCP 8-bit floating-point E4M3 layout, which has no infinities):
+ * 1 sign bit, 4 exponent bits with bias 7, 3 fraction bits.  Exponent field 0
+ * holds the subnormals (m/8) * 2^-6; S.1111.111 is the only NaN, so the largest
+ * finite magnitude is 1.75 * 2^8 = 448.
+ */
+double mla_oracle_e4m3_to_double(uint8_t x)
+{
+    int sign = x >> 7;
+    int e = (x >> 3) & 0xf;
+    int m = x & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);           /* (m / 8) * 2^-6 */
+    else
+        v = ldexp((double)(8 + m), e - 10); /* (1 + m / 8) * 2^(e - 7) */
+    return sign ? -v : v;
+}
+
+/* Round a binary32 value to bfloat16 (its upper 16 bits), to nearest with ties to even. */
+static uint16_t oracle_float_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x0040u); /* NaN stays NaN */
+    uint32_t hi = u >> 16, rest = u & 0xffffu;
+    if (rest > 0x8000u || (rest == 0x8000u && (hi & 1u))) hi += 1; /* a carry into the exponent is right */
+    return (uint16_t)hi;
+}
+
+/*
+ * Dequantize n token rows of the "FP8 with scale" KV cache (upstream FlashMLA
+ * documentation reproduced on the "FlashMLA vLLM Optimization" page, section
+ * "FP8 KV Cache"): a row is 656 bytes, the 512 float8_e4m3 latent ("NoPE")
+ * values, then 4 float32 scales (scale k belongs to latent values
+ * [128k, 128k + 128)), then the 64 bfloat16 RoPE values, which are not
+ * quantized.  The kernel "dequantizes the cache to bfloat16": latent value i
+ * becomes bf16(e4m3_i * scale_{i/128}), the product taken in binary32 (the
+ * scales' type: the exact product, rounded once to binary32) and then rounded
+ * to bfloat16; the RoPE values are kept as they are.  Output: n rows of 576
+ * bfloat16 bit patterns, latent first, the layout of the 16-bit cache.
+ * Multi-byte fields are little-endian.
+ */
+void mla_oracle_dequant_fp8_rows(const uint8_t* rows, long n, uint16_t* out)
+{
+    for (long t = 0; t < n; ++t) {
+        const uint8_t* row = rows + (size_t)t * 656;
+        uint16_t* o = out + (size_t)t * 576;
+        float scale[4];
+        memcpy(scale, row + 512, sizeof scale);
+        for (int i = 0; i < 512; ++i) {
+            double exact = mla_oracle_e4m3_to_double(row[i]) * (double)scale[i / 128]; /* exact in fp64 */
+            o[i] = oracle_float_to_bf16((float)exact);
+        }
+        for (int i = 0; i < 64; ++i) memcpy(o + 512 + i, row + 528 + 2 * i, 2);
+    }
 }
 
 int mla_oracle_num_threads(void)

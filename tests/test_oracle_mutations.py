@@ -4,7 +4,8 @@ Each case compiles a copy of the oracle source with one planted mistake (on the
 CPU, in a temporary directory) and runs the pin tests against it: at least one
 pin must fail.  This shows the pins constrain every term of the definition
 (scale, V columns, causal offset, kv-head mapping, page indexing, LSE base, the
-combine weights).
+combine weights, and the FP8 cache's scale blocks, e4m3 exponent bias and
+subnormals, RoPE offset and bfloat16 rounding).
 """
 import os
 import subprocess
@@ -13,6 +14,7 @@ import numpy as np
 import pytest
 
 import oracle
+import tests.test_oracle_fp8_pins as fp8_pins
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "mla_oracle.c")
@@ -27,6 +29,13 @@ MUTATIONS = {
     "page_offset": ("(((size_t)page * P + (j % P))", "(((size_t)page * P + (j / P))"),
     "combine_weight": ("double w = exp(lse_parts[(size_t)k * rows + r] - L);",
                        "double w = exp(lse_parts[(size_t)k * rows + r] - M);"),
+    # the "FP8 with scale" cache
+    "fp8_scale_block": ("* (double)scale[i / 128];", "* (double)scale[(i / 64) % 4];"),
+    "fp8_exponent_bias": ("e - 10); /* (1 + m / 8)", "e - 11); /* (1 + m / 8)"),
+    "fp8_subnormal": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "fp8_rope_offset": ("row + 528 + 2 * i", "row + 526 + 2 * i"),
+    "bf16_truncation": ("if (rest > 0x8000u || (rest == 0x8000u && (hi & 1u))) hi += 1;", ""),
+    "bf16_ties_away": ("(rest == 0x8000u && (hi & 1u))", "(rest == 0x8000u)"),
 }
 
 
@@ -44,6 +53,15 @@ def _pin_calls():
     for causal in (False, True):
         calls.append((f"split_combine:{causal}",
                       lambda c=causal: pins.test_split_then_combine_equals_unsplit(oracle, c)))
+    for name in ("test_e4m3_all_codes_match_torch", "test_dequant_hand_row",
+                 "test_dequant_random_rows_match_torch"):
+        calls.append((name, lambda f=getattr(fp8_pins, name): f(oracle)))
+    for args in [(0x3A, 0.828125, 0x3F84), (0x3D, 1.2109375, 0x3FFC), (0x3C, 1.0078125, 0x3FC2)]:
+        calls.append((f"fp8_rounding:{args}",
+                      lambda a=args: fp8_pins.test_dequant_rounds_to_nearest_even(oracle, *a)))
+    for kw in fp8_pins.FP8_BRUTE_CASES:
+        calls.append((f"fp8_brute:{kw['seqlens']}",
+                      lambda k=kw: fp8_pins.test_fp8_decode_brute_force_torch(oracle, k)))
     return calls
 
 
