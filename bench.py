@@ -49,6 +49,10 @@ DESCR = {
     "fp16_norope": "fp16 MLA decode without the rope part: batch 32, s_q=4, causal, h_q=64, d_qk=d_v=512, "
                    "cache_seqlens log-uniform in [512,16384], page 64, shuffled block_table, fp16 N(0,0.5), "
                    "scale 1/sqrt(512)",
+    "fp8_compute": "compute-bound MLA decode over an FP8-with-scale cache: batch 64, s_q=1, h_q=128, h_kv=1, "
+                   "d_qk=576, d_v=512, cache_seqlens uniform in [1024,8192], page 64, shuffled block_table, "
+                   "bf16 N(0,1) q, 656-byte cache rows (512 e4m3 latent + 4 fp32 scales + 64 bf16 rope, "
+                   "|value| <= 3.5), scale 1/sqrt(576)",
 }
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NVML_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
@@ -185,7 +189,7 @@ class Runner:
         self.torch, self.mla, self.p, self.dev = torch, mla, p, dev
         dt = torch.bfloat16 if p.dtype == W.BF16 else torch.float16
         self.q = torch.from_numpy(p.q.view(np.int16)).view(dt).to(dev)
-        self.kv = torch.from_numpy(p.kvcache.view(np.int16)).view(dt).to(dev)
+        self.kv = (torch.from_numpy(p.kvcache) if p.fp8_kv else torch.from_numpy(p.kvcache.view(np.int16)).view(dt)).to(dev)
         self.bt = torch.from_numpy(p.block_table).to(dev)
         self.sl = torch.from_numpy(p.cache_seqlens).to(dev)
         self.rows = p.s_q * p.h_q
@@ -197,7 +201,8 @@ class Runner:
         ws = torch.zeros(mla.workspace_bytes(p.batch, p.s_q, p.h_q, 1, parts), dtype=torch.uint8, device=dev)
         # padding heads (the spec_padded workload) are declared, so their outputs are skipped
         self.call = mla.DecodeCall(self.q, self.kv, self.bt, self.sl, p.dv, self.md, self.ns, causal=p.causal,
-                                   softmax_scale=p.scale, workspace=ws, active_heads=p.active_heads)
+                                   softmax_scale=p.scale, workspace=ws, active_heads=p.active_heads,
+                                   is_fp8_kvcache=p.fp8_kv)
         self.launches_per_step = 3
         stages = [lambda: mla.get_mla_metadata(self.sl, self.rows, 1, out=(self.md, self.ns)),
                   self.call.splitkv, self.call.combine]
@@ -343,6 +348,15 @@ def workload_line(p, t, peaks, src):
     return out
 
 
+def oracle_rows(oracle, p: W.Problem, ids):
+    """The oracle on flat query rows `ids` (an FP8 cache is dequantized by the oracle itself)."""
+    if p.fp8_kv:
+        return oracle.decode_rows_fp8(p.q, p.kvcache, p.block_table, p.cache_seqlens, ids, dv=p.dv,
+                                      causal=p.causal, scale=p.scale)
+    return oracle.decode_rows(p.q, p.kvcache, p.block_table, p.cache_seqlens, ids, dv=p.dv, dtype=p.dtype,
+                              causal=p.causal, scale=p.scale)
+
+
 def cpu_baseline(p: W.Problem, target_s: float, seed=0):
     """The FP64 oracle on a bounded sample of rows of the same workload."""
     import oracle
@@ -356,8 +370,7 @@ def cpu_baseline(p: W.Problem, target_s: float, seed=0):
     def run(n):
         ids = np.sort(order[:n]).astype(np.int64)
         t0 = time.perf_counter()
-        oracle.decode_rows(p.q, p.kvcache, p.block_table, p.cache_seqlens, ids, dv=p.dv, dtype=p.dtype,
-                           causal=p.causal, scale=p.scale)
+        oracle_rows(oracle, p, ids)
         dt = time.perf_counter() - t0
         return dt, float(2.0 * (p.d_qk + p.dv) * vis[ids].sum())
 
@@ -378,14 +391,15 @@ def e2e(torch, mla, p: W.Problem, steps: int):
     """Same metric through the public call with pinned host buffers, copies inside the timed region."""
     dt = torch.bfloat16 if p.dtype == W.BF16 else torch.float16
     q = torch.from_numpy(p.q.view(np.int16)).view(dt).pin_memory()
-    kv = torch.from_numpy(p.kvcache.view(np.int16)).view(dt).pin_memory()
+    kv = (torch.from_numpy(p.kvcache) if p.fp8_kv else torch.from_numpy(p.kvcache.view(np.int16)).view(dt)).pin_memory()
     bt = torch.from_numpy(p.block_table).pin_memory()
     sl = torch.from_numpy(p.cache_seqlens).pin_memory()
     rows = p.s_q * p.h_q
 
     def one():
         md, ns = mla.get_mla_metadata(sl.cuda(non_blocking=True), rows, 1)
-        return mla.flash_mla_with_kvcache(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale)
+        return mla.flash_mla_with_kvcache(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale,
+                                          is_fp8_kvcache=p.fp8_kv)
 
     for _ in range(2):
         one()
@@ -399,7 +413,7 @@ def e2e(torch, mla, p: W.Problem, steps: int):
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1))
     ms = float(np.mean(times))
-    h2d = q.numel() * 2 + kv.numel() * 2 + bt.numel() * 4 + 2 * sl.numel() * 4
+    h2d = q.numel() * 2 + kv.numel() * kv.element_size() + bt.numel() * 4 + 2 * sl.numel() * 4
     d2h = o.numel() * 2 + lse.numel() * 4
     return {"value": round(p.flops() / (ms * 1e-3) / 1e12, 3), "unit": "TFLOPS", "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
@@ -518,8 +532,7 @@ def run_reference(args):
     while True:
         ids = np.sort(order[:n]).astype(np.int64)
         t0 = time.perf_counter()
-        oracle.decode_rows(p.q, p.kvcache, p.block_table, p.cache_seqlens, ids, dv=p.dv, dtype=p.dtype,
-                           causal=p.causal, scale=p.scale)
+        oracle_rows(oracle, p, ids)
         dt = time.perf_counter() - t0
         if dt >= per_step / 4 or n >= rows_total:
             break
@@ -530,8 +543,7 @@ def run_reference(args):
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        oracle.decode_rows(p.q, p.kvcache, p.block_table, p.cache_seqlens, ids, dv=p.dv, dtype=p.dtype,
-                           causal=p.causal, scale=p.scale)
+        oracle_rows(oracle, p, ids)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     s = float(np.mean(times))

@@ -28,7 +28,9 @@
  *
  * Array layouts (all row-major / C order):
  *   q             [batch, s_q, h_q, d_qk]             bf16 or fp16
- *   kvcache       [num_blocks, 64, h_kv, d_qk]        same dtype as q
+ *   kvcache       [num_blocks, 64, h_kv, d_qk]        same dtype as q, or, with
+ *                 [num_blocks, 64, h_kv, 656] bytes   dtype MLA_BF16_FP8KV, "FP8 with scale"
+ *                                                     rows (see mla_dtype)
  *   block_table   [batch, max_blocks_per_seq] int32   physical page ids; only the
  *                                                     first ceil(L_b / 64) entries
  *                                                     of row b are read
@@ -70,7 +72,17 @@ typedef enum {
                                  or a sequence needs more than max_blocks_per_seq pages */
 } mla_status;
 
-typedef enum { MLA_BF16 = 0, MLA_FP16 = 1 } mla_dtype;
+/*
+ * Data types of a call.  MLA_BF16 / MLA_FP16: q, kvcache and o all of that type.
+ * MLA_BF16_FP8KV: q and o bfloat16, kvcache in the "FP8 with scale" format of the
+ * upstream FlashMLA documentation ("FP8 KV Cache" section): each token row is 656
+ * bytes, 512 float8_e4m3 latent values, then 4 little-endian float32 scales (the
+ * k-th for latent values [128k, 128k + 128)), then the 64 bfloat16 RoPE values
+ * (not quantized); d_qk must be 576.  The kernel dequantizes each latent value to
+ * bfloat16 as bf16(e4m3 * scale), the product in float32 rounded to nearest even,
+ * and computes in bfloat16 as for a bfloat16 cache.
+ */
+typedef enum { MLA_BF16 = 0, MLA_FP16 = 1, MLA_BF16_FP8KV = 2 } mla_dtype;
 
 /* Message for a status code; never NULL. */
 MLA_API const char* mla_status_string(int status);
@@ -144,8 +156,9 @@ MLA_API size_t mla_decode_workspace_zero_bytes(int batch, int s_q, int h_q, int 
  *   lse    = log(sum_j exp(x_j))                 (-inf when n = 0)
  *   o      = sum_j exp(x_j - lse) * k_j[0:512]   (0 when n = 0)
  *
- *   q, kvcache      device, dtype `dtype`, 16-byte aligned
- *   d_qk            576 or 512;  dv must be 512;  h_kv must be 1;  page_size must be 64
+ *   q, kvcache      device, dtype `dtype` (see mla_dtype), 16-byte aligned
+ *   d_qk            576 or 512 (576 for MLA_BF16_FP8KV);  dv must be 512;  h_kv must be 1;
+ *                   page_size must be 64
  *   block_table     device int32 [batch, max_blocks_per_seq]
  *   cache_seqlens   device int32 [batch]  (the same array given to mla_get_metadata)
  *   tile_md, num_splits, num_parts   from mla_get_metadata for this batch
@@ -159,7 +172,7 @@ MLA_API size_t mla_decode_workspace_zero_bytes(int batch, int s_q, int h_q, int 
  *                   combine skips them.  A value that is not a multiple of 8 in
  *                   (0, h_q] (0 included), or an h_q that is not a multiple of 8,
  *                   means every head is real.
- *   o               device [batch, s_q, h_q, 512], dtype `dtype`, 16-byte aligned, written
+ *   o               device [batch, s_q, h_q, 512], dtype of q, 16-byte aligned, written
  *                   (real heads)
  *   lse             device float32 [batch, s_q, h_q], written (real heads)
  *   workspace       device, >= mla_decode_workspace_bytes(...), 256-byte aligned

@@ -19,6 +19,8 @@ import torch
 from . import _lib
 
 _DTYPES = {torch.bfloat16: 0, torch.float16: 1}
+MLA_BF16_FP8KV = 2   # bfloat16 q / o over an "FP8 with scale" cache (656-byte rows)
+FP8_ROW_BYTES = 656
 _workspaces: dict = {}
 
 
@@ -122,9 +124,15 @@ class DecodeCall:
     """Marshalled arguments of one decode call (device tensors), reusable across stages."""
 
     def __init__(self, q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata, num_splits,
-                 causal=False, softmax_scale=None, workspace=None, out=None, lse=None, active_heads=None):
+                 causal=False, softmax_scale=None, workspace=None, out=None, lse=None, active_heads=None,
+                 is_fp8_kvcache=False):
         dev = q.device
-        if q.dtype not in _DTYPES or kvcache.dtype != q.dtype:
+        if is_fp8_kvcache:
+            if q.dtype != torch.bfloat16 or kvcache.dtype != torch.uint8 or kvcache.shape[-1] != FP8_ROW_BYTES:
+                raise ValueError("an FP8 cache takes bfloat16 q and a uint8 kvcache of 656-byte rows")
+            if q.shape[-1] != 576:
+                raise ValueError("an FP8 cache has d_qk = 576")
+        elif q.dtype not in _DTYPES or kvcache.dtype != q.dtype:
             raise ValueError("q and kvcache must both be bfloat16 or both float16")
         for name, t in (("q", q), ("kvcache", kvcache), ("block_table", block_table),
                         ("cache_seqlens", cache_seqlens), ("tile_scheduler_metadata", tile_scheduler_metadata),
@@ -135,7 +143,8 @@ class DecodeCall:
             raise ValueError("block_table and cache_seqlens must be int32")
         b, s_q, h_q, d_qk = q.shape
         num_blocks, page, h_kv, d2 = kvcache.shape
-        if d2 != d_qk or block_table.dim() != 2 or block_table.shape[0] != b or cache_seqlens.numel() != b:
+        if ((not is_fp8_kvcache and d2 != d_qk) or block_table.dim() != 2 or block_table.shape[0] != b
+                or cache_seqlens.numel() != b):
             raise ValueError("inconsistent shapes")
         num_parts = tile_scheduler_metadata.shape[0]
         if out is None:
@@ -150,11 +159,12 @@ class DecodeCall:
         self.out, self.lse, self.workspace = out, lse, workspace
         self._keep = (q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits)
         active = 0 if active_heads is None else int(active_heads)  # 0: every head is real
+        dtype = MLA_BF16_FP8KV if is_fp8_kvcache else _DTYPES[q.dtype]
         self.args = (_ptr(q), b, s_q, h_q, d_qk, _ptr(kvcache), num_blocks, page, h_kv, _ptr(block_table),
-                     block_table.shape[1], _ptr(cache_seqlens), dv, _DTYPES[q.dtype],
+                     block_table.shape[1], _ptr(cache_seqlens), dv, dtype,
                      _ptr(tile_scheduler_metadata), num_parts, _ptr(num_splits), int(bool(causal)), scale,
                      active, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel())
-        self.combine_args = (b, s_q, h_q, h_kv, dv, _DTYPES[q.dtype], _ptr(num_splits), num_parts, active,
+        self.combine_args = (b, s_q, h_q, h_kv, dv, dtype, _ptr(num_splits), num_parts, active,
                              _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel())
 
     def run(self):
@@ -178,8 +188,14 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
                            cache_seqlens: torch.Tensor, dv: int, tile_scheduler_metadata: torch.Tensor,
                            num_splits: torch.Tensor, causal: bool = False, softmax_scale: float | None = None,
                            workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
-                           lse: torch.Tensor | None = None, active_heads: int | None = None):
+                           lse: torch.Tensor | None = None, active_heads: int | None = None,
+                           is_fp8_kvcache: bool = False):
     """MLA decode over a paged cache; returns ``(o [b, s_q, h_q, dv], lse [b, s_q, h_q] float32)``.
+
+    ``is_fp8_kvcache``: ``kvcache`` is uint8 [num_blocks, 64, h_kv, 656] in the "FP8
+    with scale" format of the upstream FlashMLA documentation ("FP8 KV Cache": 512
+    float8_e4m3 latent values, 4 float32 scales, 64 bfloat16 RoPE values per token),
+    ``q`` bfloat16 with d_qk = 576; the cache is dequantized to bfloat16 in the kernel.
 
     ``active_heads``: heads ``[active_heads, h_q)`` are padding whose outputs are not
     written (a multiple of 8 no larger than ``h_q``; anything else means all heads).
@@ -198,7 +214,7 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
             (q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits))
     call = DecodeCall(q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata, num_splits,
                       causal=causal, softmax_scale=softmax_scale, workspace=workspace, out=out, lse=lse,
-                      active_heads=active_heads)
+                      active_heads=active_heads, is_fp8_kvcache=is_fp8_kvcache)
     out, lse = call.run()
     if host:
         return out.cpu(), lse.cpu()

@@ -56,6 +56,25 @@
 namespace mla {
 
 constexpr int kThreads = 256;          // 4 softmax warps + K loader + MMA issuer + V loader + Q loader
+// "FP8 with scale" cache (upstream FlashMLA documentation, "FP8 KV Cache"): 656-byte token rows
+// of 512 float8_e4m3 latent values, 4 float32 scales (one per 128 latent values) and 64 bfloat16
+// RoPE values.  Its kernel adds two warpgroups of converter warps that dequantize raw rows from
+// shared memory into the bfloat16 K and V stages the MMAs read.
+constexpr int kThreadsFp8 = 512;
+constexpr int kConvWarp0 = 8;          // converter warps 8-15
+constexpr int kConvWarps = 8;
+constexpr int kFp8Row = 656;
+constexpr int kRawKBytes = 32 * kFp8Row;       // this CTA's 32 token rows of a page, as stored
+constexpr int kRawVBytes = 2 * 4096 + 512;     // the peer's 32 rows: this CTA's two 128-value latent
+                                               // slices (V columns) and the 4 scales of each row
+// Registers per thread in the FP8 kernel: the launch holds 65536 / 512 = 128 each; the loader /
+// MMA warpgroup and the two converter warpgroups give theirs up to the softmax warpgroup.
+constexpr uint32_t kRegsLaunchFp8 = 128;
+constexpr uint32_t kRegsLoadersFp8 = 72;
+constexpr uint32_t kRegsConvFp8 = 96;
+constexpr uint32_t kRegsSoftmaxFp8 = 248;
+static_assert(128 * (kRegsLoadersFp8 + kRegsSoftmaxFp8 + 2 * kRegsConvFp8) <= kThreadsFp8 * kRegsLaunchFp8,
+              "register split exceeds the launch's registers");
 constexpr int kKWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kVWarp = 6;
@@ -72,25 +91,31 @@ constexpr int kWorkspaceHeader = 256;
 constexpr int kNumMaps = 7;  // tensor maps of the split-KV kernel: Q, K, V, O, split partials, and O and
                              // split partials with 8-row boxes
 
-// Shared-memory plan of one CTA (each CTA of the pair owns 64 query rows).
-template <bool kRope>
+// Shared-memory plan of one CTA (each CTA of the pair owns 64 query rows).  The FP8 kernel
+// trades a K stage and a V stage for rings of raw cache rows.
+template <bool kRope, bool kFp8 = false>
 struct Layout {
     static constexpr int kBoxes = kRope ? 9 : 8;               // 64-column boxes in a d_qk row
     static constexpr int kQSmemBoxes = kBoxes - kQTmemBoxes;   // Q boxes kept in shared memory
     static constexpr int kQBytes = kQSmemBoxes * 8192;         // 64 rows, one SW128 box per 64 columns
     static constexpr int kKBytes = kBoxes * 4096;              // K: this CTA's 32 tokens of a page x d_qk
-    static constexpr int kKStages = 3;
+    static constexpr int kKStages = kFp8 ? 2 : 3;
     static constexpr int kVBytes = 4 * 8192;                   // V: 64 tokens x this CTA's 256 d_v columns
+    static constexpr int kVStages = kFp8 ? 1 : 2;
     static constexpr int kPBytes = 8192;                       // P: 64 rows x 64 tokens, 16-bit
     static constexpr int kKSteps = kBoxes * 4;                 // K=16 MMA steps of Q K^T
+    static constexpr int kRawKStages = kFp8 ? 3 : 0;
+    static constexpr int kRawVStages = kFp8 ? 2 : 0;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;              // kKStages stages
-    static constexpr int kOffV = kOffK + kKStages * kKBytes;   // 2 stages
-    static constexpr int kOffP = kOffV + 2 * kVBytes;          // 2 buffers
-    static constexpr int kOffRed = kOffP + 2 * kPBytes;        // 3 x 128 floats: 2 page row-max halves, row sums
+    static constexpr int kOffV = kOffK + kKStages * kKBytes;   // kVStages stages
+    static constexpr int kOffP = kOffV + kVStages * kVBytes;   // 2 buffers
+    static constexpr int kOffRawK = kOffP + 2 * kPBytes;       // raw rows (FP8 cache only)
+    static constexpr int kOffRawV = kOffRawK + kRawKStages * kRawKBytes;
+    static constexpr int kOffRed = kOffRawV + kRawVStages * kRawVBytes;  // 3 x 128 floats: 2 page row-max halves, row sums
     static constexpr int kRedBytes = 3 * 128 * 4;
     static constexpr int kOffBar = kOffRed + kRedBytes;
-    static constexpr int kBarBytes = 256;
+    static constexpr int kBarBytes = 384;
     static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
 };
 
@@ -109,7 +134,12 @@ enum BarSlot : int {
     kBarDrain = 20,   // leader
     kBarTail = 21,    // both: V load of a sequence's last page (local)
     kBarPair = 22,    // both: 2 slots, rendezvous of softmax warps {w, w ^ 2} (one arrive per warp)
-    kBarCount = 24
+    // FP8 cache only (kBarKFull / kBarVFull then count the converter warps of both CTAs):
+    kBarRawKFull = 24,   // local, 3 stages: this CTA's raw rows of a page landed
+    kBarRawKEmpty = 27,  // local, 3 stages: the converter warps done with them
+    kBarRawVFull = 30,   // local, 2 stages: the peer rows' V slices and scales landed
+    kBarRawVEmpty = 32,  // local, 2 stages
+    kBarCount = 34
 };
 
 // Position in a ring of kN stages: stage index and the parity of its current use.
@@ -130,8 +160,13 @@ static_assert(kOffAbort + 4 <= Layout<true>::kBarBytes, "barrier area too small"
 static_assert(2 * Layout<true>::kPBytes >= 4 * 4096 && 2 * Layout<false>::kPBytes >= 4 * 4096,
               "epilogue staging (4 KB per softmax warp) must fit in the P buffers");
 static_assert(kTmemQ + 8 * 4 * kQTmemBoxes == kTmemCols, "tensor memory plan");
-static_assert(Layout<true>::kSmemBytes <= 232448 && Layout<false>::kSmemBytes <= 232448,
+static_assert(Layout<true>::kSmemBytes <= 232448 && Layout<false>::kSmemBytes <= 232448 &&
+                  Layout<true, true>::kSmemBytes <= 232448,
               "shared memory plan exceeds 227 KB");
+static_assert(Layout<true, true>::kOffK % 1024 == 0 && Layout<true, true>::kOffV % 1024 == 0 &&
+                  Layout<true, true>::kOffP % 1024 == 0 && Layout<true, true>::kOffRawK % 128 == 0 &&
+                  Layout<true, true>::kOffRawV % 128 == 0 && kRawKBytes % 128 == 0 && kRawVBytes % 128 == 0,
+              "FP8 kernel: operand tiles 1024-byte aligned, raw rows 128-byte aligned");
 static_assert(Layout<true>::kOffQ % 1024 == 0 && Layout<true>::kOffK % 1024 == 0 && Layout<true>::kOffV % 1024 == 0 &&
                   Layout<true>::kOffP % 1024 == 0 && Layout<false>::kOffK % 1024 == 0 &&
                   Layout<false>::kOffV % 1024 == 0 && Layout<false>::kOffP % 1024 == 0,
@@ -248,14 +283,16 @@ __device__ __forceinline__ int page_of(const DecodeParams& p, const int32_t* tab
 //   O   columns [0, 256):  d_v chunk i (256 wide) at [128 i, 128 i + 128)
 //   S   columns [256, 288) and [288, 320): two page buffers
 // Thread t of the softmax warps owns row t % 64 and token / d_v half t / 64.
-template <bool kRope, bool kFp16, bool kPadHeads>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <bool kRope, bool kFp16, bool kPadHeads, bool kFp8 = false>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
     mla_splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                        const __grid_constant__ CUtensorMap tm_oacc, const __grid_constant__ CUtensorMap tm_o8,
                        const __grid_constant__ CUtensorMap tm_oacc8, const DecodeParams p)
 {
-    using L = Layout<kRope>;
+    static_assert(!kFp8 || (kRope && !kFp16), "the FP8 cache has d_qk = 576 and bfloat16 queries");
+    using L = Layout<kRope, kFp8>;
+    constexpr int kNumThreads = kFp8 ? kThreadsFp8 : kThreads;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_addr(smem);
@@ -278,12 +315,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar(kBarQFull), 1 + 8);
         mbar_init(bar(kBarQFree), 1);
+        // K and V stages are filled by TMA (one arrival with the byte count) or, for the FP8
+        // cache, by the 4 converter warps of each CTA.
         for (int s = 0; s < L::kKStages; ++s) {
-            mbar_init(bar(kBarKFull + s), 1);
+            mbar_init(bar(kBarKFull + s), kFp8 ? 2 * kConvWarps : 1);
             mbar_init(bar(kBarKEmpty + s), 1);
         }
+        for (int s = 0; s < L::kRawKStages; ++s) {
+            mbar_init(bar(kBarRawKFull + s), 1);
+            mbar_init(bar(kBarRawKEmpty + s), kConvWarps);
+        }
+        for (int s = 0; s < L::kRawVStages; ++s) {
+            mbar_init(bar(kBarRawVFull + s), 1);
+            mbar_init(bar(kBarRawVEmpty + s), kConvWarps);
+        }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(kBarVFull + s), 1);
+            mbar_init(bar(kBarVFull + s), kFp8 ? 2 * kConvWarps : 1);
             mbar_init(bar(kBarVEmpty + s), 1);
             mbar_init(bar(kBarSFull + s), 1);
             mbar_init(bar(kBarPFull + s), 8);
@@ -301,7 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // Query rows past the loaded box stay zero (finite) for the whole kernel.
     if (p.box_rows < 64) {
         uint4* q4 = reinterpret_cast<uint4*>(smem + L::kOffQ);
-        for (int i = threadIdx.x; i < L::kQBytes / 16; i += kThreads) q4[i] = make_uint4(0, 0, 0, 0);
+        for (int i = threadIdx.x; i < L::kQBytes / 16; i += kNumThreads) q4[i] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
     }
     if (warp == kMmaWarp) {
@@ -329,215 +376,453 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int begin_vb = md[0];
     const int begin_split = md[4];
 
-    if (warp == kQWarp) {
-        // ============================ Q producer ============================
-        // Loads the shared-memory part of each chunk's 64 query rows (columns
-        // 384 and up) once the previous chunk's Q K^T MMAs are done; the softmax
-        // warps store columns [0, 384) into tensor memory.
-        if (lane == 0) {
-            const uint32_t q_tx = L::kQSmemBoxes * p.box_rows * 128;
-            const int y_off = 64 * static_cast<int>(cta);
-            uint32_t k = 0;
-            int vb, lo, hi;
-            bool ok = true;
-            while (ok && chunks.next(vb, lo, hi)) {
-                if (hi <= lo) continue;
-                const int b = vb / p.groups, rg = vb % p.groups;
-                if (!(ok = sync.wait(bar(kBarQFree), (k & 1) ^ 1))) break;
-                if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * q_tx);
-                for (int i = 0; i < L::kQSmemBoxes; ++i)
-                    tma_load_3d_pair(s_q + i * 8192, &tm_q, lead_bar(kBarQFull), 64 * (kQTmemBoxes + i),
-                                     rg * kRowsPerGroup + y_off, b);
-                ++k;
-            }
-            if (!ok) {
-                const uint64_t t0 = global_timer_ns();  // let issued loads land (see the V producer)
-                while (global_timer_ns() - t0 < 50000000ull) {
-                }
-            }
-        }
-    } else if (warp == kKWarp) {
-        // ============================ K producer ============================
-        if (lane == 0) {
-            Ring<L::kKStages> ring;
-            int vb, lo, hi;
-            bool ok = true;
-            while (ok && chunks.next(vb, lo, hi)) {
-                if (hi <= lo) continue;
-                const int b = vb / p.groups;
-                const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-                for (int blk = lo; blk < hi; ++blk, ring.advance()) {
-                    const uint32_t st = ring.stage;
-                    if (!(ok = sync.wait(bar(kBarKEmpty + st), ring.phase ^ 1))) break;
-                    const int page = page_of(p, table, blk);
-                    if (leader) mbar_arrive_expect_tx(bar(kBarKFull + st), 2 * L::kKBytes);
-                    const uint32_t dst = s_k + st * L::kKBytes;
-                    for (int i = 0; i < L::kBoxes; ++i)
-                        tma_load_2d_pair(dst + i * 4096, &tm_k, lead_bar(kBarKFull + st), 64 * i,
-                                         page * kPage + 32 * static_cast<int>(cta));
-                }
-            }
-            if (!ok) {
-                const uint64_t t0 = global_timer_ns();  // let issued loads land (see the V producer)
-                while (global_timer_ns() - t0 < 50000000ull) {
-                }
-            }
-        }
-    } else if (warp == kVWarp) {
-        // ============================ V producer ============================
-        // The whole warp waits (uniformly) so that it can zero the rows past the end of a
-        // sequence's last page before the MMA may read them.
-        uint32_t g = 0, tails = 0;
-        int vb, lo, hi;
-        bool ok = true;
+    if (kFp8 && warp >= kConvWarp0) {
+        // ============================ converters (FP8 cache) ============================
+        // Eight warps per CTA dequantize the raw rows into the bfloat16 K and V stages the
+        // MMAs read, in the layout TMA gives the 16-bit cache (SW128 boxes of 64 columns):
+        //   K(g): this CTA's 32 rows of page g, all 576 columns: latent value i becomes
+        //         bf16(e4m3_i * scale_{i/128}) (the product in float32, then rounded to
+        //         nearest even), the 64 RoPE values are copied;
+        //   V(g): the page's 64 rows x this CTA's 256 V columns: its own 32 rows copied from
+        //         K(g), the peer's 32 rows dequantized from their raw slices; rows past the
+        //         sequence end are zero so that P = 0 never meets NaN.
+        // K runs one page ahead of V (K(g) then V(g - 1)), in the order the MMA issuer
+        // consumes them (Q K^T of page g before P V of page g - 1).  Warp cw owns the 16-byte
+        // words 2 cq and 2 cq + 1 (cq = cw & 3) of K boxes [4 ch, 4 ch + 4) (ch = cw >> 2) in every
+        // row `lane`, and copies exactly those words into V.
+        set_max_registers<kRegsLaunchFp8, kRegsConvFp8>();
+        const int cw = warp - kConvWarp0;
+        const int cq = cw & 3, ch = cw >> 2;
+        const int sw = lane & 7;  // swizzle phase of row `lane` (and of every row congruent mod 8)
+        const uint32_t k_full_lead[2] = {lead_bar(kBarKFull), lead_bar(kBarKFull + 1)};
+        const uint32_t v_full_lead = lead_bar(kBarVFull);
         auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
-        while (ok && chunks.next(vb, lo, hi)) {
-            if (hi <= lo) continue;
-            const int b = vb / p.groups;
-            const int Lb = p.seqlens[b];
-            const int tail = Lb % kPage;
-            const int last_page = pages_of(Lb) - 1;
-            const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-            for (int blk = lo; blk < hi; ++blk, ++g) {
-                const uint32_t st = g & 1;
-                if (!(ok = wwait(bar(kBarVEmpty + st), ((g >> 1) & 1) ^ 1))) break;
-                const int page = page_of(p, table, blk);
-                const uint32_t dst = s_v + st * L::kVBytes;
-                const bool is_tail = (blk == last_page) && tail != 0;
-                if (lane == 0 && leader) mbar_arrive_expect_tx(bar(kBarVFull + st), 2 * L::kVBytes);
-                if (!is_tail) {
-                    if (lane == 0) {
-                        for (int i = 0; i < 4; ++i) {
-                            const int box = 4 * (i >> 1) + 2 * static_cast<int>(cta) + (i & 1);
-                            tma_load_2d_pair(dst + i * 8192, &tm_v, lead_bar(kBarVFull + st), 64 * box, page * kPage);
-                        }
-                    }
-                } else {
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(bar(kBarTail), L::kVBytes);
-                        for (int i = 0; i < 4; ++i) {
-                            const int box = 4 * (i >> 1) + 2 * static_cast<int>(cta) + (i & 1);
-                            tma_load_2d(dst + i * 8192, &tm_v, bar(kBarTail), 64 * box, page * kPage);
-                        }
-                    }
-                    if (!(ok = wwait(bar(kBarTail), tails & 1))) break;
-                    ++tails;
-                    // rows [tail, 64) of each of the 4 boxes: contiguous bytes [tail*128, 8192)
-                    const int per_box = (kPage - tail) * 8;  // 16-byte words
-                    for (int i = lane; i < 4 * per_box; i += 32) {
-                        const int box = i / per_box, w16 = i % per_box;
-                        *reinterpret_cast<uint4*>(smem + L::kOffV + st * L::kVBytes + box * 8192 + tail * 128 +
-                                                  w16 * 16) = make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        fence_acq_rel_cluster();
-                        mbar_complete_tx_cluster(lead_bar(kBarVFull + st), L::kVBytes);
-                    }
-                }
-            }
-        }
-        if (!ok && lane == 0) {
-            // Give loads already issued (they complete on the even CTA's barriers) time
-            // to land before shared memory goes away.
-            const uint64_t t0 = global_timer_ns();
-            while (global_timer_ns() - t0 < 50000000ull) {
-            }
-        }
-    } else if (warp == kMmaWarp) {
-        // ============================ MMA issuer (even CTA) ============================
-        // The whole warp runs the loop (so addresses and descriptors stay warp-uniform);
-        // one elected lane issues each tcgen05 instruction.
-        if (leader) {
-            constexpr uint32_t idesc_qk = instr_desc_f16(kFp16, 128, 64, false);
-            constexpr uint32_t idesc_pv = instr_desc_f16(kFp16, 128, 256, true);
-            constexpr uint16_t both = 0x3;
-            // Base descriptors; a K step or a stage moves the start address, which is
-            // the low field of the descriptor (address >> 4).
-            const uint64_t q_desc = smem_desc(s_q, 16, 1024, kLayoutSW128);
-            const uint64_t k_desc = smem_desc(s_k, 16, 1024, kLayoutSW128);
-            const uint64_t p_desc = smem_desc(s_p, 16, 1024, kLayoutSW128);
-            const uint64_t v_desc = smem_desc(s_v, 8192, 1024, kLayoutSW128);
-            const bool issuer = elect_one();
-            auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
-            uint32_t g = 0, k = 0;
-            int vb, lo, hi;
-            bool ok = true;
-            auto issue_pv = [&](uint32_t gp, bool first) -> bool {
-                const uint32_t pb = gp & 1;
-                if (!wwait(bar(kBarPFull + pb), (gp >> 1) & 1)) return false;
-                if (first && !wwait(bar(kBarOFree), (k & 1) ^ 1)) return false;
-                if (!wwait(bar(kBarVFull + pb), (gp >> 1) & 1)) return false;
-                tc_fence_after();
-                if (issuer) {
-                    const uint64_t pd0 = p_desc + ((pb * L::kPBytes) >> 4);
-                    const uint64_t vd0 = v_desc + ((pb * L::kVBytes) >> 4);
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            // A = P[64 rows, 16 tokens] K-major; B = V[16 tokens, 128 d_v] of this CTA,
-                            // MN-major: 64-column boxes 8 KB apart (LBO), 8-token groups 1 KB apart (SBO).
-                            mma_ss_pair(tmem + kTmemO + 128 * i, pd0 + ((kk * 32) >> 4),
-                                        vd0 + ((2 * i * 8192 + kk * 2048) >> 4), idesc_pv,
-                                        (first && kk == 0) ? 0u : 1u);
-                        }
-                    }
-                    mma_commit_pair(bar(kBarVEmpty + pb), both);
-                    mma_commit_pair(bar(kBarPvDone + pb), both);
-                }
-                __syncwarp();
-                return true;
+        // 16 e4m3 values (one 16-byte word) times `s` -> 16 bfloat16 values (two 16-byte words),
+        // with integer and multiply instructions only (conversion instructions issue at a
+        // fraction of their rate).  An e4m3 byte in the top byte of y, shifted right by 4 with
+        // sign extension and masked, leaves its exponent and fraction in bits 20-26 of a float
+        // and its sign in bit 31: that float is the e4m3 value times 2^-120, subnormals
+        // included (the exponent field moves unbiased; both encodings keep subnormals at field
+        // 0).  Multiplying by 2^120 restores the value exactly; multiplying by s rounds the
+        // exact product once to float32, and the pack rounds it to bfloat16 (nearest even).
+        // The multiplies run two values per instruction.
+        // The e4m3 NaN pattern S.1111.111 comes out as +-480, not NaN: the format's quantizer
+        // never writes it.
+        auto dequant16 = [](const uint4 raw, const float s, uint4& lo, uint4& hi) {
+            auto bits = [](uint32_t y) {
+                return __int_as_float((static_cast<int32_t>(y) >> 4) & static_cast<int32_t>(0x87F00000u));
             };
-            Ring<L::kKStages> kring;
-            while (ok && chunks.next(vb, lo, hi)) {
-                const int n = hi - lo;
-                if (n <= 0) continue;
-                if (!(ok = wwait(bar(kBarQFull), k & 1))) break;
-                for (int j = 0; j < n && ok; ++j, kring.advance()) {
-                    const uint32_t gp = g + j;
-                    const uint32_t sb = gp & 1;
-                    const uint32_t st = kring.stage;
-                    if (!(ok = wwait(bar(kBarKFull + st), kring.phase))) break;
-                    tc_fence_after();
-                    if (issuer) {
-                        const uint64_t kd0 = k_desc + ((st * L::kKBytes) >> 4);
-                        // Q columns [0, 384) from tensor memory (8 columns per K=16 step) ...
-#pragma unroll
-                        for (int ks = 0; ks < 4 * kQTmemBoxes; ++ks)
-                            mma_ts_pair(tmem + kTmemS + 32 * sb, tmem + kTmemQ + 8 * ks,
-                                        kd0 + (((ks >> 2) * 4096 + (ks & 3) * 32) >> 4), idesc_qk, ks > 0 ? 1u : 0u);
-                        // ... and the remaining columns from shared memory.
-#pragma unroll
-                        for (int ks = 4 * kQTmemBoxes; ks < L::kKSteps; ++ks) {
-                            const int box = ks >> 2, sub = ks & 3;
-                            mma_ss_pair(tmem + kTmemS + 32 * sb, q_desc + (((box - kQTmemBoxes) * 8192 + sub * 32) >> 4),
-                                        kd0 + ((box * 4096 + sub * 32) >> 4), idesc_qk, 1u);
-                        }
-                        mma_commit_pair(bar(kBarKEmpty + st), both);
-                        mma_commit_pair(bar(kBarSFull + sb), both);
-                        if (j == n - 1) mma_commit_pair(bar(kBarQFree), both);
-                    }
-                    __syncwarp();
-                    if (j > 0) ok = issue_pv(gp - 1, j == 1);
-                }
-                if (ok) ok = issue_pv(g + n - 1, n == 1);
-                if (ok && issuer) mma_commit_pair(bar(kBarOFull), both);
-                __syncwarp();
-                g += n;
-                ++k;
+            // two values per multiply instruction (the packed float32 form, same rounding)
+            auto pack = [s, &bits](uint32_t y0, uint32_t y1) {  // y0 -> low half
+                const float2 v = fmul2(fmul2(make_float2(bits(y0), bits(y1)), make_float2(0x1p120f, 0x1p120f)),
+                                       make_float2(s, s));
+                const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+                return *reinterpret_cast<const uint32_t*>(&h);
+            };
+            auto word = [&](uint32_t w, uint32_t& a, uint32_t& b) {  // bytes 0, 1 -> a; bytes 2, 3 -> b
+                a = pack(w << 24, w << 16);
+                b = pack(w << 8, w);
+            };
+            word(raw.x, lo.x, lo.y);
+            word(raw.y, lo.z, lo.w);
+            word(raw.z, hi.x, hi.y);
+            word(raw.w, hi.z, hi.w);
+        };
+        // Each converter warp makes its writes visible to the tensor core and arrives on the
+        // even CTA's barrier (16 arrivals: 8 warps x 2 CTAs).
+        auto publish = [&](uint32_t lead) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader)
+                    mbar_arrive(lead);
+                else
+                    mbar_arrive_remote(lead);
             }
-            // Every issued MMA completes before tensor memory is released.
-            if (issuer) {
-                mma_commit_pair(bar(kBarDrain), 0x1);
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(bar(kBarDrain), 0) && global_timer_ns() - t0 < 100000000ull) {
+        };
+        Ring<L::kKStages> kring;
+        Ring<L::kRawKStages> rk;
+        Ring<L::kRawVStages> rv;
+        uint32_t gv = 0;              // pages whose V stage has been filled
+        int prev_valid = -1;          // valid rows of the page waiting for its V stage (-1: none)
+        uint32_t prev_kstage = 0;
+        bool ok = true;
+        // V stage of the previous page: own rows from its K stage, the peer's from raw slices.
+        auto fill_v = [&]() -> bool {
+            if (!wwait(bar(kBarRawVFull + rv.stage), rv.phase)) return false;
+            if (!wwait(bar(kBarVEmpty), (gv & 1) ^ 1)) return false;
+            uint8_t* vst = smem + L::kOffV;
+            const uint8_t* kst = smem + L::kOffK + prev_kstage * L::kKBytes;
+            const int own0 = 32 * static_cast<int>(cta), peer0 = 32 - own0;
+            // All loads first, then the stores (as for K).  V box jv holds K box
+            // 4 (jv >> 1) + 2 cta + (jv & 1): this warp's own-row words are in V boxes 2 ch, 2 ch + 1.
+            const int kk = ch;  // peer rows: slice kk holds V columns [256 kk + 128 cta, +128)
+            const int chunk8 = lane & 7;
+            const uint8_t* rawv = smem + L::kOffRawV + rv.stage * kRawVBytes;
+            uint4 own[4], peer[2];
+            float ps[2];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {  // own rows: the 16-byte words this warp wrote into K(g)
+                const int jv = 2 * ch + (i >> 1), gbox = 4 * ch + 2 * static_cast<int>(cta) + (jv & 1);
+                own[i] = *reinterpret_cast<const uint4*>(kst + gbox * 4096 + lane * 128 + (((2 * cq + (i & 1)) ^ sw) << 4));
+            }
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int t = 8 * cq + 4 * m + (lane >> 3);
+                peer[m] = *reinterpret_cast<const uint4*>(rawv + kk * 4096 + t * 128 + chunk8 * 16);
+                ps[m] = *reinterpret_cast<const float*>(rawv + 8192 + t * 16 + 4 * (2 * kk + static_cast<int>(cta)));
+            }
+            {
+                const int tok = own0 + lane;
+                const bool live = tok < prev_valid;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int jv = 2 * ch + (i >> 1);
+                    *reinterpret_cast<uint4*>(vst + jv * 8192 + tok * 128 + (((2 * cq + (i & 1)) ^ sw) << 4)) =
+                        live ? own[i] : make_uint4(0, 0, 0, 0);
+                }
+            }
+            {
+                const int jv = 2 * kk + (chunk8 >> 2);
+                const int c0 = 2 * (chunk8 & 3);
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    const int tok = peer0 + 8 * cq + 4 * m + (lane >> 3);
+                    uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+                    if (tok < prev_valid) dequant16(peer[m], ps[m], lo, hi);
+                    uint8_t* row = vst + jv * 8192 + tok * 128;
+                    *reinterpret_cast<uint4*>(row + ((c0 ^ (tok & 7)) << 4)) = lo;
+                    *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (tok & 7)) << 4)) = hi;
                 }
             }
             __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarRawVEmpty + rv.stage));
+            publish(v_full_lead);
+            rv.advance();
+            ++gv;
+            prev_valid = -1;
+            return true;
+        };
+        int vb, lo, hi;
+        while (ok && chunks.next(vb, lo, hi)) {
+            if (hi <= lo) continue;
+            const int Lb = p.seqlens[vb / p.groups];
+            for (int blk = lo; blk < hi && ok; ++blk) {
+                // ---- K(g): this CTA's 32 rows
+                if (!(ok = wwait(bar(kBarRawKFull + rk.stage), rk.phase))) break;
+                if (!(ok = wwait(bar(kBarKEmpty + kring.stage), kring.phase ^ 1))) break;
+                {
+                    // Every load of the page is issued before the first store (the compiler cannot
+                    // move loads above stores into the same shared memory), so the 8 boxes'
+                    // conversions overlap.
+                    const uint8_t* rrow = smem + L::kOffRawK + rk.stage * kRawKBytes + lane * kFp8Row;
+                    uint8_t* krow = smem + L::kOffK + kring.stage * L::kKBytes + lane * 128;
+                    uint4 raw[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        raw[m] = *reinterpret_cast<const uint4*>(rrow + 64 * (4 * ch + m) + 16 * cq);
+                    const uint4 rope = *reinterpret_cast<const uint4*>(rrow + 528 + 16 * cw);
+                    const float2 sc = *reinterpret_cast<const float2*>(rrow + 512 + 8 * ch);  // boxes 4 ch .. 4 ch + 3
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {  // box 4 ch + m: latent columns [64 (4 ch + m), +64); 16 of them
+                        uint4 w0, w1;
+                        dequant16(raw[m], m < 2 ? sc.x : sc.y, w0, w1);
+                        uint8_t* box = krow + (4 * ch + m) * 4096;
+                        *reinterpret_cast<uint4*>(box + (((2 * cq) ^ sw) << 4)) = w0;
+                        *reinterpret_cast<uint4*>(box + (((2 * cq + 1) ^ sw) << 4)) = w1;
+                    }
+                    *reinterpret_cast<uint4*>(krow + 8 * 4096 + ((cw ^ sw) << 4)) = rope;  // RoPE: box 8, copied
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarRawKEmpty + rk.stage));
+                publish(k_full_lead[kring.stage]);
+                rk.advance();
+                // ---- V(g - 1)
+                if (prev_valid >= 0 && !(ok = fill_v())) break;
+                prev_valid = min(kPage, Lb - kPage * blk);
+                prev_kstage = kring.stage;
+                kring.advance();
+            }
+        }
+        if (ok && prev_valid >= 0) ok = fill_v();
+    } else if (warp >= 4) {
+        // Warpgroup 1 (Q / K / V loaders and the MMA issuer): one thread issues; few registers.
+        if constexpr (kFp8) set_max_registers<kRegsLaunchFp8, kRegsLoadersFp8>();  // before the role split: one
+                                                                                    // instruction per warpgroup
+        if (warp == kQWarp) {
+            // ============================ Q producer ============================
+            // Loads the shared-memory part of each chunk's 64 query rows (columns
+            // 384 and up) once the previous chunk's Q K^T MMAs are done; the softmax
+            // warps store columns [0, 384) into tensor memory.
+            if (lane == 0) {
+                const uint32_t q_tx = L::kQSmemBoxes * p.box_rows * 128;
+                const int y_off = 64 * static_cast<int>(cta);
+                uint32_t k = 0;
+                int vb, lo, hi;
+                bool ok = true;
+                while (ok && chunks.next(vb, lo, hi)) {
+                    if (hi <= lo) continue;
+                    const int b = vb / p.groups, rg = vb % p.groups;
+                    if (!(ok = sync.wait(bar(kBarQFree), (k & 1) ^ 1))) break;
+                    if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * q_tx);
+                    for (int i = 0; i < L::kQSmemBoxes; ++i)
+                        tma_load_3d_pair(s_q + i * 8192, &tm_q, lead_bar(kBarQFull), 64 * (kQTmemBoxes + i),
+                                         rg * kRowsPerGroup + y_off, b);
+                    ++k;
+                }
+                if (!ok) {
+                    const uint64_t t0 = global_timer_ns();  // let issued loads land (see the V producer)
+                    while (global_timer_ns() - t0 < 50000000ull) {
+                    }
+                }
+            }
+        } else if (warp == kKWarp) {
+            // ============================ K producer ============================
+            if constexpr (kFp8) {
+                // FP8 cache: this CTA's 32 rows of each page as stored (one bulk copy), for the
+                // converters.
+                if (lane == 0) {
+                    Ring<L::kRawKStages> ring;
+                    int vb, lo, hi;
+                    bool ok = true;
+                    const uint8_t* kv = static_cast<const uint8_t*>(p.kvcache);
+                    while (ok && chunks.next(vb, lo, hi)) {
+                        if (hi <= lo) continue;
+                        const int b = vb / p.groups;
+                        const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+                        for (int blk = lo; blk < hi; ++blk, ring.advance()) {
+                            const uint32_t st = ring.stage;
+                            if (!(ok = sync.wait(bar(kBarRawKEmpty + st), ring.phase ^ 1))) break;
+                            const int page = page_of(p, table, blk);
+                            mbar_arrive_expect_tx(bar(kBarRawKFull + st), kRawKBytes);
+                            bulk_load(s_base + L::kOffRawK + st * kRawKBytes,
+                                      kv + (static_cast<size_t>(page) * kPage + 32 * cta) * kFp8Row, kRawKBytes,
+                                      bar(kBarRawKFull + st));
+                        }
+                    }
+                    if (!ok) {
+                        const uint64_t t0 = global_timer_ns();  // let issued loads land (see the V producer)
+                        while (global_timer_ns() - t0 < 50000000ull) {
+                        }
+                    }
+                }
+            } else if (lane == 0) {
+                Ring<L::kKStages> ring;
+                int vb, lo, hi;
+                bool ok = true;
+                while (ok && chunks.next(vb, lo, hi)) {
+                    if (hi <= lo) continue;
+                    const int b = vb / p.groups;
+                    const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+                    for (int blk = lo; blk < hi; ++blk, ring.advance()) {
+                        const uint32_t st = ring.stage;
+                        if (!(ok = sync.wait(bar(kBarKEmpty + st), ring.phase ^ 1))) break;
+                        const int page = page_of(p, table, blk);
+                        if (leader) mbar_arrive_expect_tx(bar(kBarKFull + st), 2 * L::kKBytes);
+                        const uint32_t dst = s_k + st * L::kKBytes;
+                        for (int i = 0; i < L::kBoxes; ++i)
+                            tma_load_2d_pair(dst + i * 4096, &tm_k, lead_bar(kBarKFull + st), 64 * i,
+                                             page * kPage + 32 * static_cast<int>(cta));
+                    }
+                }
+                if (!ok) {
+                    const uint64_t t0 = global_timer_ns();  // let issued loads land (see the V producer)
+                    while (global_timer_ns() - t0 < 50000000ull) {
+                    }
+                }
+            }
+        } else if (warp == kVWarp) {
+            if constexpr (kFp8) {
+                // ============================ V producer (FP8 cache) ============================
+                // The peer's 32 rows of each page: this CTA's two 128-value latent slices (its V
+                // columns) and the rows' scales, by TMA (tm_k: 128-byte boxes, tm_v: 16-byte boxes).
+                if (lane == 0) {
+                    Ring<L::kRawVStages> ring;
+                    int vb, lo, hi;
+                    bool ok = true;
+                    while (ok && chunks.next(vb, lo, hi)) {
+                        if (hi <= lo) continue;
+                        const int b = vb / p.groups;
+                        const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+                        for (int blk = lo; blk < hi; ++blk, ring.advance()) {
+                            const uint32_t st = ring.stage;
+                            if (!(ok = sync.wait(bar(kBarRawVEmpty + st), ring.phase ^ 1))) break;
+                            const int page = page_of(p, table, blk);
+                            const int y = page * kPage + 32 * (1 - static_cast<int>(cta));
+                            const uint32_t dst = s_base + L::kOffRawV + st * kRawVBytes;
+                            mbar_arrive_expect_tx(bar(kBarRawVFull + st), kRawVBytes);
+                            tma_load_2d(dst, &tm_k, bar(kBarRawVFull + st), 128 * static_cast<int>(cta), y);
+                            tma_load_2d(dst + 4096, &tm_k, bar(kBarRawVFull + st), 256 + 128 * static_cast<int>(cta), y);
+                            tma_load_2d(dst + 8192, &tm_v, bar(kBarRawVFull + st), 512, y);
+                        }
+                    }
+                    if (!ok) {
+                        const uint64_t t0 = global_timer_ns();  // let issued loads land (see below)
+                        while (global_timer_ns() - t0 < 50000000ull) {
+                        }
+                    }
+                }
+            } else {
+                // ============================ V producer ============================
+                // The whole warp waits (uniformly) so that it can zero the rows past the end of a
+                // sequence's last page before the MMA may read them.
+                uint32_t g = 0, tails = 0;
+                int vb, lo, hi;
+                bool ok = true;
+                auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
+                while (ok && chunks.next(vb, lo, hi)) {
+                    if (hi <= lo) continue;
+                    const int b = vb / p.groups;
+                    const int Lb = p.seqlens[b];
+                    const int tail = Lb % kPage;
+                    const int last_page = pages_of(Lb) - 1;
+                    const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+                    for (int blk = lo; blk < hi; ++blk, ++g) {
+                        const uint32_t st = g & 1;
+                        if (!(ok = wwait(bar(kBarVEmpty + st), ((g >> 1) & 1) ^ 1))) break;
+                        const int page = page_of(p, table, blk);
+                        const uint32_t dst = s_v + st * L::kVBytes;
+                        const bool is_tail = (blk == last_page) && tail != 0;
+                        if (lane == 0 && leader) mbar_arrive_expect_tx(bar(kBarVFull + st), 2 * L::kVBytes);
+                        if (!is_tail) {
+                            if (lane == 0) {
+                                for (int i = 0; i < 4; ++i) {
+                                    const int box = 4 * (i >> 1) + 2 * static_cast<int>(cta) + (i & 1);
+                                    tma_load_2d_pair(dst + i * 8192, &tm_v, lead_bar(kBarVFull + st), 64 * box, page * kPage);
+                                }
+                            }
+                        } else {
+                            if (lane == 0) {
+                                mbar_arrive_expect_tx(bar(kBarTail), L::kVBytes);
+                                for (int i = 0; i < 4; ++i) {
+                                    const int box = 4 * (i >> 1) + 2 * static_cast<int>(cta) + (i & 1);
+                                    tma_load_2d(dst + i * 8192, &tm_v, bar(kBarTail), 64 * box, page * kPage);
+                                }
+                            }
+                            if (!(ok = wwait(bar(kBarTail), tails & 1))) break;
+                            ++tails;
+                            // rows [tail, 64) of each of the 4 boxes: contiguous bytes [tail*128, 8192)
+                            const int per_box = (kPage - tail) * 8;  // 16-byte words
+                            for (int i = lane; i < 4 * per_box; i += 32) {
+                                const int box = i / per_box, w16 = i % per_box;
+                                *reinterpret_cast<uint4*>(smem + L::kOffV + st * L::kVBytes + box * 8192 + tail * 128 +
+                                                          w16 * 16) = make_uint4(0, 0, 0, 0);
+                            }
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                fence_acq_rel_cluster();
+                                mbar_complete_tx_cluster(lead_bar(kBarVFull + st), L::kVBytes);
+                            }
+                        }
+                    }
+                }
+                if (!ok && lane == 0) {
+                    // Give loads already issued (they complete on the even CTA's barriers) time
+                    // to land before shared memory goes away.
+                    const uint64_t t0 = global_timer_ns();
+                    while (global_timer_ns() - t0 < 50000000ull) {
+                    }
+                }
+            }
+        } else if (warp == kMmaWarp) {
+            // ============================ MMA issuer (even CTA) ============================
+            // The whole warp runs the loop (so addresses and descriptors stay warp-uniform);
+            // one elected lane issues each tcgen05 instruction.
+            if (leader) {
+                constexpr uint32_t idesc_qk = instr_desc_f16(kFp16, 128, 64, false);
+                constexpr uint32_t idesc_pv = instr_desc_f16(kFp16, 128, 256, true);
+                constexpr uint16_t both = 0x3;
+                // Base descriptors; a K step or a stage moves the start address, which is
+                // the low field of the descriptor (address >> 4).
+                const uint64_t q_desc = smem_desc(s_q, 16, 1024, kLayoutSW128);
+                const uint64_t k_desc = smem_desc(s_k, 16, 1024, kLayoutSW128);
+                const uint64_t p_desc = smem_desc(s_p, 16, 1024, kLayoutSW128);
+                const uint64_t v_desc = smem_desc(s_v, 8192, 1024, kLayoutSW128);
+                const bool issuer = elect_one();
+                auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
+                uint32_t g = 0, k = 0;
+                int vb, lo, hi;
+                bool ok = true;
+                auto issue_pv = [&](uint32_t gp, bool first) -> bool {
+                    const uint32_t pb = gp & 1;
+                    if (!wwait(bar(kBarPFull + pb), (gp >> 1) & 1)) return false;
+                    if (first && !wwait(bar(kBarOFree), (k & 1) ^ 1)) return false;
+                    // V stage of page gp (one stage for the FP8 cache, else it pairs with the P buffer)
+                    const uint32_t vs = L::kVStages == 1 ? 0u : pb;
+                    const uint32_t vpar = L::kVStages == 1 ? (gp & 1) : ((gp >> 1) & 1);
+                    if (!wwait(bar(kBarVFull + vs), vpar)) return false;
+                    tc_fence_after();
+                    if (issuer) {
+                        const uint64_t pd0 = p_desc + ((pb * L::kPBytes) >> 4);
+                        const uint64_t vd0 = v_desc + ((vs * L::kVBytes) >> 4);
+    #pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+    #pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                // A = P[64 rows, 16 tokens] K-major; B = V[16 tokens, 128 d_v] of this CTA,
+                                // MN-major: 64-column boxes 8 KB apart (LBO), 8-token groups 1 KB apart (SBO).
+                                mma_ss_pair(tmem + kTmemO + 128 * i, pd0 + ((kk * 32) >> 4),
+                                            vd0 + ((2 * i * 8192 + kk * 2048) >> 4), idesc_pv,
+                                            (first && kk == 0) ? 0u : 1u);
+                            }
+                        }
+                        mma_commit_pair(bar(kBarVEmpty + vs), both);
+                        mma_commit_pair(bar(kBarPvDone + pb), both);
+                    }
+                    __syncwarp();
+                    return true;
+                };
+                Ring<L::kKStages> kring;
+                while (ok && chunks.next(vb, lo, hi)) {
+                    const int n = hi - lo;
+                    if (n <= 0) continue;
+                    if (!(ok = wwait(bar(kBarQFull), k & 1))) break;
+                    for (int j = 0; j < n && ok; ++j, kring.advance()) {
+                        const uint32_t gp = g + j;
+                        const uint32_t sb = gp & 1;
+                        const uint32_t st = kring.stage;
+                        if (!(ok = wwait(bar(kBarKFull + st), kring.phase))) break;
+                        tc_fence_after();
+                        if (issuer) {
+                            const uint64_t kd0 = k_desc + ((st * L::kKBytes) >> 4);
+                            // Q columns [0, 384) from tensor memory (8 columns per K=16 step) ...
+    #pragma unroll
+                            for (int ks = 0; ks < 4 * kQTmemBoxes; ++ks)
+                                mma_ts_pair(tmem + kTmemS + 32 * sb, tmem + kTmemQ + 8 * ks,
+                                            kd0 + (((ks >> 2) * 4096 + (ks & 3) * 32) >> 4), idesc_qk, ks > 0 ? 1u : 0u);
+                            // ... and the remaining columns from shared memory.
+    #pragma unroll
+                            for (int ks = 4 * kQTmemBoxes; ks < L::kKSteps; ++ks) {
+                                const int box = ks >> 2, sub = ks & 3;
+                                mma_ss_pair(tmem + kTmemS + 32 * sb, q_desc + (((box - kQTmemBoxes) * 8192 + sub * 32) >> 4),
+                                            kd0 + ((box * 4096 + sub * 32) >> 4), idesc_qk, 1u);
+                            }
+                            mma_commit_pair(bar(kBarKEmpty + st), both);
+                            mma_commit_pair(bar(kBarSFull + sb), both);
+                            if (j == n - 1) mma_commit_pair(bar(kBarQFree), both);
+                        }
+                        __syncwarp();
+                        if (j > 0) ok = issue_pv(gp - 1, j == 1);
+                    }
+                    if (ok) ok = issue_pv(g + n - 1, n == 1);
+                    if (ok && issuer) mma_commit_pair(bar(kBarOFull), both);
+                    __syncwarp();
+                    g += n;
+                    ++k;
+                }
+                // Every issued MMA completes before tensor memory is released.
+                if (issuer) {
+                    mma_commit_pair(bar(kBarDrain), 0x1);
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar(kBarDrain), 0) && global_timer_ns() - t0 < 100000000ull) {
+                    }
+                }
+                __syncwarp();
+            }
         }
     } else {
+        if constexpr (kFp8) set_max_registers<kRegsLaunchFp8, kRegsSoftmaxFp8>();
         // ======================= softmax / correction / epilogue =======================
         const int t = threadIdx.x;             // TMEM lane
         const int r = t & 63;                  // row within this CTA's 64
@@ -1221,11 +1506,11 @@ static void workspace_pointers(void* workspace, int batch, int groups, int num_p
     prm.o_accum = reinterpret_cast<float*>(ws + control_bytes(nv) + align_up(slots * kRowsPerGroup * sizeof(float), 256));
 }
 
-template <bool kRope, bool kFp16, bool kPadHeads>
+template <bool kRope, bool kFp16, bool kPadHeads, bool kFp8>
 static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorMap* maps, const DecodeParams& prm)
 {
-    auto kern = mla_splitkv_kernel<kRope, kFp16, kPadHeads>;
-    const int smem = Layout<kRope>::kSmemBytes;
+    auto kern = mla_splitkv_kernel<kRope, kFp16, kPadHeads, kFp8>;
+    const int smem = Layout<kRope, kFp8>::kSmemBytes;
     static int configured_device = -1;  // the attribute is per device; set it once per device in use
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1233,20 +1518,28 @@ static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorM
     if (configured_device != dev) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
+        if (kFp8) {
+            // The warpgroups' register re-balancing hands out exactly what the launch holds
+            // (168 per thread); with fewer at launch, setmaxnreg.inc would never return.
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, kern);
+            if (e != cudaSuccess) return e;
+            if (fa.numRegs < static_cast<int>(kRegsLaunchFp8)) return cudaErrorInvalidConfiguration;
+        }
         configured_device = dev;
     }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
-    programmatic_launch(cfg, attr, dim3(grid), dim3(kThreads), smem, stream);
+    programmatic_launch(cfg, attr, dim3(grid), dim3(kFp8 ? kThreadsFp8 : kThreads), smem, stream);
     return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], prm);
 }
 
 // The kernel variant with padding-head logic runs only when some heads are padding.
-template <bool kRope, bool kFp16>
+template <bool kRope, bool kFp16, bool kFp8 = false>
 static cudaError_t launch_splitkv_heads(int grid, cudaStream_t st, const CUtensorMap* maps, const DecodeParams& prm)
 {
-    return prm.active_heads < prm.h_q ? launch_splitkv<kRope, kFp16, true>(grid, st, maps, prm)
-                                      : launch_splitkv<kRope, kFp16, false>(grid, st, maps, prm);
+    return prm.active_heads < prm.h_q ? launch_splitkv<kRope, kFp16, true, kFp8>(grid, st, maps, prm)
+                                      : launch_splitkv<kRope, kFp16, false, kFp8>(grid, st, maps, prm);
 }
 
 }  // namespace mla
@@ -1365,8 +1658,9 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
         num_parts <= 0 || (causal != 0 && causal != 1))
         return MLA_ERR_INVALID_ARG;
-    if (dtype != MLA_BF16 && dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
+    if (dtype != MLA_BF16 && dtype != MLA_FP16 && dtype != MLA_BF16_FP8KV) return MLA_ERR_INVALID_ARG;
     if (page_size != kPage || h_kv != 1 || (d_qk != 576 && d_qk != 512) || dv != kDv) return MLA_ERR_UNSUPPORTED;
+    if (dtype == MLA_BF16_FP8KV && d_qk != 576) return MLA_ERR_UNSUPPORTED;  // the FP8 row carries 64 RoPE values
     if (batch > 0 && (!q || !kvcache || !block_table || !cache_seqlens || !tile_md || !num_splits || !o || !lse ||
                       !workspace))
         return MLA_ERR_INVALID_ARG;
@@ -1414,11 +1708,19 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     // Q: [batch][rows][d_qk], box 64 columns x (up to) 64 rows;
     // K: cache rows, box 64 columns x 32 tokens (half a page, one CTA's share);
     // V: cache rows, box 64 columns x 64 tokens (a page).
+    // FP8 cache: rows of 656 bytes; K: boxes of 128 bytes x 32 rows (latent slices), V: boxes
+    // of 16 bytes x 32 rows (the scales), no swizzle.
+    const bool fp8 = dtype == MLA_BF16_FP8KV;
     const bool ok =
         encode_3d(&maps[0], q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 64, prm.box_rows,
                   CU_TENSOR_MAP_SWIZZLE_128B) &&
-        encode_2d(&maps[1], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage / 2, CU_TENSOR_MAP_SWIZZLE_128B) &&
-        encode_2d(&maps[2], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B) &&
+        (fp8 ? encode_2d(&maps[1], kvcache, CU_TENSOR_MAP_DATA_TYPE_UINT8, kFp8Row, kv_rows, kFp8Row, 128,
+                         kPage / 2, CU_TENSOR_MAP_SWIZZLE_NONE)
+             : encode_2d(&maps[1], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage / 2,
+                         CU_TENSOR_MAP_SWIZZLE_128B)) &&
+        (fp8 ? encode_2d(&maps[2], kvcache, CU_TENSOR_MAP_DATA_TYPE_UINT8, kFp8Row, kv_rows, kFp8Row, 16,
+                         kPage / 2, CU_TENSOR_MAP_SWIZZLE_NONE)
+             : encode_2d(&maps[2], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B)) &&
         // O: [batch][rows][512] 16-bit, stored in tiles of 64 columns x 32 rows (rows past
         // the end are clipped by the TMA unit); split partials: [slots][128][512] fp32,
         // tiles of 32 columns x 32 rows.
@@ -1439,7 +1741,9 @@ static mla_status launch_splitkv_stage(const DecodeParams& prm, const CUtensorMa
 {
     const int grid = 2 * prm.num_parts;
     cudaError_t e;
-    if (prm.d_qk == 576)
+    if (prm.dtype == MLA_BF16_FP8KV)
+        e = launch_splitkv_heads<true, false, true>(grid, st, maps, prm);
+    else if (prm.d_qk == 576)
         e = prm.dtype == MLA_FP16 ? launch_splitkv_heads<true, true>(grid, st, maps, prm)
                                   : launch_splitkv_heads<true, false>(grid, st, maps, prm);
     else
@@ -1510,7 +1814,7 @@ mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int
                               size_t workspace_bytes, void* stream)
 {
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_parts <= 0) return MLA_ERR_INVALID_ARG;
-    if (dtype != MLA_BF16 && dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
+    if (dtype != MLA_BF16 && dtype != MLA_FP16 && dtype != MLA_BF16_FP8KV) return MLA_ERR_INVALID_ARG;
     if (h_kv != 1 || dv != kDv) return MLA_ERR_UNSUPPORTED;
     if (batch == 0) return MLA_OK;
     if (!num_splits || !o || !lse || !workspace) return MLA_ERR_INVALID_ARG;

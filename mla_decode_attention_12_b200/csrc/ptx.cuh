@@ -146,6 +146,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint3
         : "memory");
 }
 
+// Bulk copy of `bytes` contiguous bytes (a multiple of 16, both addresses 16-byte
+// aligned) from global memory into this CTA's shared memory, completing on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 // TMA tiled store from this CTA's shared memory (bulk async-group completion).
 __device__ __forceinline__ void tma_store_3d(const void* map, uint32_t src, int x, int y, int z)
 {
@@ -166,6 +175,31 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // in the stream has completed and its memory writes are visible (returns at once when
 // this grid was not launched with programmatic serialization).  launch_dependents:
 // let the next grid in the stream, if it opted in, start launching now.
+// Two float32 products in one instruction (sm_100), each rounded to nearest even; subnormal
+// inputs and results are kept (no flush to zero).
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// Warpgroup-wide register re-balancing from kFrom to kTo registers per thread; every
+// warp of the warpgroup executes the same instruction.  The .inc form only raises the
+// count and .dec only lowers it, so the form is chosen from the two counts.
+template <uint32_t kFrom, uint32_t kTo>
+__device__ __forceinline__ void set_max_registers()
+{
+    static_assert(kTo % 8 == 0 && kTo >= 24 && kTo <= 256, "setmaxnreg takes a multiple of 8 in [24, 256]");
+    if constexpr (kTo > kFrom)
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kTo));
+    else if constexpr (kTo < kFrom)
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kTo));
+}
+
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

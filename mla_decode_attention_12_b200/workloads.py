@@ -135,10 +135,11 @@ def _normal_bits(rng: np.random.Generator, shape, std: float, dtype: int) -> np.
 def _fp8_rows(rng: np.random.Generator, n: int) -> np.ndarray:
     """n random "FP8 with scale" token rows, uint8 [n, 656].
 
-    Latent bytes: random sign, exponent field ~ round(N(12.5, 1.5)) clipped to
+    Latent bytes: random sign, exponent field ~ round(N(13, 1.5)) clipped to
     [0, 15], uniform 3-bit fraction (the NaN pattern S.1111.111 is replaced by
-    S.1111.110); at the drawn scales (1 + U[0, 1)) * 2^-7 the values have roughly
-    unit magnitude, like a per-128-block quantized N(0, 1) latent.  RoPE: bfloat16
+    S.1111.110).  Scales (1 + U[0, 1)) * 2^-8, the range amax / 448 takes for a
+    block of 128 N(0, 1) values, so the values are at most 3.5 in magnitude and
+    mostly below 1, like a per-128-block quantized N(0, 1) latent.  RoPE: bfloat16
     N(0, 1).
     """
     rows = np.empty((n, FP8_ROW_BYTES), np.uint8)
@@ -146,11 +147,11 @@ def _fp8_rows(rng: np.random.Generator, n: int) -> np.ndarray:
     for i in range(0, n, chunk):
         m = min(chunk, n - i)
         sign = rng.integers(0, 2, size=(m, 512), dtype=np.uint8) << np.uint8(7)
-        e = np.clip(np.rint(rng.normal(12.5, 1.5, size=(m, 512))), 0, 15).astype(np.uint8)
+        e = np.clip(np.rint(rng.normal(13.0, 1.5, size=(m, 512))), 0, 15).astype(np.uint8)
         f = rng.integers(0, 8, size=(m, 512), dtype=np.uint8)
         f[(e == 15) & (f == 7)] = 6
         rows[i:i + m, :512] = sign | (e << np.uint8(3)) | f
-        scales = ((1.0 + rng.random((m, 4), dtype=np.float32)) * np.float32(2.0 ** -7)).astype("<f4")
+        scales = ((1.0 + rng.random((m, 4), dtype=np.float32)) * np.float32(2.0 ** -8)).astype("<f4")
         rows[i:i + m, 512:528] = scales.view(np.uint8)
         rope = _normal_bits(rng, (m, 64), 1.0, BF16).astype("<u2")
         rows[i:i + m, 528:] = rope.view(np.uint8)

@@ -25,7 +25,10 @@ def tdtype(dtype: int):
 def to_device(p: W.Problem, device="cuda"):
     dt = tdtype(p.dtype)
     q = torch.from_numpy(p.q.view(np.int16)).view(dt).to(device)
-    kv = torch.from_numpy(p.kvcache.view(np.int16)).view(dt).to(device)
+    if p.fp8_kv:  # "FP8 with scale" rows stay bytes
+        kv = torch.from_numpy(p.kvcache).to(device)
+    else:
+        kv = torch.from_numpy(p.kvcache.view(np.int16)).view(dt).to(device)
     bt = torch.from_numpy(p.block_table).to(device)
     sl = torch.from_numpy(p.cache_seqlens).to(device)
     return q, kv, bt, sl
@@ -37,7 +40,7 @@ def run_gpu(p: W.Problem, device="cuda", num_parts=None, check_status=True):
     ws = torch.zeros(mla.workspace_bytes(p.batch, p.s_q, p.h_q, p.h_kv, md.shape[0]), dtype=torch.uint8,
                      device=device)
     o, lse = mla.flash_mla_with_kvcache(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale,
-                                        workspace=ws)
+                                        workspace=ws, is_fp8_kvcache=p.fp8_kv)
     torch.cuda.synchronize()
     if check_status:
         st = mla.read_device_status(ws)
@@ -67,3 +70,21 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what=""):
     assert d_l.max() <= LSE_MAX_ABS, info
     assert mae <= MAE_FACTOR * mae_round + 1e-7, info
     return info
+
+
+def oracle_full(oracle_mod, p: W.Problem):
+    """FP64 oracle result of a whole problem (16-bit or FP8 cache)."""
+    if p.fp8_kv:
+        return oracle_mod.decode_fp8(p.q, p.kvcache, p.block_table, p.cache_seqlens, dv=p.dv, causal=p.causal,
+                                     scale=p.scale)
+    return oracle_mod.decode(p.q, p.kvcache, p.block_table, p.cache_seqlens, dv=p.dv, dtype=p.dtype,
+                             causal=p.causal, scale=p.scale)
+
+
+def oracle_rows(oracle_mod, p: W.Problem, rows):
+    """FP64 oracle result of selected flat rows (b * s_q + s) * h_q + h."""
+    if p.fp8_kv:
+        return oracle_mod.decode_rows_fp8(p.q, p.kvcache, p.block_table, p.cache_seqlens, rows, dv=p.dv,
+                                          causal=p.causal, scale=p.scale)
+    return oracle_mod.decode_rows(p.q, p.kvcache, p.block_table, p.cache_seqlens, rows, dv=p.dv, dtype=p.dtype,
+                                  causal=p.causal, scale=p.scale)

@@ -74,6 +74,8 @@ def _decode(lib, **over):
     (dict(causal=2), 1), (dict(dtype=7), 1), (dict(q=(1 << 20) + 2), 1), (dict(ws=(1 << 20) + 16), 1),
     (dict(page_size=32), 2), (dict(h_kv=2), 2), (dict(d_qk=192), 2), (dict(dv=256), 2),
     (dict(ws_bytes=1000), 3),
+    # the "FP8 with scale" cache (dtype 2) carries 64 RoPE values: d_qk must be 576
+    (dict(dtype=2, d_qk=512), 2), (dict(dtype=2, kvcache=(1 << 20) + 8), 1), (dict(dtype=3), 1),
 ])
 def test_decode_rejects_bad_arguments(lib, over, code):
     assert _decode(lib, **over) == code
@@ -81,6 +83,15 @@ def test_decode_rejects_bad_arguments(lib, over, code):
 
 def test_decode_empty_batch_is_a_no_op(lib):
     assert _decode(lib, batch=0, q=None, o=None) == 0
+    assert _decode(lib, batch=0, q=None, o=None, dtype=2) == 0
+
+
+def test_combine_accepts_the_fp8_cache_dtype(lib):
+    # mla_decode_combine of an FP8-cache call writes bfloat16 o: dtype 2 is valid there too
+    # (checked with an empty batch, which enqueues nothing).
+    fake = 1 << 20
+    assert lib.mla_decode_combine(0, 1, 16, 1, 512, 2, fake, 74, 0, fake, fake, fake, 1 << 30, None) == 0
+    assert lib.mla_decode_combine(0, 1, 16, 1, 512, 3, fake, 74, 0, fake, fake, fake, 1 << 30, None) == 1
 
 
 def test_metadata_rejects_bad_arguments(lib):

@@ -5,8 +5,8 @@ same seeded inputs.
   element; they span several pages, ragged page tails, several partitions,
   split and unsplit sequences, 1 to 3 row groups, causal masks that leave rows
   empty, empty sequences and NaN in never-visible cache rows.
-* The five full-size decode workloads run in the launch configuration the
-  benchmark times (default scheduler partitions); sampled rows are compared one
+* The full-size decode workloads (the five configurations and the compute one
+  over an FP8 cache) run in the launch configuration the benchmark times (default scheduler partitions); sampled rows are compared one
   by one with the oracle and every row is checked for finiteness.
 """
 import numpy as np
@@ -15,7 +15,7 @@ import torch
 
 import mla_decode_attention_12_b200 as mla
 from mla_decode_attention_12_b200 import workloads as W
-from tests.gpu_helpers import compare, run_gpu, to_device
+from tests.gpu_helpers import compare, oracle_full, oracle_rows, run_gpu, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -26,11 +26,6 @@ def _cuda():
         pytest.skip("no CUDA device")
     from mla_decode_attention_12_b200 import build
     build.build()
-
-
-def oracle_full(oracle_mod, p):
-    return oracle_mod.decode(p.q, p.kvcache, p.block_table, p.cache_seqlens, dv=p.dv, dtype=p.dtype,
-                             causal=p.causal, scale=p.scale)
 
 
 SMALL = {
@@ -221,8 +216,7 @@ def test_parity_full_size_sampled(oracle_mod, name):
         np.argmax(p.cache_seqlens) * p.s_q * p.h_q + np.arange(min(8, p.s_q * p.h_q)),
         np.argmin(p.cache_seqlens) * p.s_q * p.h_q + np.arange(min(8, p.s_q * p.h_q)),
     ])).astype(np.int64)
-    o_ref, lse_ref = oracle_mod.decode_rows(p.q, p.kvcache, p.block_table, p.cache_seqlens, sample, dv=p.dv,
-                                            dtype=p.dtype, causal=p.causal, scale=p.scale)
+    o_ref, lse_ref = oracle_rows(oracle_mod, p, sample)
     o_s = o.reshape(rows_total, p.dv)[torch.from_numpy(sample).cuda()]
     l_s = lse.reshape(rows_total)[torch.from_numpy(sample).cuda()]
     print(compare(o_s, l_s, o_ref, lse_ref, p.dtype, f"{name} sampled"))
