@@ -42,6 +42,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include <cmath>
 #include <cstdint>
@@ -397,31 +398,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         const uint32_t k_full_lead[2] = {lead_bar(kBarKFull), lead_bar(kBarKFull + 1)};
         const uint32_t v_full_lead = lead_bar(kBarVFull);
         auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
-        // 16 e4m3 values (one 16-byte word) times `s` -> 16 bfloat16 values (two 16-byte words),
-        // with integer and multiply instructions only (conversion instructions issue at a
-        // fraction of their rate).  An e4m3 byte in the top byte of y, shifted right by 4 with
-        // sign extension and masked, leaves its exponent and fraction in bits 20-26 of a float
-        // and its sign in bit 31: that float is the e4m3 value times 2^-120, subnormals
-        // included (the exponent field moves unbiased; both encodings keep subnormals at field
-        // 0).  Multiplying by 2^120 restores the value exactly; multiplying by s rounds the
-        // exact product once to float32, and the pack rounds it to bfloat16 (nearest even).
-        // The multiplies run two values per instruction.
-        // The e4m3 NaN pattern S.1111.111 comes out as +-480, not NaN: the format's quantizer
-        // never writes it.
+        // 16 e4m3 values (one 16-byte word) times `s` -> 16 bfloat16 values (two 16-byte words).
+        // Two values at a time: e4m3 -> half (exact: every e4m3 value, subnormals and NaN
+        // included, is a half), half -> float32 (exact), one packed float32 multiply by s (the
+        // exact product rounded once), then the pack to bfloat16 (round to nearest even).
         auto dequant16 = [](const uint4 raw, const float s, uint4& lo, uint4& hi) {
-            auto bits = [](uint32_t y) {
-                return __int_as_float((static_cast<int32_t>(y) >> 4) & static_cast<int32_t>(0x87F00000u));
-            };
-            // two values per multiply instruction (the packed float32 form, same rounding)
-            auto pack = [s, &bits](uint32_t y0, uint32_t y1) {  // y0 -> low half
-                const float2 v = fmul2(fmul2(make_float2(bits(y0), bits(y1)), make_float2(0x1p120f, 0x1p120f)),
-                                       make_float2(s, s));
-                const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
-                return *reinterpret_cast<const uint32_t*>(&h);
+            auto two = [s](uint32_t w16) {  // byte 0 -> low half of the result
+                const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w16), __NV_E4M3);
+                const float2 v = fmul2(__half22float2(*reinterpret_cast<const __half2*>(&h)), make_float2(s, s));
+                const __nv_bfloat162 b = __floats2bfloat162_rn(v.x, v.y);
+                return *reinterpret_cast<const uint32_t*>(&b);
             };
             auto word = [&](uint32_t w, uint32_t& a, uint32_t& b) {  // bytes 0, 1 -> a; bytes 2, 3 -> b
-                a = pack(w << 24, w << 16);
-                b = pack(w << 8, w);
+                a = two(w & 0xffffu);
+                b = two(w >> 16);
             };
             word(raw.x, lo.x, lo.y);
             word(raw.y, lo.z, lo.w);
@@ -512,21 +502,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 if (!(ok = wwait(bar(kBarRawKFull + rk.stage), rk.phase))) break;
                 if (!(ok = wwait(bar(kBarKEmpty + kring.stage), kring.phase ^ 1))) break;
                 {
-                    // Every load of the page is issued before the first store (the compiler cannot
-                    // move loads above stores into the same shared memory), so the 8 boxes'
-                    // conversions overlap.
                     const uint8_t* rrow = smem + L::kOffRawK + rk.stage * kRawKBytes + lane * kFp8Row;
                     uint8_t* krow = smem + L::kOffK + kring.stage * L::kKBytes + lane * 128;
-                    uint4 raw[4];
-#pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        raw[m] = *reinterpret_cast<const uint4*>(rrow + 64 * (4 * ch + m) + 16 * cq);
                     const uint4 rope = *reinterpret_cast<const uint4*>(rrow + 528 + 16 * cw);
                     const float2 sc = *reinterpret_cast<const float2*>(rrow + 512 + 8 * ch);  // boxes 4 ch .. 4 ch + 3
-#pragma unroll
+                    // Two boxes per iteration: a smaller loop body keeps the instruction cache warm for
+                    // the other warp roles, and the other converter warp of the scheduler hides the
+                    // load latency.
+#pragma unroll 2
                     for (int m = 0; m < 4; ++m) {  // box 4 ch + m: latent columns [64 (4 ch + m), +64); 16 of them
                         uint4 w0, w1;
-                        dequant16(raw[m], m < 2 ? sc.x : sc.y, w0, w1);
+                        dequant16(*reinterpret_cast<const uint4*>(rrow + 64 * (4 * ch + m) + 16 * cq), m < 2 ? sc.x : sc.y,
+                                  w0, w1);
                         uint8_t* box = krow + (4 * ch + m) * 4096;
                         *reinterpret_cast<uint4*>(box + (((2 * cq) ^ sw) << 4)) = w0;
                         *reinterpret_cast<uint4*>(box + (((2 * cq + 1) ^ sw) << 4)) = w1;
