@@ -194,3 +194,35 @@ def test_fp8_decode_rows_matches_decode(oracle_mod):
     ro, rl = oracle_mod.decode_rows_fp8(p.q, p.kvcache, p.block_table, p.cache_seqlens, ids,
                                         scale=p.scale)
     assert np.array_equal(ro, o.reshape(-1, 512)[ids]) and np.array_equal(rl, lse.reshape(-1)[ids])
+
+
+# ---------------------------------------------------------------------------
+# the seeded FP8 cache generator (shared input module): recipe and poisoning
+# ---------------------------------------------------------------------------
+
+
+def test_fp8_generator_recipe():
+    rng = np.random.default_rng(7)
+    rows = W._fp8_rows(rng, 4000)
+    lat = rows[:, :512]
+    assert not np.any((lat & 0x7F) == 0x7F), "no e4m3 NaN codes in drawn rows"
+    sc = rows[:, 512:528].copy().view("<f4")
+    assert np.all((sc >= 2.0 ** -8) & (sc < 2.0 ** -7))
+    vals = torch.from_numpy(np.ascontiguousarray(lat)).view(torch.float8_e4m3fn).float().numpy()
+    deq = np.abs(vals.reshape(-1, 4, 128) * sc[:, :, None])
+    assert deq.max() <= 3.5 and 0.5 < deq.mean() < 1.1
+    rope = torch.from_numpy(rows[:, 528:].copy().view(np.int16)).view(torch.bfloat16).float().numpy()
+    assert abs(rope.std() - 1.0) < 0.05
+
+
+def test_fp8_problem_poison_marks_only_never_visible_rows():
+    p = W.make_problem([100, 64, 1], s_q=1, h_q=8, fp8_kv=True, poison=True, extra_pages=2, seed=9)
+    assert p.kvcache.shape[-1] == 656 and p.kvcache.dtype == np.uint8
+    for b, L in enumerate(p.cache_seqlens):
+        for j in range(int(L)):
+            row = p.kvcache[p.block_table[b, j // 64], j % 64, 0]
+            assert not np.all(row == 0xFF)
+        if L % 64:
+            tail = p.kvcache[p.block_table[b, (L - 1) // 64], L % 64:, 0]
+            assert np.all(tail == 0xFF)
+    assert p.kv_row_bytes() == 656 and p.kv_bytes() == 165 * 656
