@@ -108,3 +108,15 @@ def test_fp8_repeat_calls_are_deterministic():
     o1, l1, _, _ = run_gpu(p)
     o2, l2, _, _ = run_gpu(p)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fp8_host_buffers_end_to_end(oracle_mod):
+    # pinned host tensors through the public call: copied in, decoded, copied back
+    p = fp8([700, 64], s_q=2, h_q=16, causal=True, seed=214)
+    q, kv, bt, sl = (t.cpu().pin_memory() for t in to_device(p))
+    md, ns = mla.get_mla_metadata(sl.cuda(), p.s_q * p.h_q, 1)
+    o, lse = mla.flash_mla_with_kvcache(q, kv, bt, sl, 512, md.cpu(), ns.cpu(), causal=True, softmax_scale=p.scale,
+                                        is_fp8_kvcache=True)
+    assert not o.is_cuda and kv.dtype == torch.uint8
+    o_ref, lse_ref = oracle_full(oracle_mod, p)
+    print(compare(o, lse, o_ref, lse_ref, p.dtype, "fp8 host buffers"))

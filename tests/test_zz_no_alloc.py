@@ -40,7 +40,7 @@ def lib():
 def _device_problem(p):
     dt = torch.bfloat16 if p.dtype == W.BF16 else torch.float16
     q = torch.from_numpy(p.q.view(np.int16)).view(dt).cuda()
-    kv = torch.from_numpy(p.kvcache.view(np.int16)).view(dt).cuda()
+    kv = (torch.from_numpy(p.kvcache) if p.fp8_kv else torch.from_numpy(p.kvcache.view(np.int16)).view(dt)).cuda()
     bt = torch.from_numpy(p.block_table).cuda()
     sl = torch.from_numpy(p.cache_seqlens).cuda()
     md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q, 1)
@@ -49,7 +49,8 @@ def _device_problem(p):
 
 def _args(p, q, kv, bt, sl, md, ns, o, lse):
     return (q.data_ptr(), p.batch, p.s_q, p.h_q, p.d_qk, kv.data_ptr(), p.num_blocks, 64, 1, bt.data_ptr(),
-            bt.shape[1], sl.data_ptr(), 512, p.dtype, md.data_ptr(), md.shape[0], ns.data_ptr(), int(p.causal),
+            bt.shape[1], sl.data_ptr(), 512, 2 if p.fp8_kv else p.dtype, md.data_ptr(), md.shape[0], ns.data_ptr(),
+            int(p.causal),
             p.scale, 0, o.data_ptr(), lse.data_ptr())
 
 
@@ -79,6 +80,7 @@ def test_noalloc_matches_regular_on_two_calls(lib):
     problems = [
         W.make_problem([20000, 7000, 3000, 100], s_q=1, h_q=128, seed=901),
         W.make_problem([2500, 64, 700, 1, 4100], s_q=2, h_q=64, causal=True, seed=902),
+        W.make_problem([20000, 3000, 100], s_q=1, h_q=128, seed=903, fp8_kv=True),  # "FP8 with scale" cache
     ]
     for p in problems:
         t = _device_problem(p)
