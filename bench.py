@@ -84,12 +84,38 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
+def _code_tokens(text: str) -> str:
+    """C / CUDA source without comments, whitespace runs collapsed (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":  # string or character literal, copied with its escapes
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_sha() -> str:
+    """Hash of the CUDA sources' code (comments and whitespace excluded): it changes exactly
+    when the compiled kernels can, so recorded counters stay attached to the code they measured."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_decode_attention_12_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_tokens(f.read()).encode())
     return h.hexdigest()[:16]
 
 

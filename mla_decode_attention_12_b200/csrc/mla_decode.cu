@@ -33,6 +33,10 @@
 //   merges as soon as each virtual batch's splits are announced.
 // * The metadata, split-KV and combine kernels are launched with programmatic launch
 //   overlap.
+// * "FP8 with scale" cache (the kFp8 instantiation, 512 threads): the K producer bulk-copies
+//   this CTA's raw 656-byte rows of each page and the V producer the peer rows' V slices and
+//   scales; two converter warpgroups dequantize them (e4m3 x float32 scale, rounded to
+//   bfloat16) into the same K and V stages, so the MMA, softmax and epilogue are unchanged.
 //
 // Every mbarrier wait is bounded: after kWaitTimeoutNs the waiting thread sets
 // an abort flag (seen by both CTAs of the cluster) and MLA_ERR_TIMEOUT in the
@@ -317,7 +321,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         mbar_init(bar(kBarQFull), 1 + 8);
         mbar_init(bar(kBarQFree), 1);
         // K and V stages are filled by TMA (one arrival with the byte count) or, for the FP8
-        // cache, by the 4 converter warps of each CTA.
+        // cache, by the 8 converter warps of each CTA.
         for (int s = 0; s < L::kKStages; ++s) {
             mbar_init(bar(kBarKFull + s), kFp8 ? 2 * kConvWarps : 1);
             mbar_init(bar(kBarKEmpty + s), 1);
