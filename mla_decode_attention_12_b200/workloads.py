@@ -54,6 +54,7 @@ class Problem:
     active_heads: int | None = None  # heads >= this are zero-filled (padded heads)
     seed: int = 0
     fp8_kv: bool = False     # kvcache holds 656-byte "FP8 with scale" rows (uint8)
+    indices: np.ndarray | None = None  # int32 [b, s_q, topk] flat cache rows (sparse decode), -1 invalid
 
     @property
     def batch(self) -> int:
@@ -224,6 +225,33 @@ def make_problem(
     return Problem(name=name, q=q, kvcache=kv, block_table=table, cache_seqlens=seqlens,
                    dtype=dtype, causal=causal, scale=float(scale), active_heads=active_heads,
                    seed=seed, fp8_kv=fp8_kv)
+
+
+def make_sparse_problem(seqlens, topk: int, *, s_q: int = 1, invalid_frac: float = 0.0, **kw) -> Problem:
+    """A paged-cache problem plus, per query token, `topk` attended rows of its own sequence.
+
+    Each query token's entries are distinct positions of its request's cached tokens drawn
+    uniformly (all of them, in random order, when the sequence is shorter than topk), mapped to
+    flat rows page * 64 + offset through the block table; the remaining slots and a random
+    `invalid_frac` of the drawn ones are -1.  Everything else is as in :func:`make_problem`
+    (causal stays off: the list is what each query sees).
+    """
+    p = make_problem(seqlens, s_q=s_q, **kw)
+    rng = np.random.Generator(np.random.PCG64(p.seed + 7877))
+    idx = np.full((p.batch, s_q, topk), -1, np.int32)
+    for b, L in enumerate(p.cache_seqlens):
+        L = int(L)
+        for s in range(s_q):
+            n = min(L, topk)
+            if n == 0:
+                continue
+            j = rng.choice(L, size=n, replace=False)
+            rows = p.block_table[b, j // PAGE].astype(np.int64) * PAGE + j % PAGE
+            if invalid_frac > 0:
+                rows[rng.random(n) < invalid_frac] = -1
+            idx[b, s, :n] = rows
+    p.indices = idx
+    return p
 
 
 # ----------------------------------------------------------------------------

@@ -26,6 +26,10 @@ Functions and the passages they follow (page title, section):
   the "FlashMLA vLLM Optimization" page): 656-byte token rows of 512
   float8_e4m3 latent values, 4 float32 scales and 64 bfloat16 RoPE values,
   dequantized to bfloat16.
+* :func:`decode_sparse`, :func:`decode_sparse_fp8` -- token-level sparse decoding (the
+  upstream FlashMLA documentation's "Sparse Attention (indices tensor)"): each query
+  token attends the flat cache rows (page * page_size + offset) listed in
+  ``indices[b, s, :topk]``; -1 (or any row past the cache) is an invalid entry.
 * :func:`decode_fp8`, :func:`decode_rows_fp8` -- attention over such a cache:
   the page says the kernel dequantizes the cache to bfloat16 and computes in
   bfloat16, so this is :func:`decode` of the dequantized rows.
@@ -100,6 +104,8 @@ def _load():
             lib.mla_oracle_combine.restype = None
             lib.mla_oracle_half_to_double.argtypes = [ctypes.c_uint16, ctypes.c_int]
             lib.mla_oracle_half_to_double.restype = ctypes.c_double
+            lib.mla_oracle_decode_sparse.argtypes = [ctypes.POINTER(_Shape), P, P, P, ctypes.c_int, P, P]
+            lib.mla_oracle_decode_sparse.restype = ctypes.c_int
             lib.mla_oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
             lib.mla_oracle_e4m3_to_double.restype = ctypes.c_double
             lib.mla_oracle_dequant_fp8_rows.argtypes = [P, ctypes.c_long, P]
@@ -124,7 +130,7 @@ class use_library:
         lib = ctypes.CDLL(self.path)
         for name in ("mla_oracle_decode", "mla_oracle_decode_range", "mla_oracle_decode_rows",
                      "mla_oracle_combine", "mla_oracle_half_to_double", "mla_oracle_num_threads",
-                     "mla_oracle_e4m3_to_double", "mla_oracle_dequant_fp8_rows"):
+                     "mla_oracle_e4m3_to_double", "mla_oracle_dequant_fp8_rows", "mla_oracle_decode_sparse"):
             src = getattr(self._saved, name)
             dst = getattr(lib, name)
             dst.argtypes, dst.restype = src.argtypes, src.restype
@@ -266,3 +272,35 @@ def decode_rows_fp8(q_bits, kv_u8, block_table, seqlens, row_ids, dv=512, causal
     """:func:`decode_rows` over an "FP8 with scale" cache."""
     return decode_rows(q_bits, dequant_fp8(kv_u8), block_table, seqlens, row_ids, dv, BF16, causal,
                        scale, page_size)
+
+
+def decode_sparse(q_bits, kv_bits, indices, dv=512, dtype=BF16, scale=None, page_size=64):
+    """Sparse attention over listed cache rows.  Returns (O [b,s_q,h_q,dv] f64, LSE [b,s_q,h_q] f64).
+
+    ``indices`` [b, s_q, topk] int32 flat row indices (page * page_size + offset); entries
+    outside the cache (-1 included) are invalid.  Each valid entry is one term (repeats count).
+    """
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    kv_bits = np.ascontiguousarray(kv_bits, dtype=np.uint16)
+    indices = np.ascontiguousarray(indices, dtype=np.int32)
+    if q_bits.ndim != 4 or kv_bits.ndim != 4 or indices.ndim != 3:
+        raise ValueError("q [b,s_q,h_q,d_qk], kvcache [blocks,page,h_kv,d_qk], indices [b,s_q,topk]")
+    b, s_q, h_q, d_qk = q_bits.shape
+    nb, ps, h_kv, d2 = kv_bits.shape
+    if d2 != d_qk or ps != page_size or indices.shape[:2] != (b, s_q) or h_q % h_kv:
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d_qk)
+    sh = _Shape(b, s_q, h_q, h_kv, d_qk, dv, page_size, 1, nb, dtype, 0, float(scale))
+    o = np.empty((b, s_q, h_q, dv), np.float64)
+    lse = np.empty((b, s_q, h_q), np.float64)
+    rc = _load().mla_oracle_decode_sparse(ctypes.byref(sh), _ptr(q_bits), _ptr(kv_bits), _ptr(indices),
+                                          int(indices.shape[2]), _ptr(o), _ptr(lse))
+    if rc:
+        raise ValueError("oracle rejected its arguments")
+    return o, lse
+
+
+def decode_sparse_fp8(q_bits, kv_u8, indices, dv=512, scale=None, page_size=64):
+    """:func:`decode_sparse` over an "FP8 with scale" cache (dequantized first)."""
+    return decode_sparse(q_bits, dequant_fp8(kv_u8), indices, dv, BF16, scale, page_size)

@@ -33,6 +33,8 @@
  *     656 bytes (512 float8_e4m3 latent values, 4 float32 scales, one per 128
  *     values, 64 bfloat16 RoPE values), dequantized to bfloat16 before the
  *     attention, which then runs as for a bfloat16 cache.
+ *   - Upstream FlashMLA documentation, "Sparse Attention (indices tensor)": the
+ *     token-level sparse decode over a flat row list per query token.
  *   - Upstream FlashMLA documentation, "Sparse MLA Prefill / Equivalent PyTorch
  *     code": the softmax written out (max, log-sum-exp, weights exp(P - lse)).
  * Readings where the pages are silent (each is listed in the design notes):
@@ -312,6 +314,86 @@ int mla_oracle_decode_rows(const mla_oracle_shape* sh, const uint16_t* q, const 
                 long L = seqlens[b];
                 lse[i] = oracle_one_row(sh, q, kv, block_table, L, b, s, h, 0, L, x, qrow,
                                         o + (size_t)i * sh->dv);
+            }
+        }
+        free(x);
+        free(qrow);
+    }
+    return err ? -1 : 0;
+}
+
+/*
+ * Token-level sparse decoding (upstream FlashMLA documentation, "Sparse Attention
+ * (indices tensor)" under "Usage / MLA Decoding"): request b's query token s attends
+ * the cache rows listed in indices[b][s][0 : topk]; an entry is the flat row index
+ * page * page_size + offset, so no block table is used.  Entries of -1 are invalid;
+ * read here: every entry outside [0, num_blocks * page_size) is invalid (the sparse
+ * prefill section on the same page allows -1 or any index past the end) and
+ * contributes nothing.  Each valid entry contributes one term, so a row listed twice
+ * counts twice: the entries are gathered, as the sparse prefill's equivalent code
+ * gathers kv[indices].  There is no causal mask: the list is what the query sees.
+ *   x_k = scale * <q[b,s,h,:], k_{row_k}>  (valid k),   LSE = log sum_k exp(x_k),
+ *   O   = sum_k exp(x_k - LSE) v_{row_k},  v = the leading dv columns of the row;
+ * with no valid entry, O = 0 and LSE = -inf.
+ * indices: [batch, s_q, topk] int32; o: [batch, s_q, h_q, dv] f64; lse: [batch, s_q, h_q] f64.
+ * Returns 0 on success, -1 on bad arguments.
+ */
+int mla_oracle_decode_sparse(const mla_oracle_shape* sh, const uint16_t* q, const uint16_t* kv,
+                             const int32_t* indices, int topk, double* o, double* lse)
+{
+    if (!sh || sh->batch < 0 || sh->s_q <= 0 || sh->h_q <= 0 || sh->h_kv <= 0 || sh->h_q % sh->h_kv ||
+        sh->dv > sh->d_qk || topk < 0 || sh->page_size <= 0 || sh->num_blocks < 0)
+        return -1;
+    const int d_qk = sh->d_qk, dv = sh->dv;
+    const long n_rows = (long)sh->num_blocks * sh->page_size;
+    const long rows = (long)sh->batch * sh->s_q * sh->h_q;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* x = (double*)malloc(sizeof(double) * (size_t)(topk > 0 ? topk : 1));
+        double* qrow = (double*)malloc(sizeof(double) * (size_t)d_qk);
+        if (!x || !qrow) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (long r = 0; r < rows; ++r) {
+                const int h = (int)(r % sh->h_q);
+                const long bs = r / sh->h_q; /* b * s_q + s */
+                const int g = h / (sh->h_q / sh->h_kv);
+                const int32_t* ix = indices + (size_t)bs * topk;
+                double* o_row = o + (size_t)r * dv;
+                for (int d = 0; d < dv; ++d) o_row[d] = 0.0;
+                const uint16_t* qp = q + (size_t)r * d_qk;
+                for (int d = 0; d < d_qk; ++d) qrow[d] = mla_oracle_half_to_double(qp[d], sh->dtype);
+                double M = -INFINITY;
+                int any = 0;
+                for (int k = 0; k < topk; ++k) {
+                    const long row = ix[k];
+                    if (row < 0 || row >= n_rows) continue; /* invalid entry */
+                    const uint16_t* kp = kv + ((size_t)row * sh->h_kv + g) * (size_t)d_qk;
+                    double acc = 0.0;
+                    for (int d = 0; d < d_qk; ++d) acc += qrow[d] * mla_oracle_half_to_double(kp[d], sh->dtype);
+                    x[k] = sh->scale * acc;
+                    if (!any || x[k] > M) M = x[k];
+                    any = 1;
+                }
+                if (!any) {
+                    lse[r] = -INFINITY;
+                    continue;
+                }
+                double sum = 0.0;
+                for (int k = 0; k < topk; ++k)
+                    if (ix[k] >= 0 && ix[k] < n_rows) sum += exp(x[k] - M);
+                const double L = M + log(sum);
+                lse[r] = L;
+                for (int k = 0; k < topk; ++k) {
+                    const long row = ix[k];
+                    if (row < 0 || row >= n_rows) continue;
+                    const uint16_t* vp = kv + ((size_t)row * sh->h_kv + g) * (size_t)d_qk;
+                    const double w = exp(x[k] - L);
+                    for (int d = 0; d < dv; ++d) o_row[d] += w * mla_oracle_half_to_double(vp[d], sh->dtype);
+                }
             }
         }
         free(x);

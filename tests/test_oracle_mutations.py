@@ -4,8 +4,9 @@ Each case compiles a copy of the oracle source with one planted mistake (on the
 CPU, in a temporary directory) and runs the pin tests against it: at least one
 pin must fail.  This shows the pins constrain every term of the definition
 (scale, V columns, causal offset, kv-head mapping, page indexing, LSE base, the
-combine weights, and the FP8 cache's scale blocks, e4m3 exponent bias and
-subnormals, RoPE offset and bfloat16 rounding).
+combine weights, the FP8 cache's scale blocks, e4m3 exponent bias and
+subnormals, RoPE offset and bfloat16 rounding, and the sparse decode's scale, LSE
+and V columns).
 """
 import os
 import subprocess
@@ -15,6 +16,7 @@ import pytest
 
 import oracle
 import tests.test_oracle_fp8_pins as fp8_pins
+import tests.test_oracle_sparse_pins as sparse_pins
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "mla_oracle.c")
@@ -36,6 +38,11 @@ MUTATIONS = {
     "fp8_rope_offset": ("row + 528 + 2 * i", "row + 526 + 2 * i"),
     "bf16_truncation": ("if (rest > 0x8000u || (rest == 0x8000u && (hi & 1u))) hi += 1;", ""),
     "bf16_ties_away": ("(rest == 0x8000u && (hi & 1u))", "(rest == 0x8000u)"),
+    # token-level sparse decoding
+    "sparse_dropped_scale": ("x[k] = sh->scale * acc;", "x[k] = acc;"),
+    "sparse_lse_without_sum": ("const double L = M + log(sum);", "const double L = M;"),
+    "sparse_v_wrong_columns": ("o_row[d] += w * mla_oracle_half_to_double(vp[d], sh->dtype);\n                }\n            }\n        }",
+                               "o_row[d] += w * mla_oracle_half_to_double(vp[d + d_qk - dv], sh->dtype);\n                }\n            }\n        }"),
 }
 
 
@@ -59,6 +66,11 @@ def _pin_calls():
     for args in [(0x3A, 0.828125, 0x3F84), (0x3D, 1.2109375, 0x3FFC), (0x3C, 1.0078125, 0x3FC2)]:
         calls.append((f"fp8_rounding:{args}",
                       lambda a=args: fp8_pins.test_dequant_rounds_to_nearest_even(oracle, *a)))
+    for kw in sparse_pins.SPARSE_CASES:
+        calls.append((f"sparse_brute:{kw['seqlens']}",
+                      lambda k=kw: sparse_pins.test_sparse_brute_force_torch(oracle, k)))
+    for name in ("test_one_row_listed_n_times", "test_full_token_list_equals_dense_decode"):
+        calls.append((name, lambda f=getattr(sparse_pins, name): f(oracle)))
     for kw in fp8_pins.FP8_BRUTE_CASES:
         calls.append((f"fp8_brute:{kw['seqlens']}",
                       lambda k=kw: fp8_pins.test_fp8_decode_brute_force_torch(oracle, k)))
