@@ -109,3 +109,32 @@ def test_host_metadata_rejects_negative_lengths(lib):
     md = np.zeros(74 * 8, np.int32)
     ns = np.zeros(3, np.int32)
     assert lib.mla_get_metadata_host(sl.ctypes.data, 2, 16, 1, 74, md.ctypes.data, ns.ctypes.data) == 1
+
+
+@pytest.mark.parametrize("case", ["fp16_q", "bf16_cache", "row_bytes", "d_qk_512", "mixed_16bit"])
+def test_binding_rejects_mismatched_cache_formats(case):
+    # The Python binding checks dtypes and row widths before it touches the library or a GPU.
+    import torch
+
+    from mla_decode_attention_12_b200 import api
+
+    q = torch.zeros(1, 1, 16, 576, dtype=torch.bfloat16)
+    kv = torch.zeros(2, 64, 1, 656, dtype=torch.uint8)
+    fp8 = True
+    if case == "fp16_q":
+        q = q.half()
+    elif case == "bf16_cache":
+        kv = torch.zeros(2, 64, 1, 576, dtype=torch.bfloat16)
+    elif case == "row_bytes":
+        kv = torch.zeros(2, 64, 1, 576, dtype=torch.uint8)
+    elif case == "d_qk_512":
+        q = torch.zeros(1, 1, 16, 512, dtype=torch.bfloat16)
+    else:  # a 16-bit call whose cache has another dtype
+        kv = torch.zeros(2, 64, 1, 576, dtype=torch.float16)
+        fp8 = False
+    bt = torch.zeros(1, 2, dtype=torch.int32)
+    sl = torch.ones(1, dtype=torch.int32)
+    md = torch.zeros(74, 8, dtype=torch.int32)
+    ns = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        api.DecodeCall(q, kv, bt, sl, 512, md, ns, is_fp8_kvcache=fp8)
