@@ -361,6 +361,8 @@ def workload_line(p, t, peaks, src):
     out = {
         "us_per_call": round(step_ms * 1e3, 2),
         "us_per_call_median": round(float(np.median(t[:, 0])) * 1e3, 2),
+        "us_per_call_p10": round(float(np.percentile(t[:, 0], 10)) * 1e3, 2),
+        "us_per_call_p90": round(float(np.percentile(t[:, 0], 90)) * 1e3, 2),
         "us_splitkv": round(sk_ms * 1e3, 2),
         "us_combine": round(float(t[:, 3].mean()) * 1e3, 2),
         "us_metadata": round(float(t[:, 1].mean()) * 1e3, 2),
