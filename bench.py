@@ -521,6 +521,8 @@ def run_ours(args):
                        "l2": "flushed between steps (write of 2 x L2 outside the timed events)",
                        "parallelism": f"{world} independent replica(s), no collective"},
             "us_per_call": main["us_per_call"],
+            "us_per_call_p10_median_p90": [main["us_per_call_p10"], main["us_per_call_median"],
+                                           main["us_per_call_p90"]],
             "kv_gbs": main["kv_gbs"],
             "tflops": main["tflops"],
             "breakdown_us": {"metadata": main["us_metadata"], "splitkv": main["us_splitkv"],
