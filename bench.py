@@ -5,12 +5,14 @@ One step = one pass of the whole decode path on one batch of synthetic input:
 the tile scheduler (metadata kernel), the split-KV kernel and the combine
 kernel.  The headline workload is the compute-bound decode (batch 64, s_q 1,
 h_q 128, d_qk 576, d_v 512, cache lengths uniform in [1024, 8192], 64-token
-pages, shuffled block table, bf16 N(0,1), scale 1/sqrt(576)).  The other four
-decode workloads are timed in the same run and reported under "workloads".
+pages, shuffled block table, bf16 N(0,1), scale 1/sqrt(576)).  The other decode
+workloads (the four other configurations, and the compute one over an FP8-with-scale
+cache) are timed in the same run and reported under "workloads".
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronisation; each step replays one captured CUDA graph holding the
-three kernels with timing events between them (on the launching stream); L2
+three kernels with timing events around them (on the launching stream; a second
+graph with events between the kernels gives each kernel's own time); L2
 is flushed between steps (a write of 2 x L2), outside the events.  For N > 1 GPUs each rank runs an independent replica
 (the path needs no collective) and rank 0 reports the maximum step time over
 ranks.
