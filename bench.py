@@ -378,6 +378,14 @@ def workload_line(p, t, peaks, src):
     return out
 
 
+def workload_config(p: W.Problem, world: int) -> dict:
+    """The ``config`` object of a JSON line: the same keys and values in both arms for one workload."""
+    return {"workload": DESCR[p.name], "batch": p.batch, "s_q": p.s_q, "h_q": p.h_q, "h_kv": 1,
+            "d_qk": p.d_qk, "d_v": p.dv, "page_size": 64, "causal": p.causal,
+            "l2": "flushed between steps (write of 2 x L2 outside the timed events)",
+            "parallelism": f"{world} independent replica(s), no collective"}
+
+
 def oracle_rows(oracle, p: W.Problem, ids):
     """The oracle on flat query rows `ids` (an FP8 cache is dequantized by the oracle itself)."""
     if p.fp8_kv:
@@ -518,10 +526,7 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "bf16" if p.dtype == W.BF16 else "fp16",
             "data": "synthetic (seeded, shapes and distributions of the workload)",
-            "config": {"workload": DESCR[p.name], "batch": p.batch, "s_q": p.s_q, "h_q": p.h_q, "h_kv": 1,
-                       "d_qk": p.d_qk, "d_v": p.dv, "page_size": 64, "causal": p.causal,
-                       "l2": "flushed between steps (write of 2 x L2 outside the timed events)",
-                       "parallelism": f"{world} independent replica(s), no collective"},
+            "config": workload_config(p, world),
             "us_per_call": main["us_per_call"],
             "us_per_call_p10_median_p90": [main["us_per_call_p10"], main["us_per_call_median"],
                                            main["us_per_call_p90"]],
@@ -585,8 +590,9 @@ def run_reference(args):
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
-        "config": {"workload": DESCR[p.name], "batch": p.batch, "s_q": p.s_q, "h_q": p.h_q, "d_qk": p.d_qk,
-                   "d_v": p.dv, "page_size": 64, "causal": p.causal},
+        # the GPU arm's config object for the same workload and N (the oracle has no L2 flush
+        # of its own to state; the keys stay identical so the two lines compare directly)
+        "config": workload_config(p, int(os.environ.get("WORLD_SIZE", str(args.gpus)))),
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -16,7 +16,8 @@
  *   - Pointers named "device" are CUDA device pointers; "host" ones are host memory.
  *   - The caller allocates and owns every buffer.  The library allocates no
  *     memory and keeps no state between calls (apart from a per-process cache
- *     of one CUDA driver entry point).
+ *     of one CUDA driver entry point and per-device kernel attributes set on
+ *     first use).
  *   - Calls taking a stream enqueue work on it and return without
  *     synchronising; results are ready when the stream reaches that point.
  *     A stream of NULL means the legacy default stream.
@@ -130,16 +131,22 @@ MLA_API mla_status mla_get_metadata_host(const int32_t* cache_seqlens, int batch
                                  int h_kv, int num_parts, int32_t* tile_md, int32_t* num_splits);
 
 /*
- * Bytes of device workspace mla_decode_with_kvcache needs: a control block
- * (the status word and two int32 counters per (request, row group)), then
- * float32 partial outputs and LSEs for up to batch * row_groups + num_parts
- * splits of 128 rows each.  Returns 0 for invalid sizes.
+ * Bytes of device workspace mla_decode_with_kvcache needs: a control block of
+ * fixed size (the status word and two int32 counters for each of up to
+ * MLA_MAX_VIRTUAL_BATCHES (request, row group) pairs), then float32 partial
+ * outputs and LSEs for up to batch * row_groups + num_parts splits of 128 rows
+ * each.  Returns 0 for invalid sizes, and for batch * row_groups above
+ * MLA_MAX_VIRTUAL_BATCHES.
  *
- * The first mla_decode_workspace_zero_bytes(...) bytes (the control block) must
- * be zero before a workspace is first used; every call that completes without
- * a device error leaves them zero again.  After a device error (see
- * mla_read_device_status) zero them before reusing the workspace.
+ * mla_decode_workspace_zero_bytes returns the size of the control block (the
+ * same for every problem).  It must be zero before a workspace is first used;
+ * every call that completes without a device error leaves it zero again, for
+ * every later call of any size: the control block does not depend on the
+ * problem, so the partial results of one call never land on the counters of
+ * another.  After a device error (see mla_read_device_status, whose clear flag
+ * zeroes the whole control block) zero it before reusing the workspace.
  */
+#define MLA_MAX_VIRTUAL_BATCHES 16384
 MLA_API size_t mla_decode_workspace_bytes(int batch, int s_q, int h_q, int h_kv, int num_parts);
 MLA_API size_t mla_decode_workspace_zero_bytes(int batch, int s_q, int h_q, int h_kv);
 
@@ -221,7 +228,10 @@ MLA_API mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int
 /*
  * Reads the device status word of a workspace (synchronises `stream`).
  * *device_status receives MLA_OK or the first device-side error recorded by a
- * decode call that used this workspace; clear != 0 resets it to MLA_OK.
+ * decode call that used this workspace; clear != 0 then zeroes the workspace's
+ * whole control block (the status word back to MLA_OK, and the split / combine
+ * counters a call that met a device error may have left nonzero), so the
+ * workspace can be used again.
  */
 MLA_API mla_status mla_read_device_status(void* workspace, int clear, int* device_status, void* stream);
 
@@ -244,9 +254,10 @@ MLA_API mla_status mla_read_device_status(void* workspace, int clear, int* devic
  *   - The first call on a device looks up the device address of the scratch
  *     array (once per device, with that device current); make that first call
  *     before capturing any stream on that device.
- *   - No memory is allocated or freed; each call clears the scratch status word
- *     with an asynchronous memset on `stream` and then enqueues the same kernels
- *     as mla_decode_with_kvcache.
+ *   - No memory is allocated or freed; each call clears the scratch's status
+ *     word and its own split / combine counters with an asynchronous memset on
+ *     `stream` and then enqueues the same kernels as mla_decode_with_kvcache.
+ *     Device-side errors of a call are read with mla_read_noalloc_status.
  *   - All calls on a device share one scratch array, which keeps the last
  *     call's contents: calls whose execution overlaps on the GPU (different
  *     streams without ordering between them) race on it and give wrong results.
@@ -261,6 +272,17 @@ MLA_API mla_status mla_decode_with_kvcache_noalloc(const void* q, int batch, int
                                                    int num_parts, const int32_t* num_splits, int causal,
                                                    float softmax_scale, int active_heads, void* o, float* lse,
                                                    void* stream);
+
+/*
+ * Device status of the allocation-free entry point's scratch on the current
+ * device (synchronises `stream`): MLA_OK, or the device-side error
+ * (MLA_ERR_DEVICE_CHECK, MLA_ERR_TIMEOUT) recorded by the last
+ * mla_decode_with_kvcache_noalloc call on this device, whose o / lse are then
+ * not to be trusted.  Read it after a call and before the next one: every
+ * call clears it when it starts.  clear != 0 resets it to MLA_OK.  Errors:
+ * MLA_ERR_INVALID_ARG (null), MLA_ERR_CUDA.
+ */
+MLA_API mla_status mla_read_noalloc_status(int clear, int* device_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -46,6 +46,7 @@ SIGNATURES = {
     "mla_read_device_status": ([_P, _I, ctypes.POINTER(_I), _P], _I),
     "mla_decode_with_kvcache_noalloc": ([_P, _I, _I, _I, _I, _P, _I, _I, _I, _P, _I, _P, _I, _I,
                                          _P, _I, _P, _I, _F, _I, _P, _P, _P], _I),
+    "mla_read_noalloc_status": ([_I, ctypes.POINTER(_I), _P], _I),
 }
 
 _lock = threading.Lock()

@@ -103,20 +103,20 @@ def workspace_zero_bytes(batch: int, s_q: int, h_q: int, h_kv: int) -> int:
     return _lib.load().mla_decode_workspace_zero_bytes(batch, s_q, h_q, h_kv)
 
 
-def get_workspace(nbytes: int, device: torch.device, zero_bytes: int = 256) -> torch.Tensor:
-    """A cached, grow-only workspace per (device, stream) whose first ``zero_bytes`` are zero.
+def get_workspace(nbytes: int, device: torch.device, zero_bytes: int) -> torch.Tensor:
+    """A cached, grow-only workspace per (device, stream) whose control block is zero.
 
-    Calls leave the control block zero; it is cleared again only when a call needs a
-    larger one than any before (its counters then reach into bytes used for other data).
+    ``zero_bytes`` is the control block's size (the same for every problem): it is
+    zeroed when the workspace is allocated, and every call that meets no device error
+    leaves it zero for the next call of any size.  ``read_device_status(ws, clear=True)``
+    zeroes it again after a device error.
     """
     key = (device.index, _stream(device))
-    ws, zeroed = _workspaces.get(key, (None, 0))
-    if ws is None or ws.numel() < nbytes:
-        ws, zeroed = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device), 0
-    if zeroed < zero_bytes:
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < max(nbytes, zero_bytes):
+        ws = torch.empty(max(nbytes, zero_bytes), dtype=torch.uint8, device=device)
         ws[:zero_bytes].zero_()
-        zeroed = zero_bytes
-    _workspaces[key] = (ws, zeroed)
+        _workspaces[key] = ws
     return ws
 
 
@@ -222,7 +222,10 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
 
 
 def read_device_status(workspace: torch.Tensor, clear: bool = True) -> int:
-    """Device-side status recorded in a workspace (synchronises the current stream)."""
+    """Device-side status recorded in a workspace (synchronises the current stream).
+
+    ``clear`` zeroes the workspace's whole control block afterwards (status word and the
+    split / combine counters), so that it can be used again after a device error."""
     v = ctypes.c_int(0)
     dev = workspace.device
     with torch.cuda.device(dev):

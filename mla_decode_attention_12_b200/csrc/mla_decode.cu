@@ -51,6 +51,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -93,6 +94,12 @@ constexpr int kQTmemBoxes = 6;         // 64-column boxes of Q kept in tensor me
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 constexpr int kWorkspaceHeader = 256;
+// The workspace's control block has room for the counters of this many virtual batches
+// (requests x row groups of 128 query rows), whatever the call: its size does not depend on
+// the problem, so the split partials of one call never overlap the counters of another.
+constexpr int kMaxVirtualBatches = MLA_MAX_VIRTUAL_BATCHES;
+constexpr size_t kControlBytes = kWorkspaceHeader + 2 * sizeof(int32_t) * kMaxVirtualBatches;
+static_assert(kControlBytes % 256 == 0, "split partials start 256-byte aligned");
 constexpr int kNumMaps = 7;  // tensor maps of the split-KV kernel: Q, K, V, O, split partials, and O and
                              // split partials with 8-row boxes
 
@@ -189,8 +196,8 @@ struct DecodeParams {
     float* o_accum;     // [slots, 128, 512]
     float* lse_accum;   // [slots, 128]
     int* status;
-    int* split_done;      // [NV]: split-KV warps that announced their partials (8 per split)
-    int* combine_passed;  // [NV]: combine CTAs past their wait
+    int* ctl;  // [kMaxVirtualBatches][2] per virtual batch: split-KV warps that announced their
+               // partials (8 per split), combine CTAs past their wait
     int batch, s_q, h_q, rows, groups, max_blocks, num_blocks, causal, box_rows;
     int active_heads;  // heads >= active_heads are padding: not written, not combined
     float scale_log2;
@@ -887,7 +894,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     bulk_wait_all();             // this warp's tile stores of that split are complete
                     fence_proxy_async_global();  // ... and ordered before the counter update
                     __threadfence();             // (with the LSE stores of the warp)
-                    atomicAdd(p.split_done + announce_vb, 1);
+                    atomicAdd(p.ctl + 2 * announce_vb, 1);
                 }
                 __syncwarp();
                 announce_vb = -1;
@@ -1218,19 +1225,21 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
     __shared__ int go;
     if (threadIdx.x == 0) {
         const int want = 8 * nsplit;
-        bool ready = ld_acquire_gpu(p.split_done + vb) >= want;
+        int* split_done = p.ctl + 2 * vb;
+        int* combine_passed = split_done + 1;
+        bool ready = ld_acquire_gpu(split_done) >= want;
         const uint64_t t0 = global_timer_ns();
         while (!ready) {
             __nanosleep(200);
-            ready = ld_acquire_gpu(p.split_done + vb) >= want;
+            ready = ld_acquire_gpu(split_done) >= want;
             if (!ready && global_timer_ns() - t0 > kWaitTimeoutNs) {
                 atomicCAS(p.status, 0, MLA_ERR_TIMEOUT);
                 break;
             }
         }
-        if (ready && atomicAdd(p.combine_passed + vb, 1) == static_cast<int>(gridDim.y) - 1) {
-            p.combine_passed[vb] = 0;
-            p.split_done[vb] = 0;
+        if (ready && atomicAdd(combine_passed, 1) == static_cast<int>(gridDim.y) - 1) {
+            *combine_passed = 0;
+            *split_done = 0;
         }
         go = ready;
     }
@@ -1479,46 +1488,64 @@ static size_t workspace_slots(int batch, int groups, int num_parts)
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace layout: a control block (the status word, then two int32 counters per virtual
-// batch: split partials announced, combine CTAs past their wait), which must be zero before
-// the first call and is left zero by every call that completes without a device error; then
-// the split LSEs and the split partial outputs.
-static size_t control_bytes(size_t nv) { return align_up(kWorkspaceHeader + 2 * nv * sizeof(int32_t), 256); }
-
+// Workspace layout: a control block of fixed size (the status word, then two int32 counters
+// per virtual batch: split partials announced, combine CTAs past their wait), which must be
+// zero before the first call and is left zero by every call that completes without a device
+// error; then the split LSEs and the split partial outputs.  The control block's size does
+// not depend on the problem, so calls of different sizes can share one workspace.
 static void workspace_pointers(void* workspace, int batch, int groups, int num_parts, DecodeParams& prm)
 {
-    const size_t nv = static_cast<size_t>(batch) * groups;
     const size_t slots = workspace_slots(batch, groups, num_parts);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     prm.status = reinterpret_cast<int*>(ws);
-    prm.split_done = reinterpret_cast<int*>(ws + kWorkspaceHeader);
-    prm.combine_passed = prm.split_done + nv;
-    prm.lse_accum = reinterpret_cast<float*>(ws + control_bytes(nv));
-    prm.o_accum = reinterpret_cast<float*>(ws + control_bytes(nv) + align_up(slots * kRowsPerGroup * sizeof(float), 256));
+    prm.ctl = reinterpret_cast<int*>(ws + kWorkspaceHeader);
+    prm.lse_accum = reinterpret_cast<float*>(ws + kControlBytes);
+    prm.o_accum = reinterpret_cast<float*>(ws + kControlBytes + align_up(slots * kRowsPerGroup * sizeof(float), 256));
 }
+
+// Runs a per-device set-up step (a kernel attribute) once for each device it is used on,
+// from any number of host threads.
+struct PerDeviceOnce {
+    static constexpr int kMaxDevices = 64;
+    std::mutex m;
+    std::atomic<bool> done[kMaxDevices] = {};
+
+    template <typename F>
+    cudaError_t run(F&& setup)
+    {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMaxDevices) return setup();  // outside the table: every call
+        if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        std::lock_guard<std::mutex> lock(m);
+        if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+        e = setup();
+        if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+        return e;
+    }
+};
 
 template <bool kRope, bool kFp16, bool kPadHeads, bool kFp8>
 static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorMap* maps, const DecodeParams& prm)
 {
     auto kern = mla_splitkv_kernel<kRope, kFp16, kPadHeads, kFp8>;
     const int smem = Layout<kRope, kFp8>::kSmemBytes;
-    static int configured_device = -1;  // the attribute is per device; set it once per device in use
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (configured_device != dev) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
+    static PerDeviceOnce configured;  // the attribute is per device
+    cudaError_t e = configured.run([&]() -> cudaError_t {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (r != cudaSuccess) return r;
         if (kFp8) {
             // The warpgroups' register re-balancing hands out exactly what the launch holds
-            // (168 per thread); with fewer at launch, setmaxnreg.inc would never return.
+            // (128 per thread); with fewer at launch, setmaxnreg.inc would never return.
             cudaFuncAttributes fa;
-            e = cudaFuncGetAttributes(&fa, kern);
-            if (e != cudaSuccess) return e;
+            r = cudaFuncGetAttributes(&fa, kern);
+            if (r != cudaSuccess) return r;
             if (fa.numRegs < static_cast<int>(kRegsLaunchFp8)) return cudaErrorInvalidConfiguration;
         }
-        configured_device = dev;
-    }
+        return cudaSuccess;
+    });
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     programmatic_launch(cfg, attr, dim3(grid), dim3(kFp8 ? kThreadsFp8 : kThreads), smem, stream);
@@ -1603,15 +1630,12 @@ mla_status mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_p
     const size_t smem = metadata_smem_bytes(nv, num_parts);
     if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;  // the schedule is built in one CTA's shared memory
     if (smem > 48 * 1024) {
-        static int configured_device = -1;
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-        if (configured_device != dev) {
-            if (cudaFuncSetAttribute(mla_metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
-                cudaSuccess)
-                return MLA_ERR_CUDA;
-            configured_device = dev;
-        }
+        static PerDeviceOnce configured;
+        if (configured.run([] {
+                return cudaFuncSetAttribute(mla_metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            200 * 1024);
+            }) != cudaSuccess)
+            return MLA_ERR_CUDA;
     }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -1624,15 +1648,16 @@ mla_status mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_p
 size_t mla_decode_workspace_zero_bytes(int batch, int s_q, int h_q, int h_kv)
 {
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || h_q % h_kv) return 0;
-    return control_bytes(static_cast<size_t>(batch) * row_groups(s_q * h_q / h_kv));
+    return kControlBytes;
 }
 
 size_t mla_decode_workspace_bytes(int batch, int s_q, int h_q, int h_kv, int num_parts)
 {
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_parts <= 0 || h_q % h_kv) return 0;
     const int groups = row_groups(s_q * h_q / h_kv);
+    if (static_cast<long long>(batch) * groups > kMaxVirtualBatches) return 0;
     const size_t slots = workspace_slots(batch, groups, num_parts);
-    size_t bytes = control_bytes(static_cast<size_t>(batch) * groups);
+    size_t bytes = kControlBytes;
     bytes += align_up(slots * kRowsPerGroup * sizeof(float), 256);
     bytes += slots * kRowsPerGroup * kDv * sizeof(float);
     return bytes;
@@ -1660,6 +1685,7 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
         return MLA_ERR_INVALID_ARG;
     const int rows = s_q * h_q;
     const int groups = row_groups(rows);
+    if (static_cast<long long>(batch) * groups > kMaxVirtualBatches) return MLA_ERR_UNSUPPORTED;
     const size_t need = mla_decode_workspace_bytes(batch, s_q, h_q, h_kv, num_parts);
     if (batch > 0 && workspace_bytes < need) return MLA_ERR_WORKSPACE;
     if (static_cast<long long>(num_blocks) * kPage >= (1ll << 31)) return MLA_ERR_UNSUPPORTED;
@@ -1807,6 +1833,7 @@ mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_parts <= 0) return MLA_ERR_INVALID_ARG;
     if (dtype != MLA_BF16 && dtype != MLA_FP16 && dtype != MLA_BF16_FP8KV) return MLA_ERR_INVALID_ARG;
     if (h_kv != 1 || dv != kDv) return MLA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(batch) * row_groups(s_q * h_q) > kMaxVirtualBatches) return MLA_ERR_UNSUPPORTED;
     if (batch == 0) return MLA_OK;
     if (!num_splits || !o || !lse || !workspace) return MLA_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return MLA_ERR_INVALID_ARG;
@@ -1837,7 +1864,8 @@ mla_status mla_read_device_status(void* workspace, int clear, int* device_status
         cudaStreamSynchronize(st) != cudaSuccess)
         return MLA_ERR_CUDA;
     *device_status = v;
-    if (clear && cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return MLA_ERR_CUDA;
+    // the whole control block: after a device error its counters may be left nonzero too
+    if (clear && cudaMemsetAsync(workspace, 0, kControlBytes, st) != cudaSuccess) return MLA_ERR_CUDA;
     return MLA_OK;
 }
 
@@ -1893,14 +1921,24 @@ extern "C" mla_status mla_decode_with_kvcache_noalloc(const void* q, int batch, 
     void* scratch = nullptr;
     mla_status st = noalloc_scratch(&scratch);
     if (st != MLA_OK) return st;
-    // The control block (status word and split / combine counters) must start at zero;
-    // the split partials are always written before they are read, so the rest of the
-    // scratch needs no clearing.
+    // The status word and this call's split / combine counters must start at zero (a call
+    // that met a device error may have left them nonzero); the split partials are always
+    // written before they are read, so the rest of the scratch needs no clearing.
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(scratch, 0, mla_decode_workspace_zero_bytes(batch, s_q, h_q, h_kv), cs) != cudaSuccess)
+    const size_t nv = static_cast<size_t>(batch) * row_groups(s_q * h_q / h_kv);
+    if (cudaMemsetAsync(scratch, 0, kWorkspaceHeader + 2 * sizeof(int32_t) * nv, cs) != cudaSuccess)
         return MLA_ERR_CUDA;
     return mla_decode_with_kvcache(q, batch, s_q, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, block_table,
                                    max_blocks_per_seq, cache_seqlens, dv, dtype, tile_md, num_parts, num_splits,
                                    causal, softmax_scale, active_heads, o, lse, scratch, MLA_NOALLOC_SCRATCH_BYTES,
                                    stream);
+}
+
+extern "C" mla_status mla_read_noalloc_status(int clear, int* device_status, void* stream)
+{
+    if (!device_status) return MLA_ERR_INVALID_ARG;
+    void* scratch = nullptr;
+    mla_status st = noalloc_scratch(&scratch);
+    if (st != MLA_OK) return st;
+    return mla_read_device_status(scratch, clear, device_status, stream);
 }

@@ -48,14 +48,21 @@ def test_sizes(lib):
     assert lib.mla_metadata_sizes(32, 256, 1, 74, ctypes.byref(a), ctypes.byref(b)) == 0
     assert b.value == 32 * 2 + 1
     assert lib.mla_metadata_sizes(-1, 128, 1, 74, ctypes.byref(a), ctypes.byref(b)) == 1
-    # workspace: control block (status word + 2 int32 counters per virtual batch, 256-byte
-    # aligned), then (NV + parts) * 128 * (1 + 512) floats
+    # workspace: a control block of fixed size (status word + 2 int32 counters for each of
+    # up to 16384 virtual batches), then (NV + parts) * 128 * (1 + 512) floats
     nv, parts = 64, 74
-    control = (256 + 2 * nv * 4 + 255) // 256 * 256
+    control = 256 + 2 * 4 * 16384
     want = control + ((nv + parts) * 128 * 4 + 255) // 256 * 256 + (nv + parts) * 128 * 512 * 4
     assert lib.mla_decode_workspace_bytes(64, 1, 128, 1, 74) == want
-    assert lib.mla_decode_workspace_zero_bytes(64, 1, 128, 1) == control == 768
+    # the same control block for every problem size, so calls of different sizes can share
+    # one workspace without one call's partials landing on another's counters
+    for sizes in ((64, 1, 128, 1), (4, 1, 128, 1), (1, 1, 16, 1), (8192, 2, 128, 1)):
+        assert lib.mla_decode_workspace_zero_bytes(*sizes) == control
     assert lib.mla_decode_workspace_bytes(64, 0, 128, 1, 74) == 0
+    # more virtual batches (requests x row groups of 128 query rows) than the control block holds
+    assert lib.mla_decode_workspace_bytes(16384, 1, 128, 1, 74) > 0
+    assert lib.mla_decode_workspace_bytes(16385, 1, 128, 1, 74) == 0
+    assert lib.mla_decode_workspace_bytes(8193, 2, 128, 1, 74) == 0
 
 
 def _decode(lib, **over):
@@ -73,7 +80,7 @@ def _decode(lib, **over):
     (dict(batch=-1), 1), (dict(s_q=0), 1), (dict(h_q=0), 1), (dict(num_blocks=0), 1),
     (dict(causal=2), 1), (dict(dtype=7), 1), (dict(q=(1 << 20) + 2), 1), (dict(ws=(1 << 20) + 16), 1),
     (dict(page_size=32), 2), (dict(h_kv=2), 2), (dict(d_qk=192), 2), (dict(dv=256), 2),
-    (dict(ws_bytes=1000), 3),
+    (dict(ws_bytes=1000), 3), (dict(batch=16385, h_q=128), 2),
     # the "FP8 with scale" cache (dtype 2) carries 64 RoPE values: d_qk must be 576
     (dict(dtype=2, d_qk=512), 2), (dict(dtype=2, kvcache=(1 << 20) + 8), 1), (dict(dtype=3), 1),
 ])
@@ -92,6 +99,11 @@ def test_combine_accepts_the_fp8_cache_dtype(lib):
     fake = 1 << 20
     assert lib.mla_decode_combine(0, 1, 16, 1, 512, 2, fake, 74, 0, fake, fake, fake, 1 << 30, None) == 0
     assert lib.mla_decode_combine(0, 1, 16, 1, 512, 3, fake, 74, 0, fake, fake, fake, 1 << 30, None) == 1
+
+
+def test_status_reads_reject_null_outputs(lib):
+    assert lib.mla_read_noalloc_status(0, None, None) == 1
+    assert lib.mla_read_device_status(None, 0, None, None) == 1
 
 
 def test_metadata_rejects_bad_arguments(lib):

@@ -41,3 +41,19 @@ def test_code_hash_ignores_comments_only():
     assert b._code_tokens(code) == b._code_tokens(code.replace("// one", "// changed").replace("two", "2"))
     assert b._code_tokens(code) != b._code_tokens(code.replace("a + 1", "a + 2"))
     assert b._code_tokens(code) != b._code_tokens(code.replace('"x // y"', '"x // z"'))
+
+
+def test_reference_arm_prints_the_gpu_arms_config(capsys, monkeypatch):
+    # The two arms of one workload carry identical config objects, so their lines compare
+    # directly.  The reference arm runs the oracle on a tiny bounded sample here.
+    import json
+    import sys
+
+    b = _bench()
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", "tiny", "--steps", "1",
+                                      "--warmup", "0"])
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    b.main()
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == b.workload_config(W.make_workload("tiny"), 1)

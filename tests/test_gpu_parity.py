@@ -148,6 +148,25 @@ def test_cached_workspace_across_growing_problems():
         assert int(ws[:zb].count_nonzero().item()) == 0, "a call must leave the control block zero"
 
 
+def test_cached_workspace_shrinking_then_growing(oracle_mod):
+    # One cached workspace (the API's default) for a large split batch, then a small split
+    # batch, then the large batch twice: the small call's split partials must not land on
+    # the counters the large call uses, so every call matches the oracle.
+    large = W.make_problem([5000, 300, 2200, 64, 4100, 900, 3000, 1500, 7000, 20], s_q=1, h_q=128, seed=165)
+    small = W.make_problem([20000, 9000], s_q=1, h_q=128, seed=166)
+    for p in (large, small, large, large):
+        q, kv, bt, sl = to_device(p)
+        md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q, 1)
+        assert int(ns[-1].item()) > ns.numel() - 1, "the case must split some sequence"
+        o, lse = mla.flash_mla_with_kvcache(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale)
+        torch.cuda.synchronize()
+        ws = mla.api.get_workspace(mla.workspace_bytes(p.batch, p.s_q, p.h_q, 1, md.shape[0]), q.device,
+                                   mla.workspace_zero_bytes(p.batch, p.s_q, p.h_q, 1))
+        assert mla.read_device_status(ws, clear=False) == 0
+        o_ref, lse_ref = oracle_full(oracle_mod, p)
+        print(compare(o, lse, o_ref, lse_ref, p.dtype, f"batch {p.batch} on the cached workspace"))
+
+
 def test_metadata_kernel_matches_host_schedule():
     rng = np.random.default_rng(7)
     for hpk in (16, 128, 256):
@@ -203,19 +222,54 @@ def test_host_buffers_end_to_end(oracle_mod):
 
 
 # ---------------------------------------------------------------- full-size workloads
-@pytest.mark.parametrize("name", W.WORKLOADS)
-def test_parity_full_size_sampled(oracle_mod, name):
-    p = W.make_workload(name)
-    o, lse, md, ns = run_gpu(p)
+def _full_size_sample(p, rng_seed=99):
     rows_total = p.batch * p.s_q * p.h_q
-    rng = np.random.default_rng(99)
-    sample = np.unique(np.concatenate([
+    rng = np.random.default_rng(rng_seed)
+    return np.unique(np.concatenate([
         rng.choice(rows_total, size=min(48, rows_total), replace=False),
         [0, rows_total - 1],
         # rows of the longest and the shortest sequence
         np.argmax(p.cache_seqlens) * p.s_q * p.h_q + np.arange(min(8, p.s_q * p.h_q)),
         np.argmin(p.cache_seqlens) * p.s_q * p.h_q + np.arange(min(8, p.s_q * p.h_q)),
     ])).astype(np.int64)
+
+
+def test_parity_full_size_active_heads(oracle_mod):
+    # The speculative workload as the benchmark times it: its 16 real heads of 64 declared
+    # with active_heads (the padding-head kernel), full size.  Sampled real-head rows match
+    # the oracle; the padding heads' O and LSE are left as they were.
+    p = W.make_workload("spec_padded")
+    assert p.active_heads == 16
+    q, kv, bt, sl = to_device(p)
+    md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q, 1)
+    o = torch.full((p.batch, p.s_q, p.h_q, 512), 7.0, dtype=q.dtype, device="cuda")
+    lse = torch.full((p.batch, p.s_q, p.h_q), 7.0, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(mla.workspace_bytes(p.batch, p.s_q, p.h_q, 1, md.shape[0]), dtype=torch.uint8, device="cuda")
+    mla.flash_mla_with_kvcache(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale,
+                               workspace=ws, out=o, lse=lse, active_heads=p.active_heads)
+    torch.cuda.synchronize()
+    assert mla.read_device_status(ws) == 0
+    rows_total = p.batch * p.s_q * p.h_q
+    heads = np.arange(rows_total) % p.h_q
+    real = heads < p.active_heads
+    sample = _full_size_sample(p)
+    sample = np.unique(np.concatenate([sample[real[sample]],
+                                       np.random.default_rng(98).choice(np.flatnonzero(real), 48, replace=False)]))
+    o_ref, lse_ref = oracle_rows(oracle_mod, p, sample)
+    idx = torch.from_numpy(sample).cuda()
+    print(compare(o.reshape(rows_total, p.dv)[idx], lse.reshape(rows_total)[idx], o_ref, lse_ref, p.dtype,
+                  "spec_padded, 16 active heads, sampled"))
+    assert bool((o[:, :, p.active_heads:] == 7.0).all()), "padding heads' O was written"
+    assert bool((lse[:, :, p.active_heads:] == 7.0).all()), "padding heads' LSE was written"
+    assert torch.isfinite(o[:, :, :p.active_heads]).all()
+    assert bool(torch.isfinite(lse[:, :, :p.active_heads]).all())
+
+@pytest.mark.parametrize("name", W.WORKLOADS)
+def test_parity_full_size_sampled(oracle_mod, name):
+    p = W.make_workload(name)
+    o, lse, md, ns = run_gpu(p)
+    rows_total = p.batch * p.s_q * p.h_q
+    sample = _full_size_sample(p)
     o_ref, lse_ref = oracle_rows(oracle_mod, p, sample)
     o_s = o.reshape(rows_total, p.dv)[torch.from_numpy(sample).cuda()]
     l_s = lse.reshape(rows_total)[torch.from_numpy(sample).cuda()]

@@ -4,10 +4,12 @@ mla_decode_with_kvcache_noalloc is for callers that cannot allocate device
 memory at decode time (pre-planned runtimes, plugins that only receive tensor
 pointers, allocation-free latency paths): it keeps its split-KV scratch in a
 fixed array inside the library instead of a caller-provided workspace.  This
-test calls it through the C ABI twice in a row, on two different problems whose
-sequences are split across partitions (so the scratch holds partial results),
-and compares each output with mla_decode_with_kvcache run on a torch-allocated
-workspace, under the tolerances of the other parity tests.
+test calls it through the C ABI several times in a row, on different problems
+whose sequences are split across partitions (so the scratch holds partial
+results), and checks that each output is bit-identical to
+mla_decode_with_kvcache run on a torch-allocated workspace (both run the same
+kernels on the same inputs with the same workspace layout), and that the
+scratch's device status reads MLA_OK after each call.
 
 The file is named so that pytest collects it last.
 """
@@ -22,10 +24,6 @@ from mla_decode_attention_12_b200 import _lib
 from mla_decode_attention_12_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
-
-O_MAX_ABS = 2e-2
-LSE_MAX_ABS = 1e-2
-
 
 @pytest.fixture(scope="module")
 def lib():
@@ -72,7 +70,9 @@ def _noalloc(lib, p, t):
     lse = torch.full((p.batch, p.s_q, p.h_q), float("nan"), dtype=torch.float32, device="cuda")
     st = torch.cuda.current_stream().cuda_stream
     assert lib.mla_decode_with_kvcache_noalloc(*_args(p, q, kv, bt, sl, md, ns, o, lse), st) == 0
-    torch.cuda.synchronize()
+    status = ctypes.c_int(-1)
+    assert lib.mla_read_noalloc_status(0, ctypes.byref(status), st) == 0  # synchronises the stream
+    assert status.value == 0, f"device status {status.value} after an allocation-free call"
     return o, lse
 
 
@@ -82,16 +82,14 @@ def test_noalloc_matches_regular_on_two_calls(lib):
         W.make_problem([2500, 64, 700, 1, 4100], s_q=2, h_q=64, causal=True, seed=902),
         W.make_problem([20000, 3000, 100], s_q=1, h_q=128, seed=903, fp8_kv=True),  # "FP8 with scale" cache
     ]
-    for p in problems:
+    # a larger problem after a smaller one, then the first again: the scratch is shared
+    for p in problems + problems[:1]:
         t = _device_problem(p)
         assert int(t[5][-1]) > p.batch * ((p.s_q * p.h_q + 127) // 128), "no sequence was split"
         o_ref, lse_ref = _regular(lib, p, t)
         o, lse = _noalloc(lib, p, t)
         assert torch.isfinite(o).all()
-        assert (o.float() - o_ref.float()).abs().max().item() <= O_MAX_ABS
-        fin = torch.isfinite(lse_ref)
-        assert torch.equal(torch.isfinite(lse), fin)
-        assert (lse[fin] - lse_ref[fin]).abs().max().item() <= LSE_MAX_ABS
+        assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(lib):
