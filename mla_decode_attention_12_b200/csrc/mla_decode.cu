@@ -92,6 +92,7 @@ constexpr uint32_t kTmemS = 256;       // S buffers: [256, 288), [288, 320)
 constexpr uint32_t kTmemQ = 320;       // Q columns [0, 384) as the A operand: [320, 512)
 constexpr int kQTmemBoxes = 6;         // 64-column boxes of Q kept in tensor memory
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kQPrefetchPages = 8;         // pages before a chunk's end at which the next Q goes to L2
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 constexpr int kWorkspaceHeader = 256;
 // The workspace's control block has room for the counters of this many virtual batches
@@ -100,8 +101,7 @@ constexpr int kWorkspaceHeader = 256;
 constexpr int kMaxVirtualBatches = MLA_MAX_VIRTUAL_BATCHES;
 constexpr size_t kControlBytes = kWorkspaceHeader + 2 * sizeof(int32_t) * kMaxVirtualBatches;
 static_assert(kControlBytes % 256 == 0, "split partials start 256-byte aligned");
-constexpr int kNumMaps = 7;  // tensor maps of the split-KV kernel: Q, K, V, O, split partials, and O and
-                             // split partials with 8-row boxes
+constexpr int kNumMaps = 3;  // tensor maps of the split-KV kernel: Q, K, V
 
 // Shared-memory plan of one CTA (each CTA of the pair owns 64 query rows).  The FP8 kernel
 // trades a K stage and a V stage for rings of raw cache rows.
@@ -136,7 +136,7 @@ enum BarSlot : int {
     kBarQFree = 1,    // both: the chunk's Q K^T MMAs completed
     kBarKFull = 2,    // leader, 3 stages
     kBarKEmpty = 5,   // both, 3 stages
-    kBarVFull = 8,    // leader, 2 stages
+    kBarVFull = 8,    // leader, 2 stages: both V producers (the even one registering the TMA bytes)
     kBarVEmpty = 10,  // both, 2 stages
     kBarSFull = 12,   // both, 2 S buffers
     kBarPFull = 14,   // leader, 2 P buffers, 8 warps (4 per CTA)
@@ -200,9 +200,78 @@ struct DecodeParams {
                // partials (8 per split), combine CTAs past their wait
     int batch, s_q, h_q, rows, groups, max_blocks, num_blocks, causal, box_rows;
     int active_heads;  // heads >= active_heads are padding: not written, not combined
+    int o_align32;     // o is 32-byte aligned: 32-byte stores
     float scale_log2;
     int dtype, d_qk, num_parts;  // host-side dispatch only
 };
+
+// ------------------------------------------------------------------ timeline
+// Built only with -DMLA_TIMELINE (the library's timeline tool builds such a copy): selected
+// threads record (event id, %globaltimer ns since the CTA started) as one 32-bit word
+// (id << 27 | ns) into a per-CTA, per-role slice of a device array, read back on the host
+// with mla_timeline_read.  The product build compiles every TL_EV to nothing.
+enum TimelineEvent : uint32_t {
+    kEvSetupDone = 1,   // softmax thread 0: barriers, tensor memory and the grid dependency done
+    kEvChunkBegin = 2,  // softmax thread 0: a chunk's page loop begins (its Q is in tensor memory)
+    kEvQStored = 3,     // softmax thread 0: a chunk's Q stored into tensor memory
+    kEvSFull = 4,       // softmax thread 0: the logits of a page are ready
+    kEvPPosted = 5,     // softmax thread 0: P of a page handed to the MMA
+    kEvOFull = 6,       // softmax thread 0: the chunk's last P V completed
+    kEvEpiDone = 7,     // softmax thread 0: the chunk's output left tensor memory
+    kEvExit = 8,        // softmax thread 0: all chunks done
+    kEvClusterUp = 9,   // softmax thread 0: barriers and tensor memory set up, before the grid dependency
+    kEvQFreeSeen = 13,  // softmax thread 0: Q's tensor memory free, the Q row loads issue
+    kEvQLoaded = 14,    // softmax thread 0: the Q row loaded and its tensor-memory stores issued
+    kEvAnnounced = 15,  // softmax thread 0: the previous split announced (epilogue start)
+    kEvFirstTile = 17,  // softmax thread 0: the first 64 output columns written
+    kEvTileLoaded = 19,   // softmax thread 0: 64 output columns loaded from tensor memory
+    kEvMmaQFull = 10,   // MMA issuer: a chunk's Q complete
+    kEvMmaKFull = 11,   // MMA issuer: a K stage landed
+    kEvMmaPvGo = 12,    // MMA issuer: P and V of a page ready, P V issued
+    kEvKLoad = 16,      // K producer: a K stage free, its loads issued
+    kEvQLoad = 18,      // Q producer: a chunk's shared-memory Q loads issued
+    kEvVLoad = 20,      // V producer: a V stage free, its loads issued
+    kEvVTailLanded = 21,  // V producer: the V tile of a sequence's last page landed (before zeroing)
+    kEvVTailDone = 22,    // V producer: its rows past the sequence end zeroed and the stage handed over
+};
+#ifdef MLA_TIMELINE
+constexpr int kTlCtaWords = 1024;  // per CTA: 2 words of start time, then the roles' slices
+constexpr int kTlMaxCtas = 160;
+// Roles 0..4 (softmax, MMA, K, Q, V producers): first word and capacity of each slice.
+__host__ __device__ constexpr int tl_role_base(int role)
+{
+    return role == 0 ? 2 : role == 1 ? 402 : role == 2 ? 802 : role == 3 ? 914 : 924;
+}
+__host__ __device__ constexpr int tl_role_cap(int role)
+{
+    return role == 0 ? 400 : role == 1 ? 400 : role == 2 ? 112 : role == 3 ? 10 : 100;
+}
+static_assert(tl_role_base(4) + tl_role_cap(4) == kTlCtaWords, "timeline slices fill a CTA's words");
+__device__ uint32_t g_timeline[kTlMaxCtas * kTlCtaWords];
+struct Timeline {
+    uint32_t* buf = nullptr;
+    int n = 0, cap = 0;
+    uint64_t t0 = 0;
+    __device__ void open(int role, uint64_t start)
+    {
+        t0 = start;
+        if (blockIdx.x < kTlMaxCtas) {
+            buf = g_timeline + blockIdx.x * kTlCtaWords + tl_role_base(role);
+            cap = tl_role_cap(role);
+        }
+    }
+    __device__ void ev(uint32_t id)
+    {
+        if (n < cap) buf[n++] = (id << 27) | static_cast<uint32_t>((global_timer_ns() - t0) & 0x7FFFFFFu);
+    }
+};
+#define TL_OPEN(role) tl.open(role, tl_start)
+#define TL_EV(id) tl.ev(id)
+#else
+struct Timeline {};
+#define TL_OPEN(role) ((void)0)
+#define TL_EV(id) ((void)0)
+#endif
 
 // ------------------------------------------------------------------ helpers
 struct Sync {
@@ -298,9 +367,7 @@ __device__ __forceinline__ int page_of(const DecodeParams& p, const int32_t* tab
 template <bool kRope, bool kFp16, bool kPadHeads, bool kFp8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
     mla_splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                       const __grid_constant__ CUtensorMap tm_oacc, const __grid_constant__ CUtensorMap tm_o8,
-                       const __grid_constant__ CUtensorMap tm_oacc8, const DecodeParams p)
+                       const __grid_constant__ CUtensorMap tm_v, const DecodeParams p)
 {
     static_assert(!kFp8 || (kRope && !kFp16), "the FP8 cache has d_qk = 576 and bfloat16 queries");
     using L = Layout<kRope, kFp8>;
@@ -314,6 +381,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
     const uint32_t s_p = s_base + L::kOffP;
     const uint32_t s_bar = s_base + L::kOffBar;
     float* red = reinterpret_cast<float*>(smem + L::kOffRed);
+    [[maybe_unused]] Timeline tl;
+#ifdef MLA_TIMELINE
+    const uint64_t tl_start = global_timer_ns();
+    if (blockIdx.x < kTlMaxCtas) {
+        for (int i = 2 + threadIdx.x; i < kTlCtaWords; i += blockDim.x) g_timeline[blockIdx.x * kTlCtaWords + i] = 0;
+        __syncthreads();  // the zeros land before any event of this CTA
+        if (threadIdx.x == 0) {
+            g_timeline[blockIdx.x * kTlCtaWords] = static_cast<uint32_t>(tl_start);
+            g_timeline[blockIdx.x * kTlCtaWords + 1] = static_cast<uint32_t>(tl_start >> 32);
+        }
+    }
+    if (threadIdx.x == 0) TL_OPEN(0);
+#endif
     auto bar = [&](int slot) { return s_bar + 8u * slot; };
 
     const int warp = threadIdx.x >> 5;
@@ -342,7 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             mbar_init(bar(kBarRawVEmpty + s), kConvWarps);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(kBarVFull + s), kFp8 ? 2 * kConvWarps : 1);
+            mbar_init(bar(kBarVFull + s), kFp8 ? 2 * kConvWarps : 2);  // 16-bit: one V producer per CTA
             mbar_init(bar(kBarVEmpty + s), 1);
             mbar_init(bar(kBarSFull + s), 1);
             mbar_init(bar(kBarPFull + s), 8);
@@ -377,6 +457,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
     cluster_sync();  // both CTAs' barriers initialised before any remote arrive / transaction
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kOffBar + kOffTmemSlot);
+    if (threadIdx.x == 0) TL_EV(kEvClusterUp);
     // The set-up above touched no global memory, so it may overlap the grid before this
     // one (the metadata kernel); everything below may read what that grid wrote.
     grid_dependency_wait();
@@ -553,6 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             // 384 and up) once the previous chunk's Q K^T MMAs are done; the softmax
             // warps store columns [0, 384) into tensor memory.
             if (lane == 0) {
+                TL_OPEN(3);
                 const uint32_t q_tx = L::kQSmemBoxes * p.box_rows * 128;
                 const int y_off = 64 * static_cast<int>(cta);
                 uint32_t k = 0;
@@ -562,6 +644,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     if (hi <= lo) continue;
                     const int b = vb / p.groups, rg = vb % p.groups;
                     if (!(ok = sync.wait(bar(kBarQFree), (k & 1) ^ 1))) break;
+                    TL_EV(kEvQLoad);
                     if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * q_tx);
                     for (int i = 0; i < L::kQSmemBoxes; ++i)
                         tma_load_3d_pair(s_q + i * 8192, &tm_q, lead_bar(kBarQFull), 64 * (kQTmemBoxes + i),
@@ -605,6 +688,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     }
                 }
             } else if (lane == 0) {
+                TL_OPEN(2);
                 Ring<L::kKStages> ring;
                 int vb, lo, hi;
                 bool ok = true;
@@ -615,6 +699,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     for (int blk = lo; blk < hi; ++blk, ring.advance()) {
                         const uint32_t st = ring.stage;
                         if (!(ok = sync.wait(bar(kBarKEmpty + st), ring.phase ^ 1))) break;
+                        TL_EV(kEvKLoad);
                         const int page = page_of(p, table, blk);
                         if (leader) mbar_arrive_expect_tx(bar(kBarKFull + st), 2 * L::kKBytes);
                         const uint32_t dst = s_k + st * L::kKBytes;
@@ -662,11 +747,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 }
             } else {
                 // ============================ V producer ============================
-                // The whole warp waits (uniformly) so that it can zero the rows past the end of a
-                // sequence's last page before the MMA may read them.
+                // Each CTA's V producer arrives once per page on the even CTA's V_full barrier.  A
+                // full page: the even CTA's arrival registers both CTAs' TMA bytes, the odd one
+                // arrives once its loads are issued.  A sequence's last, partial page: each CTA
+                // loads its tile on a barrier of its own, zeroes the rows past the sequence end
+                // (they may hold anything, NaN included, and P V must not see them) and then
+                // arrives, with release semantics, as the softmax warps hand over P.  (A relaxed
+                // transaction count preceded by a cluster-scope fence cost several microseconds
+                // per partial page under full HBM load.)  The whole warp waits, uniformly.
                 uint32_t g = 0, tails = 0;
                 int vb, lo, hi;
                 bool ok = true;
+                if (lane == 0) TL_OPEN(4);
                 auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
                 while (ok && chunks.next(vb, lo, hi)) {
                     if (hi <= lo) continue;
@@ -678,16 +770,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     for (int blk = lo; blk < hi; ++blk, ++g) {
                         const uint32_t st = g & 1;
                         if (!(ok = wwait(bar(kBarVEmpty + st), ((g >> 1) & 1) ^ 1))) break;
+                        if (lane == 0) TL_EV(kEvVLoad);
                         const int page = page_of(p, table, blk);
                         const uint32_t dst = s_v + st * L::kVBytes;
                         const bool is_tail = (blk == last_page) && tail != 0;
-                        if (lane == 0 && leader) mbar_arrive_expect_tx(bar(kBarVFull + st), 2 * L::kVBytes);
                         if (!is_tail) {
                             if (lane == 0) {
+                                if (leader) mbar_arrive_expect_tx(bar(kBarVFull + st), 2 * L::kVBytes);
                                 for (int i = 0; i < 4; ++i) {
                                     const int box = 4 * (i >> 1) + 2 * static_cast<int>(cta) + (i & 1);
                                     tma_load_2d_pair(dst + i * 8192, &tm_v, lead_bar(kBarVFull + st), 64 * box, page * kPage);
                                 }
+                                if (!leader) mbar_arrive_remote(lead_bar(kBarVFull + st));
                             }
                         } else {
                             if (lane == 0) {
@@ -698,19 +792,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                                 }
                             }
                             if (!(ok = wwait(bar(kBarTail), tails & 1))) break;
+                            if (lane == 0) TL_EV(kEvVTailLanded);
                             ++tails;
                             // rows [tail, 64) of each of the 4 boxes: contiguous bytes [tail*128, 8192)
-                            const int per_box = (kPage - tail) * 8;  // 16-byte words
-                            for (int i = lane; i < 4 * per_box; i += 32) {
-                                const int box = i / per_box, w16 = i % per_box;
-                                *reinterpret_cast<uint4*>(smem + L::kOffV + st * L::kVBytes + box * 8192 + tail * 128 +
-                                                          w16 * 16) = make_uint4(0, 0, 0, 0);
+                            for (int box = 0; box < 4; ++box) {
+                                uint4* z = reinterpret_cast<uint4*>(smem + L::kOffV + st * L::kVBytes + box * 8192 +
+                                                                    tail * 128);
+                                for (int w16 = lane; w16 < (kPage - tail) * 8; w16 += 32) z[w16] = make_uint4(0, 0, 0, 0);
                             }
                             fence_proxy_async_smem();
                             __syncwarp();
                             if (lane == 0) {
-                                fence_acq_rel_cluster();
-                                mbar_complete_tx_cluster(lead_bar(kBarVFull + st), L::kVBytes);
+                                if (leader)
+                                    mbar_arrive(bar(kBarVFull + st));
+                                else
+                                    mbar_arrive_remote(lead_bar(kBarVFull + st));
+                                TL_EV(kEvVTailDone);
                             }
                         }
                     }
@@ -738,6 +835,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 const uint64_t p_desc = smem_desc(s_p, 16, 1024, kLayoutSW128);
                 const uint64_t v_desc = smem_desc(s_v, 8192, 1024, kLayoutSW128);
                 const bool issuer = elect_one();
+                if (issuer) TL_OPEN(1);
                 auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
                 uint32_t g = 0, k = 0;
                 int vb, lo, hi;
@@ -752,6 +850,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     if (!wwait(bar(kBarVFull + vs), vpar)) return false;
                     tc_fence_after();
                     if (issuer) {
+                        TL_EV(kEvMmaPvGo);
                         const uint64_t pd0 = p_desc + ((pb * L::kPBytes) >> 4);
                         const uint64_t vd0 = v_desc + ((vs * L::kVBytes) >> 4);
     #pragma unroll
@@ -776,6 +875,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     const int n = hi - lo;
                     if (n <= 0) continue;
                     if (!(ok = wwait(bar(kBarQFull), k & 1))) break;
+                    if (issuer) TL_EV(kEvMmaQFull);
                     for (int j = 0; j < n && ok; ++j, kring.advance()) {
                         const uint32_t gp = g + j;
                         const uint32_t sb = gp & 1;
@@ -783,6 +883,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                         if (!(ok = wwait(bar(kBarKFull + st), kring.phase))) break;
                         tc_fence_after();
                         if (issuer) {
+                            TL_EV(kEvMmaKFull);
                             const uint64_t kd0 = k_desc + ((st * L::kKBytes) >> 4);
                             // Q columns [0, 384) from tensor memory (8 columns per K=16 step) ...
     #pragma unroll
@@ -838,24 +939,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             return reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
                                                   (static_cast<size_t>(qvb / p.groups) * p.rows + qrow_idx) * p.d_qk * 2);
         };
+        // The whole row (the tensor-memory columns this warp stores and the shared-memory
+        // ones the Q producer loads), once per row: threads t and t ^ 64 share it.
         auto prefetch_q_row = [&](int qvb) {
             bool valid;
             const uint8_t* a = reinterpret_cast<const uint8_t*>(q_row_ptr(qvb, valid));
-            if (valid)
-                for (int i = 0; i < 6; ++i) prefetch_l2(a + 128 * i);
+            if (valid && h == 0)
+                for (int i = 0; i < p.d_qk * 2 / 128; ++i) prefetch_l2(a + 128 * i);
         };
         // Q columns [0, 384) of this thread's row of chunk `kq` into tensor memory, the A
         // operand of Q K^T.  Threads t and t ^ 64 hold the same row and write the same
-        // values: the pair MMA reads A duplicated in lane quadrants {0,2} and {1,3}.
+        // values: the pair MMA reads A duplicated in lane quadrants {0,2} and {1,3}.  The
+        // loads are issued before the wait for the region to be free: they only fill registers.
         auto store_q = [&](int qvb, uint32_t kq) -> bool {
             bool valid;
             const uint4* qrow = q_row_ptr(qvb, valid);
-            if (!wwait(bar(kBarQFree), (kq & 1) ^ 1)) return false;
-            tc_fence_after();
             // all 48 loads in flight at once: one memory round trip
             uint4 v[48];
 #pragma unroll
             for (int i = 0; i < 48; ++i) v[i] = valid ? __ldg(qrow + i) : make_uint4(0, 0, 0, 0);
+            if (!wwait(bar(kBarQFree), (kq & 1) ^ 1)) return false;
+            if (t == 0) TL_EV(kEvQFreeSeen);
+            tc_fence_after();
 #pragma unroll
             for (int c = 0; c < 6; ++c) {
                 uint32_t w[32];
@@ -868,6 +973,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 }
                 tmem_st32(tmem + kTmemQ + lane_base + 32 * c, w);
             }
+            if (t == 0) TL_EV(kEvQLoaded);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -885,21 +991,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         // The combine of a virtual batch starts once the 8 warps of each of its splits (4 per
         // CTA of the pair) have announced their partial results.  A warp announces a split
         // at the start of its next epilogue, or at the end, when its stores have long
-        // completed, so the wait for completion costs nothing.
+        // completed, so the fences before the announcement cost little.
         int announce_vb = -1;
         auto announce = [&]() {
             if (announce_vb >= 0) {
+                __threadfence();  // this lane's partial-output and LSE stores of that split ...
                 __syncwarp();
                 if (lane == 0) {
-                    bulk_wait_all();             // this warp's tile stores of that split are complete
-                    fence_proxy_async_global();  // ... and ordered before the counter update
-                    __threadfence();             // (with the LSE stores of the warp)
+                    __threadfence();  // ... and the whole warp's, before the counter update
                     atomicAdd(p.ctl + 2 * announce_vb, 1);
                 }
                 __syncwarp();
                 announce_vb = -1;
             }
         };
+        if (t == 0) TL_EV(kEvSetupDone);
         bool have = chunks.next(vb, lo, hi);
         bool q_ready = false;  // this chunk's Q already stored (ahead of the previous epilogue)
         while (ok && have) {
@@ -916,23 +1022,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             const int n = hi - lo;
             float m_ref = -INFINITY, l_half = 0.f;
 
-            if (n > 0 && !q_ready && !(ok = store_q(vb, k))) break;
-            {
-                // The next chunk's Q row goes to L2 now, so storing it later hits L2.
-                ChunkIter peek = chunks;
-                int pvb, plo, phi;
-                while (peek.next(pvb, plo, phi))
-                    if (phi > plo) {
-                        prefetch_q_row(pvb);
-                        break;
-                    }
+            if (n > 0 && !q_ready) {
+                if (!(ok = store_q(vb, k))) break;
+                if (t == 0) TL_EV(kEvQStored);
             }
+            if (t == 0) TL_EV(kEvChunkBegin);
             q_ready = false;
+            // The next chunk's Q row goes to L2 a few pages before the end of this chunk, so
+            // that loading it at the transition hits L2 (earlier, the KV stream through L2
+            // would evict it again).
+            const int j_prefetch = max(0, n - kQPrefetchPages);
 
             for (int j = 0; j < n; ++j) {
+                if (j == j_prefetch) {
+                    ChunkIter peek = chunks;
+                    int pvb, plo, phi;
+                    while (peek.next(pvb, plo, phi))
+                        if (phi > plo) {
+                            prefetch_q_row(pvb);
+                            break;
+                        }
+                }
                 const uint32_t gp = g + j;
                 const uint32_t sb = gp & 1;
                 if (!(ok = wwait(bar(kBarSFull + sb), (gp >> 1) & 1))) break;
+                if (t == 0) TL_EV(kEvSFull);
                 tc_fence_after();
                 // Logits stay unscaled until the exponent: scale > 0 keeps the maximum, and
                 // scale * s - ref is one FFMA.  Only a page the row does not fully see
@@ -1035,6 +1149,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     else
                         mbar_arrive_remote(p_full_lead[sb]);
                 }
+                if (t == 0) TL_EV(kEvPPosted);
             }
             if (!ok) break;
 
@@ -1045,6 +1160,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             const bool have_next = chunks.next(nvb, nlo, nhi);
             if (have_next && nhi > nlo && n > 0) {
                 if (!(ok = store_q(nvb, k + 1))) break;
+                if (t == 0) TL_EV(kEvQStored);
                 q_ready = true;
             }
 
@@ -1063,53 +1179,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             const float lse_v = (l_sum > 0.f) ? (m_ref + log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
             if (!empty) {
                 if (!(ok = wwait(bar(kBarOFull), k & 1))) break;
+                if (t == 0) TL_EV(kEvOFull);
                 tc_fence_after();
             }
             announce();
-            // O leaves tensor memory 64 columns at a time.  Each warp writes its 32 rows
-            // into a 4 KB tile of shared memory (the P buffers are idle now) in the
-            // 128-byte-swizzled layout of the output tensor maps, and lane 0 hands the
-            // tile to the TMA unit: the global writes proceed asynchronously while the
-            // warp moves on.  A tile is rewritten only after the TMA unit has read it.
+            if (t == 0) TL_EV(kEvAnnounced);
+            // O leaves tensor memory 64 columns at a time and goes straight from registers to
+            // global memory: each lane writes its row's 64 values with 32-byte stores (whole
+            // sectors).  No staging tile, no TMA unit (whose queue is shared with the
+            // producers' loads), nothing to wait for.  Rows past the end and padding heads are
+            // skipped.
             {
-                const uint32_t stage = s_p + warp * 4096;
-                uint8_t* stage_row = smem + L::kOffP + warp * 4096 + lane * 128;
-                const int row_in_group = 64 * static_cast<int>(cta) + (t & 32);  // warp's first row
-                // Rows past the end are clipped by the tensor maps.  A tile whose rows are all
-                // real heads is stored whole; one that also holds padding heads is stored in
-                // 8-row groups (each all real or all padding: h_q and active_heads are
-                // multiples of 8 then), skipping the padding ones.
-                // (Without padding heads, kPadHeads = false, every tile that starts before
-                // the last row is stored whole.)
-                bool tile_live, tile_whole = true;
-                uint32_t real_rows = 0xffffffffu;
-                if constexpr (kPadHeads) {
-                    const int lane_row = rg * kRowsPerGroup + row_in_group + lane;
-                    const bool lane_padding = lane_row < p.rows && lane_row % p.h_q >= p.active_heads;
-                    real_rows = __ballot_sync(0xffffffffu, lane_row < p.rows && !lane_padding);
-                    tile_live = real_rows != 0u;
-                    tile_whole = !__any_sync(0xffffffffu, lane_padding);
-                } else {
-                    tile_live = rg * kRowsPerGroup + row_in_group < p.rows;
-                }
-                auto stage_free = [&]() {
-                    if (lane == 0) bulk_wait_read_all();
-                    __syncwarp();
-                };
-                auto stage_issue = [&](const CUtensorMap* map, const CUtensorMap* map8, int x, int y, int z) {
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0 && tile_live) {
-                        if (tile_whole) {
-                            tma_store_3d(map, stage, x, y, z);
-                        } else {
-#pragma unroll
-                            for (int g8 = 0; g8 < 4; ++g8)
-                                if ((real_rows >> (8 * g8)) & 0xffu) tma_store_3d(map8, stage + 1024 * g8, x, y + 8 * g8, z);
-                        }
-                        bulk_commit_group();
-                    }
-                };
+                const int row_g = 64 * static_cast<int>(cta) + (t & 32) + lane;  // this lane's row in the group
+                const int grow = rg * kRowsPerGroup + row_g;
+                const bool live = grow < p.rows && (!kPadHeads || grow % p.h_q < p.active_heads);
+                uint8_t* const o_row = static_cast<uint8_t*>(p.o) + (static_cast<size_t>(b) * p.rows + grow) * (kDv * 2);
+                float* const acc_row = p.o_accum + (slot * kRowsPerGroup + row_g) * static_cast<size_t>(kDv);
 #pragma unroll 1
                 for (int blk2 = 0; blk2 < 4; ++blk2) {
                     // two 32-column TMEM loads in flight per wait
@@ -1120,6 +1205,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                         tmem_wait_ld();
                         reg_fence(v2[0]);
                         reg_fence(v2[1]);
+                        if (t == 0) TL_EV(kEvTileLoaded);
                         if (blk2 == 3) {
                             // O has left tensor memory: the next chunk's P V may start
                             tc_fence_before();
@@ -1136,38 +1222,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                         for (int e = 0; e < 32; ++e) v2[0][e] = v2[1][e] = 0;
                     }
                     const int col0 = 256 * (blk2 >> 1) + 128 * h + 64 * (blk2 & 1);  // first d_v column
-                    if (nsplit == 1) {
-                        // 64 16-bit values of the row: eight 16-byte chunks
-                        stage_free();
+                    if (live) {
+                        if (nsplit == 1) {
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const uint32_t* v = v2[c >> 2] + 8 * (c & 3);
-                            uint4 w;
-                            w.x = pack2(__uint_as_float(v[0]) * inv_l, __uint_as_float(v[1]) * inv_l, kFp16);
-                            w.y = pack2(__uint_as_float(v[2]) * inv_l, __uint_as_float(v[3]) * inv_l, kFp16);
-                            w.z = pack2(__uint_as_float(v[4]) * inv_l, __uint_as_float(v[5]) * inv_l, kFp16);
-                            w.w = pack2(__uint_as_float(v[6]) * inv_l, __uint_as_float(v[7]) * inv_l, kFp16);
-                            *reinterpret_cast<uint4*>(stage_row + ((c ^ (lane & 7)) << 4)) = w;
-                        }
-                        stage_issue(&tm_o, &tm_o8, col0, rg * kRowsPerGroup + row_in_group, b);
-                    } else {
-                        // fp32 partial: two tiles of 32 columns
+                            for (int c = 0; c < 4; ++c) {  // 16 values (32 bytes) per store
+                                const uint32_t* v = v2[c >> 1] + 16 * (c & 1);
+                                uint32_t w[8];
 #pragma unroll
-                        for (int hb = 0; hb < 2; ++hb) {
-                            stage_free();
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const uint32_t* v = v2[hb] + 4 * c;
-                                *reinterpret_cast<float4*>(stage_row + ((c ^ (lane & 7)) << 4)) =
-                                    make_float4(__uint_as_float(v[0]) * inv_l, __uint_as_float(v[1]) * inv_l,
-                                                __uint_as_float(v[2]) * inv_l, __uint_as_float(v[3]) * inv_l);
+                                for (int i = 0; i < 8; ++i)
+                                    w[i] = pack2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l, kFp16);
+                                st_global_32B(o_row + (col0 + 16 * c) * 2, w, p.o_align32);
                             }
-                            stage_issue(&tm_oacc, &tm_oacc8, col0 + 32 * hb, row_in_group, static_cast<int>(slot));
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {  // 8 values (32 bytes) per store
+                                const uint32_t* v = v2[c >> 2] + 8 * (c & 3);
+                                uint32_t w[8];
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(__uint_as_float(v[i]) * inv_l);
+                                st_global_32B(acc_row + col0 + 8 * c, w, true);
+                            }
                         }
                     }
+                    if (blk2 == 0 && t == 0) TL_EV(kEvFirstTile);
                 }
-                stage_free();  // the tiles are P buffers again for the next chunk
             }
+            if (t == 0) TL_EV(kEvEpiDone);
             if (h == 0 && row_valid && (!kPadHeads || row % p.h_q < p.active_heads)) {
                 if (nsplit == 1)
                     p.lse[static_cast<size_t>(b) * p.rows + row] = lse_v;
@@ -1183,10 +1263,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             hi = nhi;
         }
         if (ok) announce();
-        // Shared memory must outlive the TMA unit's reads of the output tiles; the writes
-        // themselves are complete, and visible to the next grid, when the grid completes.
-        if (lane == 0) bulk_wait_read_all();
-        __syncwarp();
+        if (t == 0) TL_EV(kEvExit);
     }
 
     // ---------------- teardown
@@ -1549,7 +1626,7 @@ static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorM
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     programmatic_launch(cfg, attr, dim3(grid), dim3(kFp8 ? kThreadsFp8 : kThreads), smem, stream);
-    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], prm);
+    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], prm);
 }
 
 // The kernel variant with padding-head logic runs only when some heads are padding.
@@ -1710,11 +1787,11 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     prm.box_rows = rows < 64 ? rows : 64;  // query rows per CTA of the pair
     prm.scale_log2 = softmax_scale * 1.4426950408889634f;
     prm.active_heads = effective_active_heads(active_heads, h_q);
+    prm.o_align32 = (reinterpret_cast<uintptr_t>(o) & 31) == 0;
     prm.dtype = dtype;
     prm.d_qk = d_qk;
     prm.num_parts = num_parts;
     if (batch == 0) return MLA_OK;
-    const size_t slots = workspace_slots(batch, groups, num_parts);
     workspace_pointers(workspace, batch, groups, num_parts, prm);
     if (!maps) return MLA_OK;
 
@@ -1737,20 +1814,7 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
                          CU_TENSOR_MAP_SWIZZLE_128B)) &&
         (fp8 ? encode_2d(&maps[2], kvcache, CU_TENSOR_MAP_DATA_TYPE_UINT8, kFp8Row, kv_rows, kFp8Row, 16,
                          kPage / 2, CU_TENSOR_MAP_SWIZZLE_NONE)
-             : encode_2d(&maps[2], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B)) &&
-        // O: [batch][rows][512] 16-bit, stored in tiles of 64 columns x 32 rows (rows past
-        // the end are clipped by the TMA unit); split partials: [slots][128][512] fp32,
-        // tiles of 32 columns x 32 rows.
-        encode_3d(&maps[3], o, dt, kDv, rows, batch, kDv * 2, static_cast<uint64_t>(kDv) * 2 * rows, 64,
-                  rows < 32 ? rows : 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
-        encode_3d(&maps[4], prm.o_accum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kDv, kRowsPerGroup, slots, kDv * 4,
-                  static_cast<uint64_t>(kDv) * 4 * kRowsPerGroup, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
-        // the same with 8-row boxes: tiles that mix real and padding heads are stored
-        // 8 rows at a time (one 1 KB swizzle atom each), skipping the padding groups
-        encode_3d(&maps[5], o, dt, kDv, rows, batch, kDv * 2, static_cast<uint64_t>(kDv) * 2 * rows, 64,
-                  rows < 8 ? rows : 8, CU_TENSOR_MAP_SWIZZLE_128B) &&
-        encode_3d(&maps[6], prm.o_accum, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kDv, kRowsPerGroup, slots, kDv * 4,
-                  static_cast<uint64_t>(kDv) * 4 * kRowsPerGroup, 32, 8, CU_TENSOR_MAP_SWIZZLE_128B);
+             : encode_2d(&maps[2], kvcache, dt, d_qk, kv_rows, row_bytes, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B));
     return ok ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -1854,6 +1918,15 @@ mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int dv, int
     workspace_pointers(workspace, batch, groups, num_parts, prm);
     return launch_combine_stage(prm, static_cast<cudaStream_t>(stream));
 }
+
+#ifdef MLA_TIMELINE
+// Timeline build only: copies the event array (kTlMaxCtas x kTlCtaWords words) to `host`.
+MLA_API mla_status mla_timeline_read(uint32_t* host, size_t words)
+{
+    if (!host || words < static_cast<size_t>(kTlMaxCtas) * kTlCtaWords) return MLA_ERR_INVALID_ARG;
+    return cudaMemcpyFromSymbol(host, g_timeline, sizeof(g_timeline)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+#endif
 
 mla_status mla_read_device_status(void* workspace, int clear, int* device_status, void* stream)
 {

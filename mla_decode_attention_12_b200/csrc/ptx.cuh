@@ -215,6 +215,23 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* ptr)
     return v;
 }
 
+// 32 bytes to global memory: one 256-bit store when `p` is 32-byte aligned, else two 128-bit
+// stores (16-byte alignment is the caller's guarantee).
+__device__ __forceinline__ void st_global_32B(void* p, const uint32_t (&w)[8], bool aligned32)
+{
+    if (aligned32) {
+        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+                     "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                     : "memory");
+    } else {
+        asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                     : "memory");
+        asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(static_cast<uint8_t*>(p) + 16), "r"(w[4]),
+                     "r"(w[5]), "r"(w[6]), "r"(w[7])
+                     : "memory");
+    }
+}
+
 // Hint: bring the 128-byte line holding `gaddr` into L2.
 __device__ __forceinline__ void prefetch_l2(const void* gaddr)
 {
