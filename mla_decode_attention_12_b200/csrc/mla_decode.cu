@@ -91,6 +91,7 @@ constexpr uint32_t kTmemO = 0;         // O: columns [0, 256)
 constexpr uint32_t kTmemS = 256;       // S buffers: [256, 288), [288, 320)
 constexpr uint32_t kTmemQ = 320;       // Q columns [0, 384) as the A operand: [320, 512)
 constexpr int kQTmemBoxes = 6;         // 64-column boxes of Q kept in tensor memory
+constexpr int kQBoxesPerRound = 3;     // boxes of Q per round through the Q buffer
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kQPrefetchPages = 8;         // pages before a chunk's end at which the next Q goes to L2
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
@@ -109,7 +110,9 @@ template <bool kRope, bool kFp8 = false>
 struct Layout {
     static constexpr int kBoxes = kRope ? 9 : 8;               // 64-column boxes in a d_qk row
     static constexpr int kQSmemBoxes = kBoxes - kQTmemBoxes;   // Q boxes kept in shared memory
-    static constexpr int kQBytes = kQSmemBoxes * 8192;         // 64 rows, one SW128 box per 64 columns
+    // the Q buffer: 64 rows, one SW128 box per 64 columns; it also stages the tensor-memory
+    // part of Q, kQBoxesPerRound boxes at a time
+    static constexpr int kQBytes = (kQSmemBoxes > kQBoxesPerRound ? kQSmemBoxes : kQBoxesPerRound) * 8192;
     static constexpr int kKBytes = kBoxes * 4096;              // K: this CTA's 32 tokens of a page x d_qk
     static constexpr int kKStages = kFp8 ? 2 : 3;
     static constexpr int kVBytes = 4 * 8192;                   // V: 64 tokens x this CTA's 256 d_v columns
@@ -132,7 +135,7 @@ struct Layout {
 };
 
 enum BarSlot : int {
-    kBarQFull = 0,    // leader: Q of both CTAs in place (TMA bytes + 8 softmax warps' TMEM stores)
+    kBarQFull = 0,    // leader: a round of Q boxes of both CTAs landed in the Q buffer (TMA bytes)
     kBarQFree = 1,    // both: the chunk's Q K^T MMAs completed
     kBarKFull = 2,    // leader, 3 stages
     kBarKEmpty = 5,   // both, 3 stages
@@ -151,7 +154,8 @@ enum BarSlot : int {
     kBarRawKEmpty = 27,  // local, 3 stages: the converter warps done with them
     kBarRawVFull = 30,   // local, 2 stages: the peer rows' V slices and scales landed
     kBarRawVEmpty = 32,  // local, 2 stages
-    kBarCount = 34
+    kBarQCopied = 34,    // both: a round of Q boxes copied from the Q buffer into tensor memory
+    kBarCount = 35
 };
 
 // Position in a ring of kN stages: stage index and the parity of its current use.
@@ -172,6 +176,9 @@ static_assert(kOffAbort + 4 <= Layout<true>::kBarBytes, "barrier area too small"
 static_assert(2 * Layout<true>::kPBytes >= 4 * 4096 && 2 * Layout<false>::kPBytes >= 4 * 4096,
               "epilogue staging (4 KB per softmax warp) must fit in the P buffers");
 static_assert(kTmemQ + 8 * 4 * kQTmemBoxes == kTmemCols, "tensor memory plan");
+static_assert(2 * kQBoxesPerRound == kQTmemBoxes && Layout<true>::kQSmemBoxes <= kQBoxesPerRound &&
+                  Layout<false>::kQSmemBoxes <= kQBoxesPerRound,
+              "Q goes through the Q buffer in three rounds: two into tensor memory, the rest stays");
 static_assert(Layout<true>::kSmemBytes <= 232448 && Layout<false>::kSmemBytes <= 232448 &&
                   Layout<true, true>::kSmemBytes <= 232448,
               "shared memory plan exceeds 227 KB");
@@ -213,15 +220,12 @@ struct DecodeParams {
 enum TimelineEvent : uint32_t {
     kEvSetupDone = 1,   // softmax thread 0: barriers, tensor memory and the grid dependency done
     kEvChunkBegin = 2,  // softmax thread 0: a chunk's page loop begins (its Q is in tensor memory)
-    kEvQStored = 3,     // softmax thread 0: a chunk's Q stored into tensor memory
     kEvSFull = 4,       // softmax thread 0: the logits of a page are ready
     kEvPPosted = 5,     // softmax thread 0: P of a page handed to the MMA
     kEvOFull = 6,       // softmax thread 0: the chunk's last P V completed
     kEvEpiDone = 7,     // softmax thread 0: the chunk's output left tensor memory
     kEvExit = 8,        // softmax thread 0: all chunks done
     kEvClusterUp = 9,   // softmax thread 0: barriers and tensor memory set up, before the grid dependency
-    kEvQFreeSeen = 13,  // softmax thread 0: Q's tensor memory free, the Q row loads issue
-    kEvQLoaded = 14,    // softmax thread 0: the Q row loaded and its tensor-memory stores issued
     kEvAnnounced = 15,  // softmax thread 0: the previous split announced (epilogue start)
     kEvFirstTile = 17,  // softmax thread 0: the first 64 output columns written
     kEvTileLoaded = 19,   // softmax thread 0: 64 output columns loaded from tensor memory
@@ -405,8 +409,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
 
     // ---------------- set-up
     if (threadIdx.x == 0) {
-        mbar_init(bar(kBarQFull), 1 + 8);
+        mbar_init(bar(kBarQFull), 1);
         mbar_init(bar(kBarQFree), 1);
+        mbar_init(bar(kBarQCopied), 1);
         // K and V stages are filled by TMA (one arrival with the byte count) or, for the FP8
         // cache, by the 8 converter warps of each CTA.
         for (int s = 0; s < L::kKStages; ++s) {
@@ -630,12 +635,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                                                                                     // instruction per warpgroup
         if (warp == kQWarp) {
             // ============================ Q producer ============================
-            // Loads the shared-memory part of each chunk's 64 query rows (columns
-            // 384 and up) once the previous chunk's Q K^T MMAs are done; the softmax
-            // warps store columns [0, 384) into tensor memory.
+            // A chunk's 64 query rows go through the Q buffer (3 boxes of 64 columns) in three
+            // rounds, once the previous chunk's Q K^T MMAs are done: boxes 0-2 and 3-5, which
+            // the MMA warp copies into tensor memory (the A operand of columns [0, 384)), then
+            // the last boxes, which stay in the buffer.  The boxes of the later rounds go to
+            // L2 with the first, so their loads hit L2.
             if (lane == 0) {
                 TL_OPEN(3);
-                const uint32_t q_tx = L::kQSmemBoxes * p.box_rows * 128;
                 const int y_off = 64 * static_cast<int>(cta);
                 uint32_t k = 0;
                 int vb, lo, hi;
@@ -643,12 +649,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 while (ok && chunks.next(vb, lo, hi)) {
                     if (hi <= lo) continue;
                     const int b = vb / p.groups, rg = vb % p.groups;
+                    const int y = rg * kRowsPerGroup + y_off;
                     if (!(ok = sync.wait(bar(kBarQFree), (k & 1) ^ 1))) break;
                     TL_EV(kEvQLoad);
-                    if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * q_tx);
-                    for (int i = 0; i < L::kQSmemBoxes; ++i)
-                        tma_load_3d_pair(s_q + i * 8192, &tm_q, lead_bar(kBarQFull), 64 * (kQTmemBoxes + i),
-                                         rg * kRowsPerGroup + y_off, b);
+                    for (int r = 0; r < 3 && ok; ++r) {
+                        const int box0 = kQBoxesPerRound * r;
+                        const int nbox = r < 2 ? kQBoxesPerRound : L::kBoxes - 2 * kQBoxesPerRound;
+                        if (r > 0 && !(ok = sync.wait(bar(kBarQCopied), (2 * k + r - 1) & 1))) break;
+                        if (leader) mbar_arrive_expect_tx(bar(kBarQFull), 2 * nbox * p.box_rows * 128);
+                        for (int i = 0; i < nbox; ++i)
+                            tma_load_3d_pair(s_q + i * 8192, &tm_q, lead_bar(kBarQFull), 64 * (box0 + i), y, b);
+                        if (r == 0)
+                            for (int i = kQBoxesPerRound; i < L::kBoxes; ++i) tma_prefetch_3d(&tm_q, 64 * i, y, b);
+                    }
                     ++k;
                 }
                 if (!ok) {
@@ -874,7 +887,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 while (ok && chunks.next(vb, lo, hi)) {
                     const int n = hi - lo;
                     if (n <= 0) continue;
-                    if (!(ok = wwait(bar(kBarQFull), k & 1))) break;
+                    // rounds 0 and 1 of the chunk's Q: from the Q buffer into tensor memory (a
+                    // 16-byte column slice per copy), ordered before the MMAs that read them
+                    for (int r = 0; r < 2 && ok; ++r) {
+                        if (!(ok = wwait(bar(kBarQFull), (3 * k + r) & 1))) break;
+                        tc_fence_after();
+                        if (issuer) {
+#pragma unroll
+                            for (int i = 0; i < kQBoxesPerRound; ++i)
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    tmem_cp_64x128_pair(tmem + kTmemQ + 32 * (kQBoxesPerRound * r + i) + 4 * j,
+                                                        q_desc + ((i * 8192 + 16 * j) >> 4));
+                            mma_commit_pair(bar(kBarQCopied), both);
+                        }
+                        __syncwarp();
+                    }
+                    if (!ok || !(ok = wwait(bar(kBarQFull), (3 * k + 2) & 1))) break;
                     if (issuer) TL_EV(kEvMmaQFull);
                     for (int j = 0; j < n && ok; ++j, kring.advance()) {
                         const uint32_t gp = g + j;
@@ -931,7 +960,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         uint32_t pair_phase = 0;
         const uint32_t p_full_lead[2] = {lead_bar(kBarPFull), lead_bar(kBarPFull + 1)};
         const uint32_t o_free_lead = lead_bar(kBarOFree);
-        const uint32_t q_full_lead = lead_bar(kBarQFull);
         auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
         auto q_row_ptr = [&](int qvb, bool& valid) {
             const int qrow_idx = (qvb % p.groups) * kRowsPerGroup + 64 * static_cast<int>(cta) + r;
@@ -946,44 +974,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             const uint8_t* a = reinterpret_cast<const uint8_t*>(q_row_ptr(qvb, valid));
             if (valid && h == 0)
                 for (int i = 0; i < p.d_qk * 2 / 128; ++i) prefetch_l2(a + 128 * i);
-        };
-        // Q columns [0, 384) of this thread's row of chunk `kq` into tensor memory, the A
-        // operand of Q K^T.  Threads t and t ^ 64 hold the same row and write the same
-        // values: the pair MMA reads A duplicated in lane quadrants {0,2} and {1,3}.  The
-        // loads are issued before the wait for the region to be free: they only fill registers.
-        auto store_q = [&](int qvb, uint32_t kq) -> bool {
-            bool valid;
-            const uint4* qrow = q_row_ptr(qvb, valid);
-            // all 48 loads in flight at once: one memory round trip
-            uint4 v[48];
-#pragma unroll
-            for (int i = 0; i < 48; ++i) v[i] = valid ? __ldg(qrow + i) : make_uint4(0, 0, 0, 0);
-            if (!wwait(bar(kBarQFree), (kq & 1) ^ 1)) return false;
-            if (t == 0) TL_EV(kEvQFreeSeen);
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < 6; ++c) {
-                uint32_t w[32];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    w[4 * i] = v[8 * c + i].x;
-                    w[4 * i + 1] = v[8 * c + i].y;
-                    w[4 * i + 2] = v[8 * c + i].z;
-                    w[4 * i + 3] = v[8 * c + i].w;
-                }
-                tmem_st32(tmem + kTmemQ + lane_base + 32 * c, w);
-            }
-            if (t == 0) TL_EV(kEvQLoaded);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (leader)
-                    mbar_arrive(bar(kBarQFull));
-                else
-                    mbar_arrive_remote(q_full_lead);
-            }
-            return true;
         };
         uint32_t g = 0, k = 0;
         int vb, lo, hi;
@@ -1007,7 +997,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         };
         if (t == 0) TL_EV(kEvSetupDone);
         bool have = chunks.next(vb, lo, hi);
-        bool q_ready = false;  // this chunk's Q already stored (ahead of the previous epilogue)
         while (ok && have) {
             const int b = vb / p.groups, rg = vb % p.groups;
             const int Lb = p.seqlens[b];
@@ -1022,12 +1011,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             const int n = hi - lo;
             float m_ref = -INFINITY, l_half = 0.f;
 
-            if (n > 0 && !q_ready) {
-                if (!(ok = store_q(vb, k))) break;
-                if (t == 0) TL_EV(kEvQStored);
-            }
             if (t == 0) TL_EV(kEvChunkBegin);
-            q_ready = false;
             // The next chunk's Q row goes to L2 a few pages before the end of this chunk, so
             // that loading it at the transition hits L2 (earlier, the KV stream through L2
             // would evict it again).
@@ -1153,16 +1137,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             }
             if (!ok) break;
 
-            // The next chunk's Q goes into tensor memory now (its region is free once this
-            // chunk's last Q K^T is done, which S_full of the last page implies), so the MMA
-            // can start the next chunk while this epilogue drains O.
+            // (The next chunk's Q reaches tensor memory without these warps: the Q producer
+            // and the MMA warp move it while this epilogue drains O.)
             int nvb = 0, nlo = 0, nhi = 0;
             const bool have_next = chunks.next(nvb, nlo, nhi);
-            if (have_next && nhi > nlo && n > 0) {
-                if (!(ok = store_q(nvb, k + 1))) break;
-                if (t == 0) TL_EV(kEvQStored);
-                q_ready = true;
-            }
 
             // ---- epilogue: full row sum from both halves, O / l, LSE
             const bool empty = (n <= 0);

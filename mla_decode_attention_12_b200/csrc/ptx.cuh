@@ -146,6 +146,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint3
         : "memory");
 }
 
+// Brings one box of a tensor into L2 (no shared-memory destination, no completion).
+__device__ __forceinline__ void tma_prefetch_3d(const void* map, int x, int y, int z)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
 // Bulk copy of `bytes` contiguous bytes (a multiple of 16, both addresses 16-byte
 // aligned) from global memory into this CTA's shared memory, completing on an mbarrier.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
@@ -441,6 +448,16 @@ __device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, ui
         "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// Two-SM copy of a 64-row x 16-byte slice of a shared-memory matrix (descriptor as for MMA
+// operands) into tensor memory at `taddr`, in each CTA of the pair from its own shared memory:
+// rows 0-31 go to lanes 0-31 and 64-95, rows 32-63 to lanes 32-63 and 96-127 (lane L holds row
+// L % 64, the duplicated A-operand layout of the pair MMA), 4 columns of 32 bits.  Issued by
+// one thread of the even CTA; ordered before the pair MMAs the same thread issues after it.
+__device__ __forceinline__ void tmem_cp_64x128_pair(uint32_t taddr, uint64_t s_desc)
+{
+    asm volatile("tcgen05.cp.cta_group::2.64x128b.warpx2::02_13 [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
 }
 
 // Arrive once on the mbarrier at offset `bar` in every CTA of `cta_mask` when all

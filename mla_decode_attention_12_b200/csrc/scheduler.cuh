@@ -11,14 +11,15 @@
 // Work units.  A "virtual batch" vb = b * row_groups + g is request b restricted
 // to query rows [128 g, 128 g + 128) of its s_q * h_q rows.  Every chunk (one
 // partition's share of one virtual batch) costs F = kFixedCost units of
-// overhead (Q load, pipeline refill, epilogue) plus one unit per 64-token page.
+// overhead (the output epilogue, refilling the pipeline) plus one unit per 64-token page.
 // Lay the virtual batches on a line: vb takes F units followed by its pages,
 // starting at C[vb] = sum of the costs before it; W is the total.  A partition
 // that starts inside a virtual batch's pages opens one more chunk than the line
 // shows, so it gets F units fewer of the line: with D = ceil((W - F) / num_parts),
 // partition 0 takes the line units [0, F + D) and partition p >= 1 the units
 // [F + p D, F + (p + 1) D); each partition's cost (pages + F per chunk) is then
-// at most F + D.  A unit position x maps to the page position (vb, blk) with vb
+// at most F + D.  D is at least F: a small batch leaves the last partitions empty rather
+// than cutting its sequences into pieces smaller than a chunk's overhead.  A unit position x maps to the page position (vb, blk) with vb
 // the virtual batch whose span holds x and blk = clamp(x - C[vb] - F, 0,
 // pages(vb)); partition p covers the page positions from map(start p) up to
 // map(start p+1).  A virtual batch whose pages are cut by partition starts is
@@ -49,7 +50,7 @@ namespace mla {
 
 constexpr int kPage = 64;
 constexpr int kRowsPerGroup = 128;
-constexpr int kFixedCost = 16;  // per-chunk overhead in page units (Q load, epilogue, pipeline refill), tuned on B200
+constexpr int kFixedCost = 12;  // per-chunk overhead in page units (epilogue, pipeline refill), tuned on B200
 constexpr int kMdInts = 8;
 
 MLA_HD inline int row_groups(int heads_per_kv) { return (heads_per_kv + kRowsPerGroup - 1) / kRowsPerGroup; }
@@ -87,7 +88,9 @@ MLA_HD inline void partition_range(int p, int num_parts, const long long* C, con
                                    long long total, int32_t* m)
 {
     long long D = (total - kFixedCost + num_parts - 1) / num_parts;  // line units of a partition after its first F
-    if (D < 0) D = 0;
+    // A partition shorter than one chunk's overhead would cost more than it saves: small
+    // batches use fewer partitions (the rest get empty ranges) instead of one-page splits.
+    if (D < kFixedCost) D = kFixedCost;
     auto start = [&](int q) -> long long { return q == 0 ? 0 : kFixedCost + static_cast<long long>(q) * D; };
     int bv, bb, ev, eb;
     unit_to_page(start(p), C, pages, nv, total, bv, bb);

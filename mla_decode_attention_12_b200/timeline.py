@@ -7,8 +7,8 @@ launch, reads the events of the last launch and splits each cluster's time into 
 
 * start-up: kernel entry -> the first page's logits (barriers, tensor memory, first Q and K);
 * streaming: first logits -> last P of each chunk (the page loop);
-* transitions: last P of a chunk -> first logits of the next (next Q stored, last P V,
-  output drained from tensor memory, then the next chunk's logits);
+* transitions: last P of a chunk -> first logits of the next (last P V, output drained from
+  tensor memory, then the next chunk's logits; and, on the MMA warp, the next chunk's Q ready);
 * last epilogue: last P of the last chunk -> the cluster's exit;
 * idle at the end: the cluster's exit -> the last cluster's exit.
 
@@ -32,9 +32,9 @@ LIB = os.path.join(HERE, "_mla_decode_timeline.so")
 CTA_WORDS, MAX_CTAS = 1024, 160
 ROLE_BASE = {"softmax": 2, "mma": 402, "k": 802, "q": 914, "v": 924}
 ROLE_CAP = {"softmax": 400, "mma": 400, "k": 112, "q": 10, "v": 100}
-EV = dict(setup=1, chunk=2, qstored=3, sfull=4, pposted=5, ofull=6, epidone=7, exit=8, cluster_up=9, mma_qfull=10,
-          mma_kfull=11, mma_pvgo=12, qfree_seen=13, qloaded=14, announced=15, first_tile=17, kload=16, qload=18,
-          tile_loaded=19, vload=20, vtail_landed=21, vtail_done=22)
+EV = dict(setup=1, chunk=2, sfull=4, pposted=5, ofull=6, epidone=7, exit=8, cluster_up=9, mma_qfull=10,
+          mma_kfull=11, mma_pvgo=12, announced=15, first_tile=17, kload=16, qload=18, tile_loaded=19, vload=20,
+          vtail_landed=21, vtail_done=22)
 
 
 def build_timeline_lib(force: bool = False) -> str:
@@ -120,6 +120,8 @@ def phases(B, grid):
         i, t = events(B, c, "softmax", t_off)
         if not (i == EV["exit"]).any() or not (i == EV["sfull"]).any():
             continue
+        im, tm = events(B, c - (c & 1), "mma", t_off)  # the pair's MMA warp runs in the even CTA
+        q_full = tm[im == EV["mma_qfull"]]
         # chunks: split the softmax events at each chunk-begin
         begins = np.flatnonzero(i == EV["chunk"])
         chunks = []
@@ -128,8 +130,7 @@ def phases(B, grid):
             S, P = tt[ii == EV["sfull"]], tt[ii == EV["pposted"]]
             if len(S) == 0:
                 continue
-            chunks.append(dict(begin=tt[0], S=S, P=P, q_next=tt[ii == EV["qstored"]], ofull=tt[ii == EV["ofull"]],
-                               epi=tt[ii == EV["epidone"]]))
+            chunks.append(dict(begin=tt[0], S=S, P=P, ofull=tt[ii == EV["ofull"]], epi=tt[ii == EV["epidone"]]))
         if not chunks:
             continue
         exit_t = t[i == EV["exit"]][-1]
@@ -139,11 +140,12 @@ def phases(B, grid):
         page_gaps = np.concatenate([np.diff(ch["P"]) for ch in chunks if len(ch["P"]) > 1] or [np.zeros(0)])
         trans, sub = [], []
         for a, b in zip(chunks[:-1], chunks[1:]):
-            trans.append(b["S"][0] - a["P"][-1])
-            q_done = a["q_next"][0] if len(a["q_next"]) else a["P"][-1]
-            of = a["ofull"][0] if len(a["ofull"]) else q_done
+            last_p = a["P"][-1]
+            trans.append(b["S"][0] - last_p)
+            of = a["ofull"][0] if len(a["ofull"]) else last_p
             ep = a["epi"][0] if len(a["epi"]) else of
-            sub.append((q_done - a["P"][-1], of - q_done, ep - of, b["S"][0] - ep))
+            qf = q_full[q_full > last_p - 2.0]  # the next chunk's Q can be ready a little before the last P
+            sub.append((of - last_p, ep - of, b["S"][0] - ep, (qf[0] - last_p) if len(qf) else np.nan))
         last = chunks[-1]
         per.append(dict(cta=c, entry=t_off[c], setup=setup - t_off[c], startup=chunks[0]["S"][0] - setup,
                         stream=stream, pages=pages, page_med=float(np.median(page_gaps)) if len(page_gaps) else np.nan,
@@ -183,10 +185,10 @@ def summarize(name: str, per, end: float, kernel_us: float) -> str:
              f"| exit time | {q(col('exit'))} |"]
     if len(each):
         lines += [f"| one transition: last P -> next logits ({len(each)}) | {q(each)} |",
-                  f"| .. next chunk's Q stored | {q(sub[:, 0])} |",
-                  f"| .. wait for the last P V | {q(sub[:, 1])} |",
-                  f"| .. output drained | {q(sub[:, 2])} |",
-                  f"| .. then next logits | {q(sub[:, 3])} |"]
+                  f"| .. wait for the last P V | {q(sub[:, 0])} |",
+                  f"| .. output drained | {q(sub[:, 1])} |",
+                  f"| .. then next logits | {q(sub[:, 2])} |",
+                  f"| .. (MMA warp) next chunk's Q ready, after the last P | {q(sub[:, 3])} |"]
     return "\n".join(lines) + "\n"
 
 

@@ -64,9 +64,10 @@ def check_schedule(seqlens, heads_per_kv, num_parts):
         assert [s for _, _, s in lst] == list(range(len(lst)))
         assert [lo for _, lo, _ in lst] == sorted(lo for _, lo, _ in lst)
     # balance: every partition's cost, pages plus the fixed cost of each of its
-    # chunks, stays within the budget F + ceil((W - F) / num_parts)
+    # chunks, stays within the budget F + max(ceil((W - F) / num_parts), F) (a partition
+    # is never given less than one chunk's overhead of pages)
     W = sum((pages(L) + FIXED) * groups for L in seqlens)
-    T = max(-(-(W - FIXED) // num_parts), 0) + FIXED
+    T = max(-(-(W - FIXED) // num_parts), FIXED) + FIXED
     cost = np.zeros(num_parts, np.int64)
     for p, vb, lo, hi, _ in ch:
         cost[p] += (hi - lo) + FIXED
