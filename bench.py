@@ -55,6 +55,10 @@ DESCR = {
                    "d_qk=576, d_v=512, cache_seqlens uniform in [1024,8192], page 64, shuffled block_table, "
                    "bf16 N(0,1) q, 656-byte cache rows (512 e4m3 latent + 4 fp32 scales + 64 bf16 rope, "
                    "|value| <= 3.5), scale 1/sqrt(576)",
+    "sparse_fp8": "token-level sparse MLA decode over an FP8-with-scale cache: batch 64, s_q=2, h_q=128, h_kv=1, "
+                  "d_qk=576, d_v=512, topk=2048 entries per query token drawn without repetition from its "
+                  "request's cache (cache_seqlens uniform in [8192,16384]), 656-byte cache rows, bf16 N(0,1) q, "
+                  "scale 1/sqrt(576)",
 }
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NVML_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
@@ -222,17 +226,22 @@ class Runner:
         self.sl = torch.from_numpy(p.cache_seqlens).to(dev)
         self.rows = p.s_q * p.h_q
         parts = mla.num_sm_parts(dev)
-        n_md, n_ns = mla.metadata_sizes(p.batch, self.rows, 1, parts)
+        sparse = p.indices is not None  # token-level sparse decode: the entry lists replace the block table
+        self.ind = torch.from_numpy(p.indices).to(dev) if sparse else None
+        md_kw = dict(h_q=p.h_q, topk=p.indices.shape[2]) if sparse else {}
+        n_md, n_ns = mla.metadata_sizes(p.batch * p.s_q if sparse else p.batch, p.h_q if sparse else self.rows, 1,
+                                        parts)
         self.md = torch.zeros(parts, 8, dtype=torch.int32, device=dev)
         self.ns = torch.zeros(n_ns, dtype=torch.int32, device=dev)
-        mla.get_mla_metadata(self.sl, self.rows, 1, out=(self.md, self.ns))
-        ws = torch.zeros(mla.workspace_bytes(p.batch, p.s_q, p.h_q, 1, parts), dtype=torch.uint8, device=dev)
+        mla.get_mla_metadata(self.sl, self.rows, 1, out=(self.md, self.ns), **md_kw)
+        ws_b, ws_s = (p.batch * p.s_q, 1) if sparse else (p.batch, p.s_q)
+        ws = torch.zeros(mla.workspace_bytes(ws_b, ws_s, p.h_q, 1, parts), dtype=torch.uint8, device=dev)
         # padding heads (the spec_padded workload) are declared, so their outputs are skipped
         self.call = mla.DecodeCall(self.q, self.kv, self.bt, self.sl, p.dv, self.md, self.ns, causal=p.causal,
                                    softmax_scale=p.scale, workspace=ws, active_heads=p.active_heads,
-                                   is_fp8_kvcache=p.fp8_kv)
+                                   is_fp8_kvcache=p.fp8_kv, indices=self.ind)
         self.launches_per_step = 3
-        stages = [lambda: mla.get_mla_metadata(self.sl, self.rows, 1, out=(self.md, self.ns)),
+        stages = [lambda: mla.get_mla_metadata(self.sl, self.rows, 1, out=(self.md, self.ns), **md_kw),
                   self.call.splitkv, self.call.combine]
         s = torch.cuda.Stream(dev)
         s.wait_stream(torch.cuda.current_stream(dev))
@@ -496,7 +505,7 @@ def run_ours(args):
 
     extra = {}
     names = [] if args.extra_workloads == "none" else (
-        [w for w in W.WORKLOADS if w != args.workload] if args.extra_workloads == "all"
+        [w for w in W.WORKLOADS + W.SPARSE_WORKLOADS if w != args.workload] if args.extra_workloads == "all"
         else [w for w in args.extra_workloads.split(",") if w and w != args.workload])
     if rank == 0:
         for name in names:

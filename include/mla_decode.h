@@ -226,6 +226,52 @@ MLA_API mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int
                                       void* stream);
 
 /*
+ * Token-level sparse decoding over an "FP8 with scale" cache (upstream FlashMLA
+ * documentation, "Sparse Attention (indices tensor)": indices [batch, s_q, topk],
+ * indices[i][j][k] = page * page_size + offset of the k-th row query token j of
+ * request i attends, -1 invalid, no block table; the support matrix lists sparse
+ * decoding with the FP8 cache only).
+ *
+ * For request b, query token s and head h (kv head 0):
+ *   E      = { k < topk : 0 <= indices[b][s][k] < num_blocks * 64 }   (other entries are invalid)
+ *   x_k    = softmax_scale * <q[b,s,h,:], row(indices[b][s][k])>,  k in E   (a row listed twice
+ *            counts twice)
+ *   lse    = log(sum_{k in E} exp(x_k))                   (-inf when E is empty)
+ *   o      = sum_{k in E} exp(x_k - lse) * row(...)[0:512] (0 when E is empty)
+ * with rows dequantized as for MLA_BF16_FP8KV.  No causal mask (the list is what the
+ * token sees).
+ *
+ * mla_get_metadata_sparse: the tile scheduler for num_tokens = batch * s_q query tokens of
+ *   topk entries each, h_q heads (h_q / h_kv rows per token); tile_md as for
+ *   mla_get_metadata with num_parts rows, num_splits [num_tokens * ceil(h_q / h_kv / 128) + 1].
+ * mla_decode_sparse:
+ *   q            device [batch, s_q, h_q, 576] bfloat16, 16-byte aligned
+ *   kvcache      device [num_blocks, 64, 1, 656] bytes ("FP8 with scale" rows), 16-byte aligned
+ *   indices      device int32 [batch, s_q, topk]
+ *   dtype        must be MLA_BF16_FP8KV (MLA_ERR_UNSUPPORTED otherwise); d_qk 576, dv 512, h_kv 1,
+ *                page_size 64
+ *   tile_md, num_splits, num_parts   from mla_get_metadata_sparse for this batch * s_q and topk
+ *   active_heads, softmax_scale, o, lse  as for mla_decode_with_kvcache
+ *   workspace    >= mla_decode_workspace_bytes(batch * s_q, 1, h_q, 1, num_parts)
+ * Enqueues the split-KV kernel and the combine kernel on `stream`.
+ * mla_decode_sparse_splitkv: its first stage alone; mla_decode_combine with batch * s_q,
+ *   s_q = 1 is the second (as for mla_decode_splitkv).
+ */
+MLA_API mla_status mla_get_metadata_sparse(int num_tokens, int topk, int h_q, int h_kv, int num_parts,
+                                           int32_t* tile_md, int32_t* num_splits, void* stream);
+MLA_API mla_status mla_decode_sparse(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache,
+                                     int num_blocks, int page_size, int h_kv, const int32_t* indices, int topk,
+                                     int dv, int dtype, const int32_t* tile_md, int num_parts,
+                                     const int32_t* num_splits, float softmax_scale, int active_heads, void* o,
+                                     float* lse, void* workspace, size_t workspace_bytes, void* stream);
+MLA_API mla_status mla_decode_sparse_splitkv(const void* q, int batch, int s_q, int h_q, int d_qk,
+                                             const void* kvcache, int num_blocks, int page_size, int h_kv,
+                                             const int32_t* indices, int topk, int dv, int dtype,
+                                             const int32_t* tile_md, int num_parts, const int32_t* num_splits,
+                                             float softmax_scale, int active_heads, void* o, float* lse,
+                                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Reads the device status word of a workspace (synchronises `stream`).
  * *device_status receives MLA_OK or the first device-side error recorded by a
  * decode call that used this workspace; clear != 0 then zeroes the workspace's

@@ -47,6 +47,14 @@ SIGNATURES = {
     "mla_decode_with_kvcache_noalloc": ([_P, _I, _I, _I, _I, _P, _I, _I, _I, _P, _I, _P, _I, _I,
                                          _P, _I, _P, _I, _F, _I, _P, _P, _P], _I),
     "mla_read_noalloc_status": ([_I, ctypes.POINTER(_I), _P], _I),
+    "mla_get_metadata_sparse": ([_I, _I, _I, _I, _I, _P, _P, _P], _I),
+    "mla_decode_sparse": ([_P, _I, _I, _I, _I,          # q, batch, s_q, h_q, d_qk
+                           _P, _I, _I, _I,              # kvcache, num_blocks, page_size, h_kv
+                           _P, _I, _I, _I,              # indices, topk, dv, dtype
+                           _P, _I, _P, _F, _I,          # tile_md, num_parts, num_splits, scale, active_heads
+                           _P, _P, _P, _SZ, _P], _I),   # o, lse, workspace, ws_bytes, stream
+    "mla_decode_sparse_splitkv": ([_P, _I, _I, _I, _I, _P, _I, _I, _I, _P, _I, _I, _I,
+                                   _P, _I, _P, _F, _I, _P, _P, _P, _SZ, _P], _I),
 }
 
 _lock = threading.Lock()

@@ -48,13 +48,18 @@ def metadata_sizes(batch: int, heads_per_kv: int, h_kv: int, num_parts: int):
 
 
 def get_mla_metadata(cache_seqlens: torch.Tensor, heads_per_kv: int, h_kv: int = 1, num_parts: int | None = None,
-                     out=None):
+                     out=None, h_q: int | None = None, topk: int | None = None):
     """Tile-scheduler metadata for one decoding step.
 
     ``cache_seqlens``: int32 [batch] on a CUDA device.  ``heads_per_kv`` is
     ``s_q * h_q // h_kv``.  Returns ``(tile_scheduler_metadata [num_parts, 8] int32,
     num_splits [batch * ceil(heads_per_kv / 128) + 1] int32)`` on the same device;
     ``out`` = (md, ns) writes into existing tensors instead.
+
+    With ``topk`` (and ``h_q``): the schedule of the token-level sparse decode, whose
+    batch * s_q query tokens each attend ``topk`` listed entries (upstream FlashMLA
+    documentation, "Sparse Attention (indices tensor)"); num_splits then has
+    ``batch * s_q * ceil(h_q / h_kv / 128) + 1`` entries.
     """
     if not cache_seqlens.is_cuda or cache_seqlens.dtype != torch.int32 or not cache_seqlens.is_contiguous():
         raise ValueError("cache_seqlens must be a contiguous int32 CUDA tensor")
@@ -64,6 +69,22 @@ def get_mla_metadata(cache_seqlens: torch.Tensor, heads_per_kv: int, h_kv: int =
     if num_parts is None:
         num_parts = num_sm_parts(dev)
     batch = cache_seqlens.numel()
+    if topk is not None:
+        if h_q is None or (heads_per_kv * h_kv) % h_q:
+            raise ValueError("the sparse schedule needs h_q, a divisor of heads_per_kv * h_kv")
+        tokens = batch * (heads_per_kv * h_kv // h_q)
+        n_md, n_ns = metadata_sizes(tokens, h_q // h_kv, h_kv, num_parts)
+        if out is not None:
+            md, ns = out
+            if md.numel() != n_md or ns.numel() != n_ns or md.dtype != torch.int32 or ns.dtype != torch.int32:
+                raise ValueError("metadata output tensors have the wrong size or dtype")
+        else:
+            md = torch.empty(n_md, dtype=torch.int32, device=dev).view(num_parts, 8)
+            ns = torch.empty(n_ns, dtype=torch.int32, device=dev)
+        with torch.cuda.device(dev):
+            _lib.check(_lib.load().mla_get_metadata_sparse(tokens, int(topk), h_q, h_kv, num_parts, _ptr(md),
+                                                           _ptr(ns), _stream(dev)), "mla_get_metadata_sparse")
+        return md, ns
     n_md, n_ns = metadata_sizes(batch, heads_per_kv, h_kv, num_parts)
     if out is not None:
         md, ns = out
@@ -125,8 +146,16 @@ class DecodeCall:
 
     def __init__(self, q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata, num_splits,
                  causal=False, softmax_scale=None, workspace=None, out=None, lse=None, active_heads=None,
-                 is_fp8_kvcache=False):
+                 is_fp8_kvcache=False, indices=None):
         dev = q.device
+        self.sparse = indices is not None
+        if self.sparse:
+            if not is_fp8_kvcache:
+                raise ValueError("the sparse decode (indices) reads an FP8-with-scale cache")
+            if indices.dtype != torch.int32 or indices.dim() != 3 or indices.shape[:2] != q.shape[:2]:
+                raise ValueError("indices must be int32 [batch, s_q, topk]")
+            if not indices.is_contiguous() or indices.device != dev:
+                raise ValueError(f"indices must be contiguous and on {dev}")
         if is_fp8_kvcache:
             if q.dtype != torch.bfloat16 or kvcache.dtype != torch.uint8 or kvcache.shape[-1] != FP8_ROW_BYTES:
                 raise ValueError("an FP8 cache takes bfloat16 q and a uint8 kvcache of 656-byte rows")
@@ -134,49 +163,59 @@ class DecodeCall:
                 raise ValueError("an FP8 cache has d_qk = 576")
         elif q.dtype not in _DTYPES or kvcache.dtype != q.dtype:
             raise ValueError("q and kvcache must both be bfloat16 or both float16")
-        for name, t in (("q", q), ("kvcache", kvcache), ("block_table", block_table),
-                        ("cache_seqlens", cache_seqlens), ("tile_scheduler_metadata", tile_scheduler_metadata),
-                        ("num_splits", num_splits)):
+        tensors = [("q", q), ("kvcache", kvcache), ("tile_scheduler_metadata", tile_scheduler_metadata),
+                   ("num_splits", num_splits)]
+        if not self.sparse:  # the sparse decode reads no block table and no lengths
+            tensors += [("block_table", block_table), ("cache_seqlens", cache_seqlens)]
+        for name, t in tensors:
             if not t.is_contiguous() or t.device != dev:
                 raise ValueError(f"{name} must be contiguous and on {dev}")
-        if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32:
-            raise ValueError("block_table and cache_seqlens must be int32")
         b, s_q, h_q, d_qk = q.shape
         num_blocks, page, h_kv, d2 = kvcache.shape
-        if ((not is_fp8_kvcache and d2 != d_qk) or block_table.dim() != 2 or block_table.shape[0] != b
-                or cache_seqlens.numel() != b):
-            raise ValueError("inconsistent shapes")
+        if not self.sparse:
+            if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32:
+                raise ValueError("block_table and cache_seqlens must be int32")
+            if ((not is_fp8_kvcache and d2 != d_qk) or block_table.dim() != 2 or block_table.shape[0] != b
+                    or cache_seqlens.numel() != b):
+                raise ValueError("inconsistent shapes")
         num_parts = tile_scheduler_metadata.shape[0]
         if out is None:
             out = torch.empty(b, s_q, h_q, dv, dtype=q.dtype, device=dev)
         if lse is None:
             lse = torch.empty(b, s_q, h_q, dtype=torch.float32, device=dev)
+        ws_b, ws_s = (b * s_q, 1) if self.sparse else (b, s_q)  # sparse: every token is a request
         if workspace is None:
-            workspace = get_workspace(workspace_bytes(b, s_q, h_q, h_kv, num_parts), dev,
-                                      workspace_zero_bytes(b, s_q, h_q, h_kv))
+            workspace = get_workspace(workspace_bytes(ws_b, ws_s, h_q, h_kv, num_parts), dev,
+                                      workspace_zero_bytes(ws_b, ws_s, h_q, h_kv))
         scale = float(softmax_scale) if softmax_scale is not None else 1.0 / math.sqrt(d_qk)
         self.device = dev
         self.out, self.lse, self.workspace = out, lse, workspace
-        self._keep = (q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits)
+        self._keep = (q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits, indices)
         active = 0 if active_heads is None else int(active_heads)  # 0: every head is real
         dtype = MLA_BF16_FP8KV if is_fp8_kvcache else _DTYPES[q.dtype]
-        self.args = (_ptr(q), b, s_q, h_q, d_qk, _ptr(kvcache), num_blocks, page, h_kv, _ptr(block_table),
-                     block_table.shape[1], _ptr(cache_seqlens), dv, dtype,
-                     _ptr(tile_scheduler_metadata), num_parts, _ptr(num_splits), int(bool(causal)), scale,
-                     active, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel())
-        self.combine_args = (b, s_q, h_q, h_kv, dv, dtype, _ptr(num_splits), num_parts, active,
+        if self.sparse:
+            self.args = (_ptr(q), b, s_q, h_q, d_qk, _ptr(kvcache), num_blocks, page, h_kv, _ptr(indices),
+                         indices.shape[2], dv, dtype, _ptr(tile_scheduler_metadata), num_parts, _ptr(num_splits),
+                         scale, active, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel())
+        else:
+            self.args = (_ptr(q), b, s_q, h_q, d_qk, _ptr(kvcache), num_blocks, page, h_kv, _ptr(block_table),
+                         block_table.shape[1], _ptr(cache_seqlens), dv, dtype,
+                         _ptr(tile_scheduler_metadata), num_parts, _ptr(num_splits), int(bool(causal)), scale,
+                         active, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel())
+        self.combine_args = (ws_b, ws_s, h_q, h_kv, dv, dtype, _ptr(num_splits), num_parts, active,
                              _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel())
 
     def run(self):
-        """Split-KV kernel then combine kernel (mla_decode_with_kvcache)."""
+        """Split-KV kernel then combine kernel (mla_decode_with_kvcache / mla_decode_sparse)."""
+        fn = "mla_decode_sparse" if self.sparse else "mla_decode_with_kvcache"
         with torch.cuda.device(self.device):
-            _lib.check(_lib.load().mla_decode_with_kvcache(*self.args, _stream(self.device)),
-                       "mla_decode_with_kvcache")
+            _lib.check(getattr(_lib.load(), fn)(*self.args, _stream(self.device)), fn)
         return self.out, self.lse
 
     def splitkv(self):
+        fn = "mla_decode_sparse_splitkv" if self.sparse else "mla_decode_splitkv"
         with torch.cuda.device(self.device):
-            _lib.check(_lib.load().mla_decode_splitkv(*self.args, _stream(self.device)), "mla_decode_splitkv")
+            _lib.check(getattr(_lib.load(), fn)(*self.args, _stream(self.device)), fn)
 
     def combine(self):
         with torch.cuda.device(self.device):
@@ -189,7 +228,7 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
                            num_splits: torch.Tensor, causal: bool = False, softmax_scale: float | None = None,
                            workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
                            lse: torch.Tensor | None = None, active_heads: int | None = None,
-                           is_fp8_kvcache: bool = False):
+                           is_fp8_kvcache: bool = False, indices: torch.Tensor | None = None):
     """MLA decode over a paged cache; returns ``(o [b, s_q, h_q, dv], lse [b, s_q, h_q] float32)``.
 
     ``is_fp8_kvcache``: ``kvcache`` is uint8 [num_blocks, 64, h_kv, 656] in the "FP8
@@ -200,6 +239,13 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
     ``active_heads``: heads ``[active_heads, h_q)`` are padding whose outputs are not
     written (a multiple of 8 no larger than ``h_q``; anything else means all heads).
 
+    ``indices`` int32 [b, s_q, topk]: token-level sparse decoding (upstream FlashMLA
+    documentation, "Sparse Attention (indices tensor)"): query token (i, j) attends the
+    cache rows ``indices[i, j, k]`` (page * 64 + offset; -1 or any row outside the cache is
+    invalid) instead of a block-table prefix; ``block_table``, ``cache_seqlens`` and
+    ``causal`` are not used, the cache must be FP8 with scale, and the metadata comes from
+    ``get_mla_metadata(..., h_q=h_q, topk=topk)``.
+
     ``q`` [b, s_q, h_q, d_qk] and ``kvcache`` [num_blocks, 64, h_kv, d_qk] are bf16 or
     fp16; ``block_table`` [b, max_blocks] and ``cache_seqlens`` [b] are int32.  With
     ``q`` on the CPU the inputs are copied to the current CUDA device (non-blocking
@@ -209,12 +255,12 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
     if host:
         dev = torch.device("cuda", torch.cuda.current_device())
         nb = q.is_pinned()
-        q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits = (
-            t.to(dev, non_blocking=nb) for t in
-            (q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits))
+        q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits, indices = (
+            None if t is None else t.to(dev, non_blocking=nb) for t in
+            (q, kvcache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits, indices))
     call = DecodeCall(q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata, num_splits,
                       causal=causal, softmax_scale=softmax_scale, workspace=workspace, out=out, lse=lse,
-                      active_heads=active_heads, is_fp8_kvcache=is_fp8_kvcache)
+                      active_heads=active_heads, is_fp8_kvcache=is_fp8_kvcache, indices=indices)
     out, lse = call.run()
     if host:
         return out.cpu(), lse.cpu()

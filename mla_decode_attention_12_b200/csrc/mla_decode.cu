@@ -76,9 +76,9 @@ constexpr int kRawVBytes = 2 * 4096 + 512;     // the peer's 32 rows: this CTA's
 // Registers per thread in the FP8 kernel: the launch holds 65536 / 512 = 128 each; the loader /
 // MMA warpgroup and the two converter warpgroups give theirs up to the softmax warpgroup.
 constexpr uint32_t kRegsLaunchFp8 = 128;
-constexpr uint32_t kRegsLoadersFp8 = 72;
-constexpr uint32_t kRegsConvFp8 = 96;
-constexpr uint32_t kRegsSoftmaxFp8 = 248;
+constexpr uint32_t kRegsLoadersFp8 = 104;
+constexpr uint32_t kRegsConvFp8 = 128;
+constexpr uint32_t kRegsSoftmaxFp8 = 152;
 static_assert(128 * (kRegsLoadersFp8 + kRegsSoftmaxFp8 + 2 * kRegsConvFp8) <= kThreadsFp8 * kRegsLaunchFp8,
               "register split exceeds the launch's registers");
 constexpr int kKWarp = 4;
@@ -172,7 +172,9 @@ struct Ring {
 };
 constexpr int kOffTmemSlot = kBarCount * 8;  // uint32 written by tcgen05.alloc
 constexpr int kOffAbort = kOffTmemSlot + 4;  // int abort flag
-static_assert(kOffAbort + 4 <= Layout<true>::kBarBytes, "barrier area too small");
+constexpr int kOffMaskK = kOffAbort + 4;     // sparse decode: validity bits of the raw K stages' 32 rows
+constexpr int kOffMaskV = kOffMaskK + 4 * 3; // ... and of the raw V stages' 32 (peer) rows
+static_assert(kOffMaskV + 4 * 2 <= Layout<true>::kBarBytes, "barrier area too small");
 static_assert(2 * Layout<true>::kPBytes >= 4 * 4096 && 2 * Layout<false>::kPBytes >= 4 * 4096,
               "epilogue staging (4 KB per softmax warp) must fit in the P buffers");
 static_assert(kTmemQ + 8 * 4 * kQTmemBoxes == kTmemCols, "tensor memory plan");
@@ -193,7 +195,8 @@ static_assert(Layout<true>::kOffQ % 1024 == 0 && Layout<true>::kOffK % 1024 == 0
 
 struct DecodeParams {
     const int32_t* block_table;
-    const int32_t* seqlens;
+    const int32_t* seqlens;   // [batch]; null for the sparse decode (every request has topk entries)
+    const int32_t* indices;   // sparse decode: [batch][topk] flat cache rows (page * 64 + offset), -1 invalid
     const int32_t* md;
     const int32_t* num_splits;
     const void* q;
@@ -208,6 +211,8 @@ struct DecodeParams {
     int batch, s_q, h_q, rows, groups, max_blocks, num_blocks, causal, box_rows;
     int active_heads;  // heads >= active_heads are padding: not written, not combined
     int o_align32;     // o is 32-byte aligned: 32-byte stores
+    int topk;          // sparse decode: entries per request
+    int cache_rows;    // num_blocks * 64: a sparse entry outside [0, cache_rows) is invalid
     float scale_log2;
     int dtype, d_qk, num_parts;  // host-side dispatch only
 };
@@ -316,15 +321,22 @@ struct Sync {
     }
 };
 
+// Work length of request b: its cached tokens, or, for the sparse decode, its entries.
+__device__ __forceinline__ int request_len(const int32_t* seqlens, int const_len, int b)
+{
+    return seqlens ? seqlens[b] : const_len;
+}
+
 // Iterates the chunks (vb, blk_lo, blk_hi) of one scheduler partition.
 struct ChunkIter {
     int vb, blk, end_vb, end_blk, groups;
     const int32_t* seqlens;
+    int const_len;  // the length of every request when seqlens is null
 
     __device__ bool next(int& out_vb, int& lo, int& hi)
     {
         if (!(vb < end_vb || (vb == end_vb && blk < end_blk))) return false;
-        const int n = pages_of(seqlens[vb / groups]);
+        const int n = pages_of(request_len(seqlens, const_len, vb / groups));
         out_vb = vb;
         lo = blk;
         hi = (vb == end_vb) ? end_blk : n;
@@ -368,12 +380,13 @@ __device__ __forceinline__ int page_of(const DecodeParams& p, const int32_t* tab
 //   O   columns [0, 256):  d_v chunk i (256 wide) at [128 i, 128 i + 128)
 //   S   columns [256, 288) and [288, 320): two page buffers
 // Thread t of the softmax warps owns row t % 64 and token / d_v half t / 64.
-template <bool kRope, bool kFp16, bool kPadHeads, bool kFp8 = false>
+template <bool kRope, bool kFp16, bool kPadHeads, bool kFp8 = false, bool kSparse = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
     mla_splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const DecodeParams p)
 {
     static_assert(!kFp8 || (kRope && !kFp16), "the FP8 cache has d_qk = 576 and bfloat16 queries");
+    static_assert(!kSparse || kFp8, "the sparse decode reads an FP8 cache");
     using L = Layout<kRope, kFp8>;
     constexpr int kNumThreads = kFp8 ? kThreadsFp8 : kThreads;
     extern __shared__ uint8_t smem_raw[];
@@ -385,6 +398,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
     const uint32_t s_p = s_base + L::kOffP;
     const uint32_t s_bar = s_base + L::kOffBar;
     float* red = reinterpret_cast<float*>(smem + L::kOffRed);
+    volatile uint32_t* mask_k = reinterpret_cast<volatile uint32_t*>(smem + L::kOffBar + kOffMaskK);
+    volatile uint32_t* mask_v = reinterpret_cast<volatile uint32_t*>(smem + L::kOffBar + kOffMaskV);
     [[maybe_unused]] Timeline tl;
 #ifdef MLA_TIMELINE
     const uint64_t tl_start = global_timer_ns();
@@ -470,7 +485,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
 
     Sync sync{s_bar + kOffAbort, map_to_cta(s_bar + kOffAbort, cta ^ 1u), p.status};
     const int32_t* md = p.md + part * kMdInts;
-    ChunkIter chunks{md[0], md[1], md[2], md[3], p.groups, p.seqlens};
+    ChunkIter chunks{md[0], md[1], md[2], md[3], p.groups, p.seqlens, p.topk};
     const int begin_vb = md[0];
     const int begin_split = md[4];
 
@@ -531,12 +546,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         Ring<L::kRawKStages> rk;
         Ring<L::kRawVStages> rv;
         uint32_t gv = 0;              // pages whose V stage has been filled
-        int prev_valid = -1;          // valid rows of the page waiting for its V stage (-1: none)
+        bool pending = false;         // a page waits for its V stage
+        uint32_t own_live = 0, peer_live = 0;  // its rows that are visible: bit i = own / peer row i
         uint32_t prev_kstage = 0;
         bool ok = true;
-        // V stage of the previous page: own rows from its K stage, the peer's from raw slices.
+        // V stage of the previous page: own rows from its K stage, the peer's from raw slices;
+        // rows not visible (past the sequence end, or invalid sparse entries) are zero.
         auto fill_v = [&]() -> bool {
             if (!wwait(bar(kBarRawVFull + rv.stage), rv.phase)) return false;
+            if constexpr (kSparse) peer_live = mask_v[rv.stage];
             if (!wwait(bar(kBarVEmpty), (gv & 1) ^ 1)) return false;
             uint8_t* vst = smem + L::kOffV;
             const uint8_t* kst = smem + L::kOffK + prev_kstage * L::kKBytes;
@@ -561,7 +579,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             }
             {
                 const int tok = own0 + lane;
-                const bool live = tok < prev_valid;
+                const bool live = (own_live >> lane) & 1u;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int jv = 2 * ch + (i >> 1);
@@ -574,9 +592,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 const int c0 = 2 * (chunk8 & 3);
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {
-                    const int tok = peer0 + 8 * cq + 4 * m + (lane >> 3);
+                    const int t_peer = 8 * cq + 4 * m + (lane >> 3), tok = peer0 + t_peer;
                     uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-                    if (tok < prev_valid) dequant16(peer[m], ps[m], lo, hi);
+                    if ((peer_live >> t_peer) & 1u) dequant16(peer[m], ps[m], lo, hi);
                     uint8_t* row = vst + jv * 8192 + tok * 128;
                     *reinterpret_cast<uint4*>(row + ((c0 ^ (tok & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (tok & 7)) << 4)) = hi;
@@ -587,16 +605,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             publish(v_full_lead);
             rv.advance();
             ++gv;
-            prev_valid = -1;
+            pending = false;
             return true;
         };
         int vb, lo, hi;
         while (ok && chunks.next(vb, lo, hi)) {
             if (hi <= lo) continue;
-            const int Lb = p.seqlens[vb / p.groups];
+            const int Lb = request_len(p.seqlens, p.topk, vb / p.groups);
             for (int blk = lo; blk < hi && ok; ++blk) {
                 // ---- K(g): this CTA's 32 rows
                 if (!(ok = wwait(bar(kBarRawKFull + rk.stage), rk.phase))) break;
+                // visible rows of page g (read before the raw stage is handed back)
+                uint32_t own_g, peer_g = 0;
+                if constexpr (kSparse) {
+                    own_g = mask_k[rk.stage];
+                } else {
+                    const int valid = min(kPage, Lb - kPage * blk);  // rows [0, valid) of the page
+                    auto half_bits = [&](int first) {
+                        const int c = min(max(valid - first, 0), 32);
+                        return c >= 32 ? 0xffffffffu : ((1u << c) - 1u);
+                    };
+                    own_g = half_bits(32 * static_cast<int>(cta));
+                    peer_g = half_bits(32 - 32 * static_cast<int>(cta));
+                }
                 if (!(ok = wwait(bar(kBarKEmpty + kring.stage), kring.phase ^ 1))) break;
                 {
                     const uint8_t* rrow = smem + L::kOffRawK + rk.stage * kRawKBytes + lane * kFp8Row;
@@ -622,13 +653,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 publish(k_full_lead[kring.stage]);
                 rk.advance();
                 // ---- V(g - 1)
-                if (prev_valid >= 0 && !(ok = fill_v())) break;
-                prev_valid = min(kPage, Lb - kPage * blk);
+                if (pending && !(ok = fill_v())) break;
+                pending = true;
+                own_live = own_g;
+                peer_live = peer_g;  // (the sparse decode reads it with the raw V stage)
                 prev_kstage = kring.stage;
                 kring.advance();
             }
         }
-        if (ok && prev_valid >= 0) ok = fill_v();
+        if (ok && pending) ok = fill_v();
     } else if (warp >= 4) {
         // Warpgroup 1 (Q / K / V loaders and the MMA issuer): one thread issues; few registers.
         if constexpr (kFp8) set_max_registers<kRegsLaunchFp8, kRegsLoadersFp8>();  // before the role split: one
@@ -672,7 +705,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             }
         } else if (warp == kKWarp) {
             // ============================ K producer ============================
-            if constexpr (kFp8) {
+            if constexpr (kSparse) {
+                // Sparse decode: row i of this CTA's half of "page" blk is entry 64 blk + 32 cta + i
+                // of the request's list.  Lane i bulk-copies its row (656 bytes as stored) when
+                // the entry is valid; lane 0 records the half's validity bits with the stage and
+                // registers the bytes.  Entries are read one page ahead.
+                Ring<L::kRawKStages> ring;
+                int vb, lo, hi;
+                bool ok = true;
+                const uint8_t* kv = static_cast<const uint8_t*>(p.kvcache);
+                auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
+                while (ok && chunks.next(vb, lo, hi)) {
+                    if (hi <= lo) continue;
+                    const int32_t* ent = p.indices + static_cast<size_t>(vb / p.groups) * p.topk;
+                    auto entry = [&](int blk) {
+                        const int e = kPage * blk + 32 * static_cast<int>(cta) + lane;
+                        return e < p.topk ? __ldg(ent + e) : -1;
+                    };
+                    int idx = entry(lo);
+                    for (int blk = lo; blk < hi; ++blk, ring.advance()) {
+                        const int idx_next = blk + 1 < hi ? entry(blk + 1) : -1;
+                        const uint32_t st = ring.stage;
+                        if (!(ok = wwait(bar(kBarRawKEmpty + st), ring.phase ^ 1))) break;
+                        const bool valid = idx >= 0 && idx < p.cache_rows;
+                        const uint32_t mask = __ballot_sync(0xffffffffu, valid);
+                        if (lane == 0) {
+                            mask_k[st] = mask;
+                            mbar_arrive_expect_tx(bar(kBarRawKFull + st), __popc(mask) * kFp8Row);
+                        }
+                        __syncwarp();
+                        if (valid)
+                            bulk_load(s_base + L::kOffRawK + st * kRawKBytes + lane * kFp8Row,
+                                      kv + static_cast<size_t>(idx) * kFp8Row, kFp8Row, bar(kBarRawKFull + st));
+                        idx = idx_next;
+                    }
+                }
+                if (!ok && lane == 0) {
+                    const uint64_t t0 = global_timer_ns();  // let issued loads land (see the V producer)
+                    while (global_timer_ns() - t0 < 50000000ull) {
+                    }
+                }
+            } else if constexpr (kFp8) {
                 // FP8 cache: this CTA's 32 rows of each page as stored (one bulk copy), for the
                 // converters.
                 if (lane == 0) {
@@ -728,7 +801,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 }
             }
         } else if (warp == kVWarp) {
-            if constexpr (kFp8) {
+            if constexpr (kSparse) {
+                // ======================== V producer (sparse decode) ========================
+                // The peer's 32 rows of "page" blk (entries 64 blk + 32 (1 - cta) + i): lane i copies
+                // this CTA's two 128-byte latent slices (its V columns) and the 16 bytes of scales
+                // of its row when the entry is valid, in the layout the TMA boxes give the dense
+                // decode; lane 0 records the validity bits with the stage.
+                Ring<L::kRawVStages> ring;
+                int vb, lo, hi;
+                bool ok = true;
+                const uint8_t* kv = static_cast<const uint8_t*>(p.kvcache);
+                auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
+                while (ok && chunks.next(vb, lo, hi)) {
+                    if (hi <= lo) continue;
+                    const int32_t* ent = p.indices + static_cast<size_t>(vb / p.groups) * p.topk;
+                    auto entry = [&](int blk) {
+                        const int e = kPage * blk + 32 * (1 - static_cast<int>(cta)) + lane;
+                        return e < p.topk ? __ldg(ent + e) : -1;
+                    };
+                    int idx = entry(lo);
+                    for (int blk = lo; blk < hi; ++blk, ring.advance()) {
+                        const int idx_next = blk + 1 < hi ? entry(blk + 1) : -1;
+                        const uint32_t st = ring.stage;
+                        if (!(ok = wwait(bar(kBarRawVEmpty + st), ring.phase ^ 1))) break;
+                        const bool valid = idx >= 0 && idx < p.cache_rows;
+                        const uint32_t mask = __ballot_sync(0xffffffffu, valid);
+                        if (lane == 0) {
+                            mask_v[st] = mask;
+                            mbar_arrive_expect_tx(bar(kBarRawVFull + st), __popc(mask) * (2 * 128 + 16));
+                        }
+                        __syncwarp();
+                        if (valid) {
+                            const uint8_t* row = kv + static_cast<size_t>(idx) * kFp8Row;
+                            const uint32_t dst = s_base + L::kOffRawV + st * kRawVBytes;
+                            bulk_load(dst + lane * 128, row + 128 * cta, 128, bar(kBarRawVFull + st));
+                            bulk_load(dst + 4096 + lane * 128, row + 256 + 128 * cta, 128, bar(kBarRawVFull + st));
+                            bulk_load(dst + 8192 + lane * 16, row + 512, 16, bar(kBarRawVFull + st));
+                        }
+                        idx = idx_next;
+                    }
+                }
+                if (!ok && lane == 0) {
+                    const uint64_t t0 = global_timer_ns();  // let issued loads land (see below)
+                    while (global_timer_ns() - t0 < 50000000ull) {
+                    }
+                }
+            } else if constexpr (kFp8) {
                 // ============================ V producer (FP8 cache) ============================
                 // The peer's 32 rows of each page: this CTA's two 128-value latent slices (its V
                 // columns) and the rows' scales, by TMA (tm_k: 128-byte boxes, tm_v: 16-byte boxes).
@@ -776,7 +894,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 while (ok && chunks.next(vb, lo, hi)) {
                     if (hi <= lo) continue;
                     const int b = vb / p.groups;
-                    const int Lb = p.seqlens[b];
+                    const int Lb = request_len(p.seqlens, p.topk, b);
                     const int tail = Lb % kPage;
                     const int last_page = pages_of(Lb) - 1;
                     const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
@@ -999,7 +1117,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         bool have = chunks.next(vb, lo, hi);
         while (ok && have) {
             const int b = vb / p.groups, rg = vb % p.groups;
-            const int Lb = p.seqlens[b];
+            const int Lb = request_len(p.seqlens, p.topk, b);
             const int row = rg * kRowsPerGroup + 64 * static_cast<int>(cta) + r;
             const bool row_valid = row < p.rows;
             const int s_tok = row / p.h_q;
@@ -1016,6 +1134,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             // that loading it at the transition hits L2 (earlier, the KV stream through L2
             // would evict it again).
             const int j_prefetch = max(0, n - kQPrefetchPages);
+            // Sparse decode: a page's visible columns are its valid entries.  Lane i of this warp
+            // reads entry 64 page + 32 h + i (one page ahead) and a ballot gives the warp's 32 bits.
+            const int32_t* ent = kSparse ? p.indices + static_cast<size_t>(b) * p.topk : nullptr;
+            auto entry = [&](int blk) {
+                const int e = kPage * blk + 32 * h + lane;
+                return e < p.topk ? __ldg(ent + e) : -1;
+            };
+            int sp_idx = (kSparse && n > 0) ? entry(lo) : -1;
 
             for (int j = 0; j < n; ++j) {
                 if (j == j_prefetch) {
@@ -1037,17 +1163,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 // (the sequence's last page, the causal diagonal) needs the mask.
                 float x[32];
                 {
+                    uint32_t vis = 0xffffffffu;  // visible columns (bit c: column 32 h + c)
+                    if constexpr (kSparse) {
+                        const int sp_next = (j + 1 < n) ? entry(lo + j + 1) : -1;
+                        vis = __ballot_sync(0xffffffffu, sp_idx >= 0 && sp_idx < p.cache_rows);
+                        sp_idx = sp_next;
+                    }
                     uint32_t a[32];
                     tmem_ld32(tmem + kTmemS + 32 * sb + lane_base, a);
                     tmem_wait_ld();
                     reg_fence(a);
-                    const int lim = n_vis - (lo + j) * kPage - 32 * h;  // columns >= lim are not visible
-                    if (__all_sync(0xffffffffu, lim >= 32)) {
+                    if constexpr (!kSparse) {
+                        const int lim = n_vis - (lo + j) * kPage - 32 * h;  // columns >= lim are not visible
+                        vis = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+                    }
+                    if (__all_sync(0xffffffffu, vis == 0xffffffffu)) {
 #pragma unroll
                         for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(a[c]);
                     } else {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) x[c] = (c < lim) ? __uint_as_float(a[c]) : -INFINITY;
+                        for (int c = 0; c < 32; ++c) x[c] = ((vis >> c) & 1u) ? __uint_as_float(a[c]) : -INFINITY;
                     }
                 }
                 float mx;
@@ -1413,8 +1548,9 @@ __device__ void block_exclusive_scan(T* data, int n, T* warp_tot, T& total)
 // pages [nv] int32, extra-split counts [nv] int32, begins [num_parts] int32 x 2.
 constexpr int kMetaThreads = 256;
 
-__global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_t* seqlens, int batch, int groups,
-                                                                    int num_parts, int32_t* md, int32_t* num_splits)
+__global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_t* seqlens, int const_len, int batch,
+                                                                    int groups, int num_parts, int32_t* md,
+                                                                    int32_t* num_splits)
 {
     extern __shared__ __align__(16) uint8_t meta_smem[];
     grid_dependency_wait();
@@ -1427,7 +1563,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
     int32_t* extra = pages + nv;
     int32_t* begins = extra + nv;  // [num_parts][2]
     for (int v = threadIdx.x; v < nv; v += blockDim.x) {
-        pages[v] = pages_of(seqlens[v / groups]);
+        pages[v] = pages_of(seqlens ? seqlens[v / groups] : const_len);
         C[v] = pages[v] + kFixedCost;
         extra[v] = 0;
     }
@@ -1581,10 +1717,10 @@ struct PerDeviceOnce {
     }
 };
 
-template <bool kRope, bool kFp16, bool kPadHeads, bool kFp8>
+template <bool kRope, bool kFp16, bool kPadHeads, bool kFp8, bool kSparse>
 static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorMap* maps, const DecodeParams& prm)
 {
-    auto kern = mla_splitkv_kernel<kRope, kFp16, kPadHeads, kFp8>;
+    auto kern = mla_splitkv_kernel<kRope, kFp16, kPadHeads, kFp8, kSparse>;
     const int smem = Layout<kRope, kFp8>::kSmemBytes;
     static PerDeviceOnce configured;  // the attribute is per device
     cudaError_t e = configured.run([&]() -> cudaError_t {
@@ -1608,11 +1744,38 @@ static cudaError_t launch_splitkv(int grid, cudaStream_t stream, const CUtensorM
 }
 
 // The kernel variant with padding-head logic runs only when some heads are padding.
-template <bool kRope, bool kFp16, bool kFp8 = false>
+template <bool kRope, bool kFp16, bool kFp8 = false, bool kSparse = false>
 static cudaError_t launch_splitkv_heads(int grid, cudaStream_t st, const CUtensorMap* maps, const DecodeParams& prm)
 {
-    return prm.active_heads < prm.h_q ? launch_splitkv<kRope, kFp16, true, kFp8>(grid, st, maps, prm)
-                                      : launch_splitkv<kRope, kFp16, false, kFp8>(grid, st, maps, prm);
+    return prm.active_heads < prm.h_q ? launch_splitkv<kRope, kFp16, true, kFp8, kSparse>(grid, st, maps, prm)
+                                      : launch_splitkv<kRope, kFp16, false, kFp8, kSparse>(grid, st, maps, prm);
+}
+
+// The metadata kernel on `stream`: lengths from `seqlens`, or `const_len` for every request
+// when `seqlens` is null (the sparse decode).
+static mla_status launch_metadata(const int32_t* seqlens, int const_len, int batch, int heads_per_kv, int h_kv,
+                                  int num_parts, int32_t* tile_md, int32_t* num_splits, void* stream)
+{
+    if (batch < 0 || heads_per_kv <= 0 || h_kv <= 0 || num_parts <= 0 || !tile_md || !num_splits)
+        return MLA_ERR_INVALID_ARG;
+    if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
+    const int nv = batch * row_groups(heads_per_kv);
+    const size_t smem = metadata_smem_bytes(nv, num_parts);
+    if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;  // the schedule is built in one CTA's shared memory
+    if (smem > 48 * 1024) {
+        static PerDeviceOnce configured;
+        if (configured.run([] {
+                return cudaFuncSetAttribute(mla_metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            200 * 1024);
+            }) != cudaSuccess)
+            return MLA_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    programmatic_launch(cfg, attr, dim3(1), dim3(kMetaThreads), smem, static_cast<cudaStream_t>(stream));
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, mla_metadata_kernel, seqlens, const_len, batch,
+                                             row_groups(heads_per_kv), num_parts, tile_md, num_splits);
+    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // namespace mla
@@ -1677,27 +1840,15 @@ mla_status mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int he
 mla_status mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv, int num_parts,
                             int32_t* tile_md, int32_t* num_splits, void* stream)
 {
-    if (batch < 0 || heads_per_kv <= 0 || h_kv <= 0 || num_parts <= 0 || !tile_md || !num_splits ||
-        (batch > 0 && !cache_seqlens))
-        return MLA_ERR_INVALID_ARG;
-    if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
-    const int nv = batch * row_groups(heads_per_kv);
-    const size_t smem = metadata_smem_bytes(nv, num_parts);
-    if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;  // the schedule is built in one CTA's shared memory
-    if (smem > 48 * 1024) {
-        static PerDeviceOnce configured;
-        if (configured.run([] {
-                return cudaFuncSetAttribute(mla_metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            200 * 1024);
-            }) != cudaSuccess)
-            return MLA_ERR_CUDA;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    programmatic_launch(cfg, attr, dim3(1), dim3(kMetaThreads), smem, static_cast<cudaStream_t>(stream));
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, mla_metadata_kernel, cache_seqlens, batch, row_groups(heads_per_kv),
-                                             num_parts, tile_md, num_splits);
-    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    if (batch > 0 && !cache_seqlens) return MLA_ERR_INVALID_ARG;
+    return launch_metadata(cache_seqlens, 0, batch, heads_per_kv, h_kv, num_parts, tile_md, num_splits, stream);
+}
+
+mla_status mla_get_metadata_sparse(int num_tokens, int topk, int h_q, int h_kv, int num_parts, int32_t* tile_md,
+                                   int32_t* num_splits, void* stream)
+{
+    if (topk < 0 || h_kv <= 0 || h_q % h_kv) return MLA_ERR_INVALID_ARG;
+    return launch_metadata(nullptr, topk, num_tokens, h_q / h_kv, h_kv, num_parts, tile_md, num_splits, stream);
 }
 
 size_t mla_decode_workspace_zero_bytes(int batch, int s_q, int h_q, int h_kv)
@@ -1724,16 +1875,21 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
                                  int max_blocks_per_seq, const int32_t* cache_seqlens, int dv, int dtype,
                                  const int32_t* tile_md, int num_parts, const int32_t* num_splits, int causal,
                                  float softmax_scale, int active_heads, void* o, float* lse, void* workspace,
-                                 size_t workspace_bytes, DecodeParams& prm, CUtensorMap* maps)
+                                 size_t workspace_bytes, const int32_t* indices, int topk, DecodeParams& prm,
+                                 CUtensorMap* maps)
 {
+    // indices != null: the sparse decode, with batch = requests x query tokens and s_q = 1;
+    // no block table, no sequence lengths, no causal mask
+    const bool sparse = indices != nullptr;
     if (batch < 0 || s_q <= 0 || h_q <= 0 || h_kv <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
-        num_parts <= 0 || (causal != 0 && causal != 1))
+        num_parts <= 0 || (causal != 0 && causal != 1) || topk < 0)
         return MLA_ERR_INVALID_ARG;
     if (dtype != MLA_BF16 && dtype != MLA_FP16 && dtype != MLA_BF16_FP8KV) return MLA_ERR_INVALID_ARG;
     if (page_size != kPage || h_kv != 1 || (d_qk != 576 && d_qk != 512) || dv != kDv) return MLA_ERR_UNSUPPORTED;
     if (dtype == MLA_BF16_FP8KV && d_qk != 576) return MLA_ERR_UNSUPPORTED;  // the FP8 row carries 64 RoPE values
-    if (batch > 0 && (!q || !kvcache || !block_table || !cache_seqlens || !tile_md || !num_splits || !o || !lse ||
-                      !workspace))
+    if (sparse && dtype != MLA_BF16_FP8KV) return MLA_ERR_UNSUPPORTED;        // the sparse decode reads an FP8 cache
+    if (batch > 0 && (!q || !kvcache || (!sparse && (!block_table || !cache_seqlens)) || !tile_md || !num_splits ||
+                      !o || !lse || !workspace))
         return MLA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kvcache) & 15) ||
         (reinterpret_cast<uintptr_t>(o) & 15) || (reinterpret_cast<uintptr_t>(workspace) & 255))
@@ -1746,8 +1902,11 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     if (static_cast<long long>(num_blocks) * kPage >= (1ll << 31)) return MLA_ERR_UNSUPPORTED;
     if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt(static_cast<float>(d_qk));
     prm = DecodeParams{};
-    prm.block_table = block_table;
-    prm.seqlens = cache_seqlens;
+    prm.block_table = sparse ? nullptr : block_table;
+    prm.seqlens = sparse ? nullptr : cache_seqlens;
+    prm.indices = indices;
+    prm.topk = topk;
+    prm.cache_rows = num_blocks * kPage;
     prm.md = tile_md;
     prm.num_splits = num_splits;
     prm.q = q;
@@ -1761,7 +1920,7 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     prm.groups = groups;
     prm.max_blocks = max_blocks_per_seq;
     prm.num_blocks = num_blocks;
-    prm.causal = causal;
+    prm.causal = sparse ? 0 : causal;
     prm.box_rows = rows < 64 ? rows : 64;  // query rows per CTA of the pair
     prm.scale_log2 = softmax_scale * 1.4426950408889634f;
     prm.active_heads = effective_active_heads(active_heads, h_q);
@@ -1800,7 +1959,9 @@ static mla_status launch_splitkv_stage(const DecodeParams& prm, const CUtensorMa
 {
     const int grid = 2 * prm.num_parts;
     cudaError_t e;
-    if (prm.dtype == MLA_BF16_FP8KV)
+    if (prm.indices)
+        e = launch_splitkv_heads<true, false, true, true>(grid, st, maps, prm);
+    else if (prm.dtype == MLA_BF16_FP8KV)
         e = launch_splitkv_heads<true, false, true>(grid, st, maps, prm);
     else if (prm.d_qk == 576)
         e = prm.dtype == MLA_FP16 ? launch_splitkv_heads<true, true>(grid, st, maps, prm)
@@ -1835,7 +1996,7 @@ static mla_status launch_combine_stage(const DecodeParams& prm, cudaStream_t st)
 #define MLA_DECODE_ARGS                                                                                          \
     q, batch, s_q, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, block_table, max_blocks_per_seq,            \
         cache_seqlens, dv, dtype, tile_md, num_parts, num_splits, causal, softmax_scale, active_heads, o, lse,   \
-        workspace, workspace_bytes
+        workspace, workspace_bytes, nullptr, 0
 
 mla_status mla_decode_with_kvcache(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache,
                                    int num_blocks, int page_size, int h_kv, const int32_t* block_table,
@@ -1905,6 +2066,57 @@ MLA_API mla_status mla_timeline_read(uint32_t* host, size_t words)
     return cudaMemcpyFromSymbol(host, g_timeline, sizeof(g_timeline)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 #endif
+
+}  // extern "C"
+
+// The sparse decode: the split-KV stage, then (unless `only_splitkv`) the combine stage.
+static mla_status decode_sparse(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache,
+                                int num_blocks, int page_size, int h_kv, const int32_t* indices, int topk, int dv,
+                                int dtype, const int32_t* tile_md, int num_parts, const int32_t* num_splits,
+                                float softmax_scale, int active_heads, void* o, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream, bool only_splitkv)
+{
+    if (batch < 0 || s_q <= 0 || topk < 0) return MLA_ERR_INVALID_ARG;
+    if (batch > 0 && !indices) return MLA_ERR_INVALID_ARG;
+    if (static_cast<long long>(batch) * s_q > (1ll << 30)) return MLA_ERR_UNSUPPORTED;
+    DecodeParams prm;
+    CUtensorMap maps[kNumMaps];
+    // every query token is a request of its own: batch * s_q requests of one token
+    const int tokens = batch * s_q;
+    const int32_t* one = indices ? indices : reinterpret_cast<const int32_t*>(&prm);  // not read when batch == 0
+    mla_status s = prepare_decode(q, tokens, 1, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, nullptr, 1,
+                                  nullptr, dv, dtype, tile_md, num_parts, num_splits, 0, softmax_scale, active_heads,
+                                  o, lse, workspace, workspace_bytes, one, topk, prm, maps);
+    if (s != MLA_OK || tokens == 0) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = launch_splitkv_stage(prm, maps, st);
+    if (s != MLA_OK || only_splitkv) return s;
+    return launch_combine_stage(prm, st);
+}
+
+extern "C" {
+
+mla_status mla_decode_sparse(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache, int num_blocks,
+                             int page_size, int h_kv, const int32_t* indices, int topk, int dv, int dtype,
+                             const int32_t* tile_md, int num_parts, const int32_t* num_splits, float softmax_scale,
+                             int active_heads, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                             void* stream)
+{
+    return decode_sparse(q, batch, s_q, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, indices, topk, dv, dtype,
+                         tile_md, num_parts, num_splits, softmax_scale, active_heads, o, lse, workspace,
+                         workspace_bytes, stream, false);
+}
+
+mla_status mla_decode_sparse_splitkv(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache,
+                                     int num_blocks, int page_size, int h_kv, const int32_t* indices, int topk,
+                                     int dv, int dtype, const int32_t* tile_md, int num_parts,
+                                     const int32_t* num_splits, float softmax_scale, int active_heads, void* o,
+                                     float* lse, void* workspace, size_t workspace_bytes, void* stream)
+{
+    return decode_sparse(q, batch, s_q, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, indices, topk, dv, dtype,
+                         tile_md, num_parts, num_splits, softmax_scale, active_heads, o, lse, workspace,
+                         workspace_bytes, stream, true);
+}
 
 mla_status mla_read_device_status(void* workspace, int clear, int* device_status, void* stream)
 {

@@ -80,8 +80,16 @@ class Problem:
     def num_blocks(self) -> int:
         return self.kvcache.shape[0]
 
+    def valid_entries(self) -> np.ndarray:
+        """Sparse problems: [b, s_q, topk] bool, the entries inside the cache."""
+        rows = self.num_blocks * self.page_size
+        return (self.indices >= 0) & (self.indices < rows)
+
     def visible(self) -> np.ndarray:
-        """[b, s_q] number of cached tokens each query token attends (causal: bottom-right)."""
+        """[b, s_q] number of cached tokens each query token attends (causal: bottom-right;
+        sparse: its valid entries)."""
+        if self.indices is not None:
+            return self.valid_entries().sum(axis=2).astype(np.int64)
         L = self.cache_seqlens.astype(np.int64)[:, None]
         if not self.causal:
             return np.broadcast_to(L, (self.batch, self.s_q)).copy()
@@ -97,13 +105,17 @@ class Problem:
         return FP8_ROW_BYTES if self.fp8_kv else self.d_qk * 2
 
     def kv_bytes(self) -> int:
-        """Cached rows read once: sum_b L_b * h_kv * row bytes."""
+        """Cached rows read once: sum_b L_b * h_kv * row bytes (sparse: every query token's
+        valid entries, each read once for that token)."""
+        if self.indices is not None:
+            return int(self.valid_entries().sum()) * self.h_kv * self.kv_row_bytes()
         return int(self.cache_seqlens.astype(np.int64).sum()) * self.h_kv * self.kv_row_bytes()
 
     def io_bytes(self) -> int:
-        """Algorithmic bytes: KV once + Q + O (16-bit) + LSE (fp32)."""
+        """Algorithmic bytes: KV once + Q + O (16-bit) + LSE (fp32) (+ the entry lists)."""
         rows = self.batch * self.s_q * self.h_q
-        return self.kv_bytes() + rows * (self.d_qk * 2 + self.dv * 2 + 4)
+        extra = 0 if self.indices is None else self.indices.size * 4
+        return self.kv_bytes() + rows * (self.d_qk * 2 + self.dv * 2 + 4) + extra
 
 
 def _round_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -260,6 +272,8 @@ def make_sparse_problem(seqlens, topk: int, *, s_q: int = 1, invalid_frac: float
 # ----------------------------------------------------------------------------
 
 WORKLOADS = ("tiny", "compute", "spec_padded", "long_split", "fp16_norope", "fp8_compute")
+# Token-level sparse decode over an FP8 cache (its own path: indices instead of a block table).
+SPARSE_WORKLOADS = ("sparse_fp8",)
 
 
 def workload_seqlens(name: str, rng: np.random.Generator) -> np.ndarray:
@@ -267,6 +281,8 @@ def workload_seqlens(name: str, rng: np.random.Generator) -> np.ndarray:
         return np.array([256, 193], np.int32)
     if name in ("compute", "fp8_compute"):
         return rng.integers(1024, 8192, size=64, endpoint=True).astype(np.int32)
+    if name == "sparse_fp8":
+        return rng.integers(8192, 16384, size=64, endpoint=True).astype(np.int32)
     if name == "spec_padded":
         return rng.integers(4096 - 512, 4096 + 512, size=128, endpoint=True).astype(np.int32)
     if name == "long_split":
@@ -283,7 +299,7 @@ def make_workload(name: str, *, poison: bool = False, seqlens=None) -> Problem:
     ``seqlens`` overrides the sequence lengths (for scaled-down parity cases with
     the same head / dtype / mask structure).
     """
-    k = WORKLOADS.index(name) + 1
+    k = (WORKLOADS + SPARSE_WORKLOADS).index(name) + 1
     seed = 1000 + k
     rng = np.random.Generator(np.random.PCG64(seed + 7919))
     L = workload_seqlens(name, rng) if seqlens is None else np.asarray(seqlens, np.int32)
@@ -301,4 +317,6 @@ def make_workload(name: str, *, poison: bool = False, seqlens=None) -> Problem:
                             **common)
     if name == "fp8_compute":
         return make_problem(L, s_q=1, h_q=128, d_qk=576, fp8_kv=True, **common)
+    if name == "sparse_fp8":
+        return make_sparse_problem(L, 2048, s_q=2, h_q=128, fp8_kv=True, **common)
     raise KeyError(name)

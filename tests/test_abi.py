@@ -150,3 +150,31 @@ def test_binding_rejects_mismatched_cache_formats(case):
     ns = torch.zeros(2, dtype=torch.int32)
     with pytest.raises(ValueError):
         api.DecodeCall(q, kv, bt, sl, 512, md, ns, is_fp8_kvcache=fp8)
+
+
+def _sparse(lib, **over):
+    fake = 1 << 20
+    args = dict(q=fake, batch=2, s_q=1, h_q=16, d_qk=576, kvcache=fake, num_blocks=8, page_size=64, h_kv=1,
+                indices=fake, topk=128, dv=512, dtype=2, md=fake, num_parts=74, num_splits=fake, scale=0.0,
+                active_heads=0, o=fake, lse=fake, ws=fake, ws_bytes=1 << 40, stream=None)
+    args.update(over)
+    return lib.mla_decode_sparse(*args.values())
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(indices=None), 1), (dict(topk=-1), 1), (dict(s_q=0), 1), (dict(batch=-1), 1),
+    (dict(dtype=0), 2), (dict(dtype=1), 2), (dict(d_qk=512), 2), (dict(page_size=32), 2), (dict(h_kv=2), 2),
+    (dict(ws_bytes=1000), 3), (dict(kvcache=(1 << 20) + 8), 1),
+])
+def test_sparse_decode_rejects_bad_arguments(lib, over, code):
+    # The sparse decode reads an FP8-with-scale cache through a list of entries: anything else is
+    # rejected on the host before a launch.
+    assert _sparse(lib, **over) == code
+
+
+def test_sparse_metadata_rejects_bad_arguments(lib):
+    fake = 1 << 20
+    assert lib.mla_get_metadata_sparse(4, -1, 128, 1, 74, fake, fake, None) == 1
+    assert lib.mla_get_metadata_sparse(4, 64, 0, 1, 74, fake, fake, None) == 1
+    assert lib.mla_get_metadata_sparse(4, 64, 128, 2, 74, fake, fake, None) == 2
+    assert lib.mla_get_metadata_sparse(4, 64, 128, 1, 0, fake, fake, None) == 1
