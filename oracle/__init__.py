@@ -26,6 +26,9 @@ Functions and the passages they follow (page title, section):
   the "FlashMLA vLLM Optimization" page): 656-byte token rows of 512
   float8_e4m3 latent values, 4 float32 scales and 64 bfloat16 RoPE values,
   dequantized to bfloat16.
+* :func:`sparse_prefill` -- the sparse MLA prefill (upstream FlashMLA documentation,
+  "Sparse MLA Prefill"): out, base-2 max_logits and base-2 lse over per-query index lists
+  into a flat kv.
 * :func:`decode_sparse`, :func:`decode_sparse_fp8` -- token-level sparse decoding (the
   upstream FlashMLA documentation's "Sparse Attention (indices tensor)"): each query
   token attends the flat cache rows (page * page_size + offset) listed in
@@ -106,6 +109,10 @@ def _load():
             lib.mla_oracle_half_to_double.restype = ctypes.c_double
             lib.mla_oracle_decode_sparse.argtypes = [ctypes.POINTER(_Shape), P, P, P, ctypes.c_int, P, P]
             lib.mla_oracle_decode_sparse.restype = ctypes.c_int
+            I = ctypes.c_int
+            lib.mla_oracle_sparse_prefill.argtypes = [I, I, I, I, I, ctypes.c_long, I, I, ctypes.c_double,
+                                                      P, P, P, P, P, P]
+            lib.mla_oracle_sparse_prefill.restype = ctypes.c_int
             lib.mla_oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
             lib.mla_oracle_e4m3_to_double.restype = ctypes.c_double
             lib.mla_oracle_dequant_fp8_rows.argtypes = [P, ctypes.c_long, P]
@@ -130,7 +137,8 @@ class use_library:
         lib = ctypes.CDLL(self.path)
         for name in ("mla_oracle_decode", "mla_oracle_decode_range", "mla_oracle_decode_rows",
                      "mla_oracle_combine", "mla_oracle_half_to_double", "mla_oracle_num_threads",
-                     "mla_oracle_e4m3_to_double", "mla_oracle_dequant_fp8_rows", "mla_oracle_decode_sparse"):
+                     "mla_oracle_e4m3_to_double", "mla_oracle_dequant_fp8_rows", "mla_oracle_decode_sparse",
+                     "mla_oracle_sparse_prefill"):
             src = getattr(self._saved, name)
             dst = getattr(lib, name)
             dst.argtypes, dst.restype = src.argtypes, src.restype
@@ -304,3 +312,31 @@ def decode_sparse(q_bits, kv_bits, indices, dv=512, dtype=BF16, scale=None, page
 def decode_sparse_fp8(q_bits, kv_u8, indices, dv=512, scale=None, page_size=64):
     """:func:`decode_sparse` over an "FP8 with scale" cache (dequantized first)."""
     return decode_sparse(q_bits, dequant_fp8(kv_u8), indices, dv, BF16, scale, page_size)
+
+
+def sparse_prefill(q_bits, kv_bits, indices, sm_scale, dv=512, dtype=BF16):
+    """Sparse MLA prefill (upstream FlashMLA documentation, "Sparse MLA Prefill").
+
+    ``q_bits`` [s_q, h_q, d_qk], ``kv_bits`` [s_kv, h_kv, d_qk] (16-bit bit patterns),
+    ``indices`` [s_q, h_kv, topk] int32 (-1 or any index >= s_kv is invalid).  Returns
+    ``(out [s_q, h_q, dv], max_logits [s_q, h_q], lse [s_q, h_q])`` in float64, with
+    max_logits and lse in base 2 of the logits scaled by sm_scale * log2(e).
+    """
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    kv_bits = np.ascontiguousarray(kv_bits, dtype=np.uint16)
+    indices = np.ascontiguousarray(indices, dtype=np.int32)
+    if q_bits.ndim != 3 or kv_bits.ndim != 3 or indices.ndim != 3:
+        raise ValueError("q [s_q,h_q,d_qk], kv [s_kv,h_kv,d_qk], indices [s_q,h_kv,topk]")
+    s_q, h_q, d_qk = q_bits.shape
+    s_kv, h_kv, d2 = kv_bits.shape
+    if d2 != d_qk or indices.shape[:2] != (s_q, h_kv):
+        raise ValueError("shape mismatch")
+    out = np.empty((s_q, h_q, dv), np.float64)
+    mx = np.empty((s_q, h_q), np.float64)
+    lse = np.empty((s_q, h_q), np.float64)
+    rc = _load().mla_oracle_sparse_prefill(s_q, h_q, h_kv, d_qk, dv, s_kv, int(indices.shape[2]), dtype,
+                                           float(sm_scale), _ptr(q_bits), _ptr(kv_bits), _ptr(indices),
+                                           _ptr(out), _ptr(mx), _ptr(lse))
+    if rc:
+        raise ValueError("oracle rejected its arguments")
+    return out, mx, lse

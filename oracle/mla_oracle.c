@@ -403,6 +403,87 @@ int mla_oracle_decode_sparse(const mla_oracle_shape* sh, const uint16_t* q, cons
 }
 
 /*
+ * Sparse MLA prefill (upstream FlashMLA documentation, "Sparse MLA Prefill / Return Values
+ * and Equivalent PyTorch Code"), step by step in the documentation's order and base-2 notation.
+ * q [s_q, h_q, d_qk], kv [s_kv, h_kv, d_qk] (16-bit bit patterns), indices [s_q, h_kv, topk].
+ * For query i, head h (kv head g = h / (h_q / h_kv)), over the valid entries k (0 <= idx < s_kv;
+ * -1 or any index >= s_kv is invalid):
+ *   focused_k  = kv[idx_k, g, :]
+ *   P_k        = <q[i,h,:], focused_k> * sm_scale * log2(e)
+ *   max_logits = max_k P_k
+ *   lse        = log2(sum_k 2^{P_k})          (computed as max_logits + log2 sum_k 2^{P_k - max_logits})
+ *   S_k        = 2^{P_k - lse}
+ *   out        = sum_k S_k * focused_k[0 : dv]  (V is the leading dv columns of the row)
+ * With no valid entry: out = 0, max_logits = lse = -inf.
+ * out [s_q, h_q, dv], max_logits / lse [s_q, h_q].  Returns 0, or -1 for bad arguments.
+ */
+int mla_oracle_sparse_prefill(int s_q, int h_q, int h_kv, int d_qk, int dv, long s_kv, int topk, int dtype,
+                              double sm_scale, const uint16_t* q, const uint16_t* kv, const int32_t* indices,
+                              double* out, double* max_logits, double* lse)
+{
+    if (s_q < 0 || h_q <= 0 || h_kv <= 0 || h_q % h_kv || d_qk <= 0 || dv <= 0 || dv > d_qk || s_kv < 0 ||
+        topk < 0)
+        return -1;
+    const double log2e = 1.4426950408889634073599246810019;
+    const long rows = (long)s_q * h_q;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* P = (double*)malloc(sizeof(double) * (size_t)(topk > 0 ? topk : 1));
+        double* qrow = (double*)malloc(sizeof(double) * (size_t)d_qk);
+        if (!P || !qrow) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (long r = 0; r < rows; ++r) {
+                const long i = r / h_q;
+                const int h = (int)(r % h_q);
+                const int g = h / (h_q / h_kv);
+                const int32_t* ix = indices + ((size_t)i * h_kv + g) * topk;
+                double* o_row = out + (size_t)r * dv;
+                for (int d = 0; d < dv; ++d) o_row[d] = 0.0;
+                const uint16_t* qp = q + (size_t)r * d_qk;
+                for (int d = 0; d < d_qk; ++d) qrow[d] = mla_oracle_half_to_double(qp[d], dtype);
+                /* P = (Q @ focused_kv^T) * sm_scale * log2(e); max_logits = P.max() */
+                double mx = -INFINITY;
+                for (int k = 0; k < topk; ++k) {
+                    const long row = ix[k];
+                    if (row < 0 || row >= s_kv) continue;
+                    const uint16_t* kp = kv + ((size_t)row * h_kv + g) * (size_t)d_qk;
+                    double acc = 0.0;
+                    for (int d = 0; d < d_qk; ++d) acc += qrow[d] * mla_oracle_half_to_double(kp[d], dtype);
+                    P[k] = acc * sm_scale * log2e;
+                    if (P[k] > mx) mx = P[k];
+                }
+                max_logits[r] = mx;
+                if (mx == -INFINITY) { /* no valid entry */
+                    lse[r] = -INFINITY;
+                    continue;
+                }
+                /* lse = log2 sum 2^P */
+                double sum = 0.0;
+                for (int k = 0; k < topk; ++k)
+                    if (ix[k] >= 0 && ix[k] < s_kv) sum += exp2(P[k] - mx);
+                const double l2 = mx + log2(sum);
+                lse[r] = l2;
+                /* S = 2^(P - lse); out = S @ focused_kv[:, :dv] */
+                for (int k = 0; k < topk; ++k) {
+                    const long row = ix[k];
+                    if (row < 0 || row >= s_kv) continue;
+                    const uint16_t* vp = kv + ((size_t)row * h_kv + g) * (size_t)d_qk;
+                    const double w = exp2(P[k] - l2);
+                    for (int d = 0; d < dv; ++d) o_row[d] += w * mla_oracle_half_to_double(vp[d], dtype);
+                }
+            }
+        }
+        free(P);
+        free(qrow);
+    }
+    return err ? -1 : 0;
+}
+
+/*
  * Merge of n_parts partial results of the same rows, each the attention over a
  * disjoint token range:  LSE = log sum_k exp(lse_k),  O = sum_k exp(lse_k - LSE) O_k.
  * Parts with lse_k = -inf carry no tokens and get weight 0; if every part is

@@ -5,8 +5,8 @@ CPU, in a temporary directory) and runs the pin tests against it: at least one
 pin must fail.  This shows the pins constrain every term of the definition
 (scale, V columns, causal offset, kv-head mapping, page indexing, LSE base, the
 combine weights, the FP8 cache's scale blocks, e4m3 exponent bias and
-subnormals, RoPE offset and bfloat16 rounding, and the sparse decode's scale, LSE
-and V columns).
+subnormals, RoPE offset and bfloat16 rounding, the sparse decode's scale, LSE
+and V columns, and the sparse prefill's log2(e), LSE base, weights and V columns).
 """
 import os
 import subprocess
@@ -16,6 +16,7 @@ import pytest
 
 import oracle
 import tests.test_oracle_fp8_pins as fp8_pins
+import tests.test_oracle_prefill_pins as prefill_pins
 import tests.test_oracle_sparse_pins as sparse_pins
 import tests.test_oracle_pins as pins
 
@@ -24,8 +25,8 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "mla_oracle.c")
 MUTATIONS = {
     "causal_offset": ("L - sh->s_q + 1 + s", "L - sh->s_q + s"),
     "dropped_scale": ("x[j - lo] = sh->scale * acc;", "x[j - lo] = acc;"),
-    "v_wrong_columns": ("o_row[d] += w * mla_oracle_half_to_double(vp[d]",
-                        "o_row[d] += w * mla_oracle_half_to_double(vp[d + sh->d_qk - sh->dv]"),
+    "v_wrong_columns": ("o_row[d] += w * mla_oracle_half_to_double(vp[d], sh->dtype)",
+                        "o_row[d] += w * mla_oracle_half_to_double(vp[d + sh->d_qk - sh->dv], sh->dtype)"),
     "lse_base2": ("double lse = M + log(sum);", "double lse = M + log2(sum);"),
     "kv_head_map": ("const int g = h / (sh->h_q / sh->h_kv);", "const int g = h % sh->h_kv;"),
     "page_offset": ("(((size_t)page * P + (j % P))", "(((size_t)page * P + (j / P))"),
@@ -43,6 +44,14 @@ MUTATIONS = {
     "sparse_lse_without_sum": ("const double L = M + log(sum);", "const double L = M;"),
     "sparse_v_wrong_columns": ("o_row[d] += w * mla_oracle_half_to_double(vp[d], sh->dtype);\n                }\n            }\n        }",
                                "o_row[d] += w * mla_oracle_half_to_double(vp[d + d_qk - dv], sh->dtype);\n                }\n            }\n        }"),
+    # the sparse prefill
+    "prefill_dropped_log2e": ("P[k] = acc * sm_scale * log2e;", "P[k] = acc * sm_scale;"),
+    "prefill_lse_natural_log": ("const double l2 = mx + log2(sum);", "const double l2 = mx + log(sum);"),
+    "prefill_weights_unnormalized": ("const double w = exp2(P[k] - l2);", "const double w = exp2(P[k] - mx);"),
+    "prefill_v_wrong_columns": ("o_row[d] += w * mla_oracle_half_to_double(vp[d], dtype);",
+                                "o_row[d] += w * mla_oracle_half_to_double(vp[d + d_qk - dv], dtype);"),
+    "prefill_kv_head_map": ("const int32_t* ix = indices + ((size_t)i * h_kv + g) * topk;",
+                            "const int32_t* ix = indices + ((size_t)i * h_kv) * topk;"),
 }
 
 
@@ -71,6 +80,11 @@ def _pin_calls():
                       lambda k=kw: sparse_pins.test_sparse_brute_force_torch(oracle, k)))
     for name in ("test_one_row_listed_n_times", "test_full_token_list_equals_dense_decode"):
         calls.append((name, lambda f=getattr(sparse_pins, name): f(oracle)))
+    for kw in prefill_pins.PREFILL_CASES:
+        calls.append((f"prefill_brute:{kw}", lambda k=kw: prefill_pins.test_prefill_brute_force_torch(oracle, k)))
+    for name in ("test_prefill_hand_two_entries", "test_prefill_single_entry_and_no_entry",
+                 "test_prefill_row_listed_n_times", "test_prefill_is_the_sparse_decode_in_base_2"):
+        calls.append((name, lambda f=getattr(prefill_pins, name): f(oracle)))
     for kw in fp8_pins.FP8_BRUTE_CASES:
         calls.append((f"fp8_brute:{kw['seqlens']}",
                       lambda k=kw: fp8_pins.test_fp8_decode_brute_force_torch(oracle, k)))
