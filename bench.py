@@ -59,6 +59,9 @@ DESCR = {
                   "d_qk=576, d_v=512, topk=2048 entries per query token drawn without repetition from its "
                   "request's cache (cache_seqlens uniform in [8192,16384]), 656-byte cache rows, bf16 N(0,1) q, "
                   "scale 1/sqrt(576)",
+    "sparse_prefill": "sparse MLA prefill: s_q=2048 query tokens, h_q=128, h_kv=1, d_qk=576, d_v=512, s_kv=16384 "
+                      "kv rows, topk=2048 distinct rows per token drawn uniformly, bf16 N(0,1) q and kv, "
+                      "sm_scale 1/sqrt(576); outputs out, base-2 max_logits and lse",
 }
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NVML_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
@@ -210,6 +213,82 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- GPU arm
+class PrefillRunner:
+    """The sparse prefill's step (the metadata kernel, then split-KV and combine in one call),
+    captured like Runner's; the breakdown has two stages: metadata, split-KV + combine."""
+
+    def __init__(self, torch, mla, p, dev):
+        self.torch, self.mla, self.p, self.dev = torch, mla, p, dev
+        dt = torch.bfloat16 if p.dtype == W.BF16 else torch.float16
+        self.q = torch.from_numpy(p.q.view(np.int16)).view(dt).to(dev)
+        self.kv = torch.from_numpy(p.kv.view(np.int16)).view(dt).to(dev)
+        self.ind = torch.from_numpy(p.indices).to(dev)
+        self.parts = mla.num_sm_parts(dev)
+        _, n_ns = mla.metadata_sizes(p.s_q, p.h_q, 1, self.parts)
+        self.md = torch.zeros(self.parts, 8, dtype=torch.int32, device=dev)
+        self.ns = torch.zeros(n_ns, dtype=torch.int32, device=dev)
+        self.out = torch.empty(p.s_q, p.h_q, p.dv, dtype=dt, device=dev)
+        self.mx = torch.empty(p.s_q, p.h_q, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(p.s_q, p.h_q, dtype=torch.float32, device=dev)
+        self.ws = torch.zeros(mla.workspace_bytes(p.s_q, 1, p.h_q, 1, self.parts), dtype=torch.uint8, device=dev)
+        from mla_decode_attention_12_b200 import _lib
+        lib, topk = _lib.load(), p.indices.shape[2]
+        ptr = lambda t: t.data_ptr()
+
+        def metadata():
+            _lib.check(lib.mla_get_metadata_sparse(p.s_q, topk, p.h_q, 1, self.parts, ptr(self.md), ptr(self.ns),
+                                                   torch.cuda.current_stream(dev).cuda_stream), "metadata")
+
+        def prefill():
+            _lib.check(lib.mla_sparse_prefill(ptr(self.q), p.s_q, p.h_q, p.d_qk, ptr(self.kv), p.s_kv, 1, ptr(self.ind),
+                                              topk, p.dv, p.dtype, p.sm_scale, ptr(self.md), self.parts, ptr(self.ns),
+                                              ptr(self.out), ptr(self.mx), ptr(self.lse), ptr(self.ws),
+                                              self.ws.numel(), torch.cuda.current_stream(dev).cuda_stream), "prefill")
+
+        stages = [metadata, prefill]
+        self.launches_per_step = 3
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            for _ in range(2):
+                for f in stages:
+                    f()
+        torch.cuda.current_stream(dev).wait_stream(s)
+        torch.cuda.synchronize(dev)
+        self.events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.events[0].record()
+            for f in stages:
+                f()
+            self.events[1].record()
+        self.stage_events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+        self.stage_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.stage_graph):
+            self.stage_events[0].record()
+            for i, f in enumerate(stages):
+                f()
+                self.stage_events[i + 1].record()
+        torch.cuda.synchronize(dev)
+
+    def step(self):
+        self.graph.replay()
+
+    def step_staged(self):
+        self.stage_graph.replay()
+
+    def times_ms(self):
+        return self.events[0].elapsed_time(self.events[1])
+
+    def stage_times_ms(self):
+        """(metadata, split-KV + combine, 0): the prefill's two kernels run in one call."""
+        e = self.stage_events
+        return (e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), 0.0)
+
+    def status(self):
+        return self.mla.read_device_status(self.ws, clear=True)
+
+
 class Runner:
     """Device tensors and the three launches of one decode step for one workload.
 
@@ -505,10 +584,22 @@ def run_ours(args):
 
     extra = {}
     names = [] if args.extra_workloads == "none" else (
-        [w for w in W.WORKLOADS + W.SPARSE_WORKLOADS if w != args.workload] if args.extra_workloads == "all"
+        [w for w in W.WORKLOADS + W.SPARSE_WORKLOADS + W.PREFILL_WORKLOADS if w != args.workload]
+        if args.extra_workloads == "all"
         else [w for w in args.extra_workloads.split(",") if w and w != args.workload])
     if rank == 0:
         for name in names:
+            if name in W.PREFILL_WORKLOADS:
+                pw = W.make_prefill_workload(name)
+                r = PrefillRunner(torch, mla, pw, dev)
+                tw = time_steps(torch, r, flush, min(args.steps, 50), min(args.warmup, 5), lambda: None)
+                extra[name] = workload_line(pw, tw, peaks, src)
+                extra[name]["workload"] = DESCR[name]
+                extra[name]["device_status"] = r.status()
+                extra[name]["note"] = "us_splitkv is split-KV + combine (one call); the kv is L2-resident and counted once"
+                del r
+                torch.cuda.empty_cache()
+                continue
             pw = W.make_workload(name)
             r = Runner(torch, mla, pw, dev)
             tw = time_steps(torch, r, flush, min(args.steps, 200), min(args.warmup, 10), lambda: None)

@@ -246,10 +246,13 @@ MLA_API mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int
  *   mla_get_metadata with num_parts rows, num_splits [num_tokens * ceil(h_q / h_kv / 128) + 1].
  * mla_decode_sparse:
  *   q            device [batch, s_q, h_q, 576] bfloat16, 16-byte aligned
- *   kvcache      device [num_blocks, 64, 1, 656] bytes ("FP8 with scale" rows), 16-byte aligned
+ *   kvcache      device [num_blocks, 64, 1, 656] bytes ("FP8 with scale" rows) for MLA_BF16_FP8KV,
+ *                or [num_blocks, 64, 1, 576] bf16 / fp16 rows for MLA_BF16 / MLA_FP16 (a
+ *                16-bit cache: not on the pages, whose sparse decode reads FP8; same definition);
+ *                16-byte aligned
  *   indices      device int32 [batch, s_q, topk]
- *   dtype        must be MLA_BF16_FP8KV (MLA_ERR_UNSUPPORTED otherwise); d_qk 576, dv 512, h_kv 1,
- *                page_size 64
+ *   dtype        MLA_BF16_FP8KV, MLA_BF16 or MLA_FP16; d_qk 576 (MLA_ERR_UNSUPPORTED otherwise), dv 512,
+ *                h_kv 1, page_size 64
  *   tile_md, num_splits, num_parts   from mla_get_metadata_sparse for this batch * s_q and topk
  *   active_heads, softmax_scale, o, lse  as for mla_decode_with_kvcache
  *   workspace    >= mla_decode_workspace_bytes(batch * s_q, 1, h_q, 1, num_parts)
@@ -270,6 +273,39 @@ MLA_API mla_status mla_decode_sparse_splitkv(const void* q, int batch, int s_q, 
                                              const int32_t* tile_md, int num_parts, const int32_t* num_splits,
                                              float softmax_scale, int active_heads, void* o, float* lse,
                                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Sparse MLA prefill (upstream FlashMLA documentation, "Sparse MLA Prefill": flash_mla_sparse_fwd(q,
+ * kv, indices, sm_scale) returns (out, max_logits, lse), equivalent to the documentation's PyTorch
+ * code).  No batch dimension and no pages: query token i attends the rows indices[i][0][k] of kv.
+ *
+ * For query token i and head h (kv head 0), over the valid entries E = { k < topk :
+ * 0 <= indices[i][0][k] < s_kv } (-1 or any index >= s_kv is invalid):
+ *   P_k        = <q[i,h,:], kv[idx_k,0,:]> * sm_scale * log2(e)
+ *   max_logits = max_{k in E} P_k                      (-inf when E is empty)
+ *   lse        = log2(sum_{k in E} 2^{P_k})             (base 2; -inf when E is empty)
+ *   out        = sum_{k in E} 2^{P_k - lse} kv[idx_k,0,0:512]   (0 when E is empty)
+ * (The documentation's equivalent code multiplies by the whole focused row; as everywhere in
+ * the MQA mode, V is the leading dv = 512 columns.)
+ *
+ *   q            device [s_q, h_q, 576] bf16 or fp16, 16-byte aligned
+ *   kv           device [s_kv, 1, 576], the dtype of q, 16-byte aligned
+ *   indices      device int32 [s_q, 1, topk]
+ *   dtype        MLA_BF16 or MLA_FP16;  dv 512;  h_kv 1
+ *   sm_scale     > 0, or <= 0 for 1/sqrt(576)
+ *   tile_md, num_splits, num_parts   from mla_get_metadata_sparse(s_q, topk, h_q, 1, num_parts, ...)
+ *   out          device [s_q, h_q, 512], the dtype of q, written
+ *   max_logits   device float32 [s_q, h_q], written
+ *   lse          device float32 [s_q, h_q], written (base 2)
+ *   workspace    >= mla_decode_workspace_bytes(s_q, 1, h_q, 1, num_parts), zero control block
+ * Enqueues the split-KV kernel and the combine kernel on `stream`.  Errors: as for
+ * mla_decode_with_kvcache; MLA_ERR_UNSUPPORTED for an FP8 dtype.
+ */
+MLA_API mla_status mla_sparse_prefill(const void* q, int s_q, int h_q, int d_qk, const void* kv, int s_kv, int h_kv,
+                                      const int32_t* indices, int topk, int dv, int dtype, float sm_scale,
+                                      const int32_t* tile_md, int num_parts, const int32_t* num_splits, void* out,
+                                      float* max_logits, float* lse, void* workspace, size_t workspace_bytes,
+                                      void* stream);
 
 /*
  * Reads the device status word of a workspace (synchronises `stream`).

@@ -55,6 +55,10 @@ SIGNATURES = {
                            _P, _P, _P, _SZ, _P], _I),   # o, lse, workspace, ws_bytes, stream
     "mla_decode_sparse_splitkv": ([_P, _I, _I, _I, _I, _P, _I, _I, _I, _P, _I, _I, _I,
                                    _P, _I, _P, _F, _I, _P, _P, _P, _SZ, _P], _I),
+    "mla_sparse_prefill": ([_P, _I, _I, _I, _P, _I, _I,      # q, s_q, h_q, d_qk, kv, s_kv, h_kv
+                            _P, _I, _I, _I, _F,              # indices, topk, dv, dtype, sm_scale
+                            _P, _I, _P,                      # tile_md, num_parts, num_splits
+                            _P, _P, _P, _P, _SZ, _P], _I),   # out, max_logits, lse, workspace, bytes, stream
 }
 
 _lock = threading.Lock()

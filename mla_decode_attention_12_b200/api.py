@@ -150,8 +150,6 @@ class DecodeCall:
         dev = q.device
         self.sparse = indices is not None
         if self.sparse:
-            if not is_fp8_kvcache:
-                raise ValueError("the sparse decode (indices) reads an FP8-with-scale cache")
             if indices.dtype != torch.int32 or indices.dim() != 3 or indices.shape[:2] != q.shape[:2]:
                 raise ValueError("indices must be int32 [batch, s_q, topk]")
             if not indices.is_contiguous() or indices.device != dev:
@@ -172,6 +170,8 @@ class DecodeCall:
                 raise ValueError(f"{name} must be contiguous and on {dev}")
         b, s_q, h_q, d_qk = q.shape
         num_blocks, page, h_kv, d2 = kvcache.shape
+        if not is_fp8_kvcache and d2 != d_qk:
+            raise ValueError("q and kvcache rows must have the same width")
         if not self.sparse:
             if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32:
                 raise ValueError("block_table and cache_seqlens must be int32")
@@ -265,6 +265,52 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
     if host:
         return out.cpu(), lse.cpu()
     return out, lse
+
+
+def flash_mla_sparse_fwd(q: torch.Tensor, kv: torch.Tensor, indices: torch.Tensor, sm_scale: float, d_v: int = 512,
+                         num_parts: int | None = None, workspace: torch.Tensor | None = None):
+    """Sparse MLA prefill (upstream FlashMLA documentation, "Sparse MLA Prefill").
+
+    ``q`` [s_q, h_q, 576] and ``kv`` [s_kv, 1, 576] bf16 (or fp16), ``indices`` int32
+    [s_q, 1, topk] (-1 or any index >= s_kv is invalid).  Returns ``(out [s_q, h_q, d_v],
+    max_logits [s_q, h_q] float32, lse [s_q, h_q] float32)``, max_logits and lse in base 2 of
+    the logits scaled by ``sm_scale * log2(e)``.  The tile schedule is computed on the device
+    as part of the call.
+    """
+    if q.dtype not in _DTYPES or kv.dtype != q.dtype:
+        raise ValueError("q and kv must both be bfloat16 or both float16")
+    if q.dim() != 3 or kv.dim() != 3 or indices.dim() != 3 or indices.dtype != torch.int32:
+        raise ValueError("q [s_q, h_q, d_qk], kv [s_kv, h_kv, d_qk], indices int32 [s_q, h_kv, topk]")
+    s_q, h_q, d_qk = q.shape
+    s_kv, h_kv, d2 = kv.shape
+    if d2 != d_qk or indices.shape[:2] != (s_q, h_kv):
+        raise ValueError("inconsistent shapes")
+    dev = q.device
+    for name, t in (("q", q), ("kv", kv), ("indices", indices)):
+        if not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must be contiguous and on {dev}")
+    topk = indices.shape[2]
+    if num_parts is None:
+        num_parts = num_sm_parts(dev)
+    n_md, n_ns = metadata_sizes(s_q, h_q // h_kv, h_kv, num_parts)
+    md = torch.empty(n_md, dtype=torch.int32, device=dev).view(num_parts, 8)
+    ns = torch.empty(n_ns, dtype=torch.int32, device=dev)
+    out = torch.empty(s_q, h_q, d_v, dtype=q.dtype, device=dev)
+    max_logits = torch.empty(s_q, h_q, dtype=torch.float32, device=dev)
+    lse = torch.empty(s_q, h_q, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = get_workspace(workspace_bytes(s_q, 1, h_q, h_kv, num_parts), dev,
+                                  workspace_zero_bytes(s_q, 1, h_q, h_kv))
+    lib = _lib.load()
+    with torch.cuda.device(dev):
+        st = _stream(dev)
+        _lib.check(lib.mla_get_metadata_sparse(s_q, topk, h_q, h_kv, num_parts, _ptr(md), _ptr(ns), st),
+                   "mla_get_metadata_sparse")
+        _lib.check(lib.mla_sparse_prefill(_ptr(q), s_q, h_q, d_qk, _ptr(kv), s_kv, h_kv, _ptr(indices), topk, d_v,
+                                          _DTYPES[q.dtype], float(sm_scale), _ptr(md), num_parts, _ptr(ns),
+                                          _ptr(out), _ptr(max_logits), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                          st), "mla_sparse_prefill")
+    return out, max_logits, lse
 
 
 def read_device_status(workspace: torch.Tensor, clear: bool = True) -> int:

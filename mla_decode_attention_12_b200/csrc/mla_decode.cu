@@ -203,8 +203,10 @@ struct DecodeParams {
     const void* kvcache;
     void* o;
     float* lse;
+    float* max_logits;  // sparse prefill: [tokens, h_q], the largest base-2 scaled logit (null: not wanted)
     float* o_accum;     // [slots, 128, 512]
     float* lse_accum;   // [slots, 128]
+    float* max_accum;   // [slots, 128] split maxima of the base-2 scaled logits
     int* status;
     int* ctl;  // [kMaxVirtualBatches][2] per virtual batch: split-KV warps that announced their
                // partials (8 per split), combine CTAs past their wait
@@ -212,6 +214,7 @@ struct DecodeParams {
     int active_heads;  // heads >= active_heads are padding: not written, not combined
     int o_align32;     // o is 32-byte aligned: 32-byte stores
     int topk;          // sparse decode: entries per request
+    int lse_base2;     // write the LSE in base 2 (the sparse prefill's convention)
     int cache_rows;    // num_blocks * 64: a sparse entry outside [0, cache_rows) is invalid
     float scale_log2;
     int dtype, d_qk, num_parts;  // host-side dispatch only
@@ -386,7 +389,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                        const __grid_constant__ CUtensorMap tm_v, const DecodeParams p)
 {
     static_assert(!kFp8 || (kRope && !kFp16), "the FP8 cache has d_qk = 576 and bfloat16 queries");
-    static_assert(!kSparse || kFp8, "the sparse decode reads an FP8 cache");
     using L = Layout<kRope, kFp8>;
     constexpr int kNumThreads = kFp8 ? kThreadsFp8 : kThreads;
     extern __shared__ uint8_t smem_raw[];
@@ -705,7 +707,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             }
         } else if (warp == kKWarp) {
             // ============================ K producer ============================
-            if constexpr (kSparse) {
+            if constexpr (kSparse && kFp8) {
+                static_assert(L::kRawKStages > 0, "the FP8 layout's raw ring");
                 // Sparse decode: row i of this CTA's half of "page" blk is entry 64 blk + 32 cta + i
                 // of the request's list.  Lane i bulk-copies its row (656 bytes as stored) when
                 // the entry is valid; lane 0 records the half's validity bits with the stage and
@@ -773,6 +776,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                         }
                     }
                 }
+            } else if constexpr (kSparse) {
+                static_assert(!kFp8, "16-bit rows");
+                // Sparse, 16-bit rows: row i of this CTA's half of "page" blk is entry 64 blk + 32 cta + i.
+                // Lane g < 8 gathers rows 4 g .. 4 g + 3 of every 64-column box (TMA tile::gather4);
+                // an invalid entry names the row just past the tensor, which reads zeros.
+                Ring<L::kKStages> ring;
+                int vb, lo, hi;
+                bool ok = true;
+                auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
+                while (ok && chunks.next(vb, lo, hi)) {
+                    if (hi <= lo) continue;
+                    const int32_t* ent = p.indices + static_cast<size_t>(vb / p.groups) * p.topk;
+                    auto entry = [&](int blk) {
+                        const int e = kPage * blk + 32 * static_cast<int>(cta) + lane;
+                        const int idx = e < p.topk ? __ldg(ent + e) : -1;
+                        return (idx >= 0 && idx < p.cache_rows) ? idx : p.cache_rows;
+                    };
+                    int row = entry(lo);
+                    for (int blk = lo; blk < hi; ++blk, ring.advance()) {
+                        const int row_next = blk + 1 < hi ? entry(blk + 1) : p.cache_rows;
+                        const uint32_t st = ring.stage;
+                        if (!(ok = wwait(bar(kBarKEmpty + st), ring.phase ^ 1))) break;
+                        if (lane == 0 && leader) mbar_arrive_expect_tx(bar(kBarKFull + st), 2 * L::kKBytes);
+                        const int g = lane & 7;
+                        const int r0 = __shfl_sync(0xffffffffu, row, 4 * g), r1 = __shfl_sync(0xffffffffu, row, 4 * g + 1);
+                        const int r2 = __shfl_sync(0xffffffffu, row, 4 * g + 2), r3 = __shfl_sync(0xffffffffu, row, 4 * g + 3);
+                        if (lane < 8)
+                            for (int i = 0; i < L::kBoxes; ++i)
+                                tma_gather4_pair(s_k + st * L::kKBytes + i * 4096 + 512 * g, &tm_k, lead_bar(kBarKFull + st),
+                                                 64 * i, r0, r1, r2, r3);
+                        row = row_next;
+                    }
+                }
+                if (!ok && lane == 0) {
+                    const uint64_t t0 = global_timer_ns();  // let issued loads land (see the V producer)
+                    while (global_timer_ns() - t0 < 50000000ull) {
+                    }
+                }
             } else if (lane == 0) {
                 TL_OPEN(2);
                 Ring<L::kKStages> ring;
@@ -801,8 +842,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 }
             }
         } else if (warp == kVWarp) {
-            if constexpr (kSparse) {
-                // ======================== V producer (sparse decode) ========================
+            if constexpr (kSparse && kFp8) {
+                static_assert(L::kRawVStages > 0, "the FP8 layout's raw ring");
+                // ===================== V producer (sparse decode, FP8 cache) =====================
                 // The peer's 32 rows of "page" blk (entries 64 blk + 32 (1 - cta) + i): lane i copies
                 // this CTA's two 128-byte latent slices (its V columns) and the 16 bytes of scales
                 // of its row when the entry is valid, in the layout the TMA boxes give the dense
@@ -874,6 +916,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                         const uint64_t t0 = global_timer_ns();  // let issued loads land (see below)
                         while (global_timer_ns() - t0 < 50000000ull) {
                         }
+                    }
+                }
+            } else if constexpr (kSparse) {
+                static_assert(!kFp8, "16-bit rows");
+                // ==================== V producer (sparse, 16-bit rows) ====================
+                // The page's 64 entries x this CTA's 4 V boxes, by gather4 (lane g < 16: rows 4 g ..
+                // 4 g + 3); invalid entries read zeros, so nothing needs clearing.
+                Ring<L::kVStages> ring;
+                int vb, lo, hi;
+                bool ok = true;
+                auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
+                while (ok && chunks.next(vb, lo, hi)) {
+                    if (hi <= lo) continue;
+                    const int32_t* ent = p.indices + static_cast<size_t>(vb / p.groups) * p.topk;
+                    auto entry = [&](int e) {
+                        const int idx = e < p.topk ? __ldg(ent + e) : -1;
+                        return (idx >= 0 && idx < p.cache_rows) ? idx : p.cache_rows;
+                    };
+                    int row_a = entry(kPage * lo + lane), row_b = entry(kPage * lo + 32 + lane);
+                    for (int blk = lo; blk < hi; ++blk, ring.advance()) {
+                        const bool more = blk + 1 < hi;
+                        const int next_a = more ? entry(kPage * (blk + 1) + lane) : p.cache_rows;
+                        const int next_b = more ? entry(kPage * (blk + 1) + 32 + lane) : p.cache_rows;
+                        const uint32_t st = ring.stage;
+                        if (!(ok = wwait(bar(kBarVEmpty + st), ring.phase ^ 1))) break;
+                        if (lane == 0 && leader) mbar_arrive_expect_tx(bar(kBarVFull + st), 2 * L::kVBytes);
+                        const int g = lane & 15, src = 4 * (g & 7);  // rows 4 g .. 4 g + 3 of the page
+                        const int r0a = __shfl_sync(0xffffffffu, row_a, src), r1a = __shfl_sync(0xffffffffu, row_a, src + 1);
+                        const int r2a = __shfl_sync(0xffffffffu, row_a, src + 2), r3a = __shfl_sync(0xffffffffu, row_a, src + 3);
+                        const int r0b = __shfl_sync(0xffffffffu, row_b, src), r1b = __shfl_sync(0xffffffffu, row_b, src + 1);
+                        const int r2b = __shfl_sync(0xffffffffu, row_b, src + 2), r3b = __shfl_sync(0xffffffffu, row_b, src + 3);
+                        if (lane < 16) {
+                            const bool hi_half = g >= 8;
+                            for (int i = 0; i < 4; ++i) {
+                                const int box = 4 * (i >> 1) + 2 * static_cast<int>(cta) + (i & 1);
+                                tma_gather4_pair(s_v + st * L::kVBytes + i * 8192 + 512 * g, &tm_v, lead_bar(kBarVFull + st),
+                                                 64 * box, hi_half ? r0b : r0a, hi_half ? r1b : r1a,
+                                                 hi_half ? r2b : r2a, hi_half ? r3b : r3a);
+                            }
+                        }
+                        __syncwarp();
+                        if (lane == 0 && !leader) mbar_arrive_remote(lead_bar(kBarVFull + st));
+                        row_a = next_a;
+                        row_b = next_b;
+                    }
+                }
+                if (!ok && lane == 0) {
+                    const uint64_t t0 = global_timer_ns();  // let issued loads land (see below)
+                    while (global_timer_ns() - t0 < 50000000ull) {
                     }
                 }
             } else {
@@ -1128,6 +1219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             const size_t slot = static_cast<size_t>(p.num_splits[vb]) + split_idx;  // split partial's workspace slot
             const int n = hi - lo;
             float m_ref = -INFINITY, l_half = 0.f;
+            float row_max = -INFINITY;  // the chunk's largest scaled logit, base 2 (the prefill's max_logits)
 
             if (t == 0) TL_EV(kEvChunkBegin);
             // The next chunk's Q row goes to L2 a few pages before the end of this chunk, so
@@ -1201,6 +1293,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 if (lane == 0) mbar_arrive(pair_bar);
                 if (!(ok = wwait(pair_bar, pair_phase++ & 1))) break;
                 mx = fmaxf(mx, red[sb * 128 + (t ^ 64)]);
+                row_max = fmaxf(row_max, mx);
                 // the same decision in both halves of the row
                 float alpha = 1.f;
                 bool rescale = false;
@@ -1289,7 +1382,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             if (lane == 0) mbar_arrive(pair_bar);  // red[256..] free for the next chunk once both have read it
             if (!(ok = wwait(pair_bar, pair_phase++ & 1))) break;
             const float inv_l = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
-            const float lse_v = (l_sum > 0.f) ? (m_ref + log2f(l_sum)) * 0.69314718055994531f : -INFINITY;
+            const float lse2 = (l_sum > 0.f) ? m_ref + log2f(l_sum) : -INFINITY;  // base 2
+            const float lse_v = lse2 * 0.69314718055994531f;                        // natural log
             if (!empty) {
                 if (!(ok = wwait(bar(kBarOFull), k & 1))) break;
                 if (t == 0) TL_EV(kEvOFull);
@@ -1362,10 +1456,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             }
             if (t == 0) TL_EV(kEvEpiDone);
             if (h == 0 && row_valid && (!kPadHeads || row % p.h_q < p.active_heads)) {
-                if (nsplit == 1)
-                    p.lse[static_cast<size_t>(b) * p.rows + row] = lse_v;
-                else
+                if (nsplit == 1) {
+                    const size_t at = static_cast<size_t>(b) * p.rows + row;
+                    p.lse[at] = p.lse_base2 ? lse2 : lse_v;
+                    if (p.max_logits) p.max_logits[at] = row_max;
+                } else {
                     p.lse_accum[slot * kRowsPerGroup + 64 * cta + r] = lse_v;
+                    p.max_accum[slot * kRowsPerGroup + 64 * cta + r] = row_max;
+                }
             }
             if (nsplit > 1) announce_vb = vb;
             if (!empty) ++k;
@@ -1452,6 +1550,13 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
 #pragma unroll
     for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float lse = (mx == -INFINITY) ? -INFINITY : mx + logf(sum);
+    float row_max = -INFINITY;  // the largest base-2 scaled logit over the splits (the prefill's max_logits)
+    if (p.max_logits) {
+        const float* max_k = p.max_accum + static_cast<size_t>(slot0) * kRowsPerGroup + r;
+        for (int k = lane; k < nsplit; k += 32) row_max = fmaxf(row_max, __ldcg(max_k + static_cast<size_t>(k) * kRowsPerGroup));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) row_max = fmaxf(row_max, __shfl_xor_sync(0xffffffffu, row_max, o));
+    }
     float4 acc[4];  // float4 columns lane, lane + 32, lane + 64, lane + 96
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1501,7 +1606,11 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         dst[lane + 32 * i] = make_uint2(pack2(acc[i].x, acc[i].y, kFp16), pack2(acc[i].z, acc[i].w, kFp16));
-    if (lane == 0) p.lse[static_cast<size_t>(b) * p.rows + row] = lse;
+    if (lane == 0) {
+        const size_t at = static_cast<size_t>(b) * p.rows + row;
+        p.lse[at] = p.lse_base2 ? lse * 1.4426950408889634f : lse;
+        if (p.max_logits) p.max_logits[at] = row_max;
+    }
 }
 
 // ------------------------------------------------------------------ metadata kernel
@@ -1690,8 +1799,10 @@ static void workspace_pointers(void* workspace, int batch, int groups, int num_p
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     prm.status = reinterpret_cast<int*>(ws);
     prm.ctl = reinterpret_cast<int*>(ws + kWorkspaceHeader);
+    const size_t small = align_up(slots * kRowsPerGroup * sizeof(float), 256);  // one float per slot row
     prm.lse_accum = reinterpret_cast<float*>(ws + kControlBytes);
-    prm.o_accum = reinterpret_cast<float*>(ws + kControlBytes + align_up(slots * kRowsPerGroup * sizeof(float), 256));
+    prm.max_accum = reinterpret_cast<float*>(ws + kControlBytes + small);
+    prm.o_accum = reinterpret_cast<float*>(ws + kControlBytes + 2 * small);
 }
 
 // Runs a per-device set-up step (a kernel attribute) once for each device it is used on,
@@ -1864,7 +1975,7 @@ size_t mla_decode_workspace_bytes(int batch, int s_q, int h_q, int h_kv, int num
     if (static_cast<long long>(batch) * groups > kMaxVirtualBatches) return 0;
     const size_t slots = workspace_slots(batch, groups, num_parts);
     size_t bytes = kControlBytes;
-    bytes += align_up(slots * kRowsPerGroup * sizeof(float), 256);
+    bytes += 2 * align_up(slots * kRowsPerGroup * sizeof(float), 256);  // split LSEs and maxima
     bytes += slots * kRowsPerGroup * kDv * sizeof(float);
     return bytes;
 }
@@ -1876,7 +1987,7 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
                                  const int32_t* tile_md, int num_parts, const int32_t* num_splits, int causal,
                                  float softmax_scale, int active_heads, void* o, float* lse, void* workspace,
                                  size_t workspace_bytes, const int32_t* indices, int topk, DecodeParams& prm,
-                                 CUtensorMap* maps)
+                                 CUtensorMap* maps, long long cache_rows_override = 0)
 {
     // indices != null: the sparse decode, with batch = requests x query tokens and s_q = 1;
     // no block table, no sequence lengths, no causal mask
@@ -1887,7 +1998,7 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     if (dtype != MLA_BF16 && dtype != MLA_FP16 && dtype != MLA_BF16_FP8KV) return MLA_ERR_INVALID_ARG;
     if (page_size != kPage || h_kv != 1 || (d_qk != 576 && d_qk != 512) || dv != kDv) return MLA_ERR_UNSUPPORTED;
     if (dtype == MLA_BF16_FP8KV && d_qk != 576) return MLA_ERR_UNSUPPORTED;  // the FP8 row carries 64 RoPE values
-    if (sparse && dtype != MLA_BF16_FP8KV) return MLA_ERR_UNSUPPORTED;        // the sparse decode reads an FP8 cache
+    if (sparse && d_qk != 576) return MLA_ERR_UNSUPPORTED;  // the sparse kernels are built for 576-wide rows
     if (batch > 0 && (!q || !kvcache || (!sparse && (!block_table || !cache_seqlens)) || !tile_md || !num_splits ||
                       !o || !lse || !workspace))
         return MLA_ERR_INVALID_ARG;
@@ -1900,13 +2011,15 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     const size_t need = mla_decode_workspace_bytes(batch, s_q, h_q, h_kv, num_parts);
     if (batch > 0 && workspace_bytes < need) return MLA_ERR_WORKSPACE;
     if (static_cast<long long>(num_blocks) * kPage >= (1ll << 31)) return MLA_ERR_UNSUPPORTED;
+    // rows of the cache the sparse gathers address: every page's rows, or a flat kv's own count
+    const long long cache_rows = cache_rows_override > 0 ? cache_rows_override : static_cast<long long>(num_blocks) * kPage;
     if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt(static_cast<float>(d_qk));
     prm = DecodeParams{};
     prm.block_table = sparse ? nullptr : block_table;
     prm.seqlens = sparse ? nullptr : cache_seqlens;
     prm.indices = indices;
     prm.topk = topk;
-    prm.cache_rows = num_blocks * kPage;
+    prm.cache_rows = static_cast<int>(cache_rows);
     prm.md = tile_md;
     prm.num_splits = num_splits;
     prm.q = q;
@@ -1935,13 +2048,23 @@ static mla_status prepare_decode(const void* q, int batch, int s_q, int h_q, int
     const CUtensorMapDataType dt =
         dtype == MLA_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const uint64_t row_bytes = static_cast<uint64_t>(d_qk) * 2;
-    const uint64_t kv_rows = static_cast<uint64_t>(num_blocks) * kPage;
+    const uint64_t kv_rows = static_cast<uint64_t>(cache_rows);
     // Q: [batch][rows][d_qk], box 64 columns x (up to) 64 rows;
     // K: cache rows, box 64 columns x 32 tokens (half a page, one CTA's share);
     // V: cache rows, box 64 columns x 64 tokens (a page).
     // FP8 cache: rows of 656 bytes; K: boxes of 128 bytes x 32 rows (latent slices), V: boxes
     // of 16 bytes x 32 rows (the scales), no swizzle.
     const bool fp8 = dtype == MLA_BF16_FP8KV;
+    if (sparse && !fp8) {
+        // 16-bit sparse: K and V gathered row by row (tile::gather4, one-row boxes of 64 columns);
+        // the maps end at the last row, so an invalid entry's row (cache_rows) reads zeros
+        const bool ok_g =
+            encode_3d(&maps[0], q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 64, prm.box_rows,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&maps[1], kvcache, dt, d_qk, kv_rows, row_bytes, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&maps[2], kvcache, dt, d_qk, kv_rows, row_bytes, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+        return ok_g ? MLA_OK : MLA_ERR_CUDA;
+    }
     const bool ok =
         encode_3d(&maps[0], q, dt, d_qk, rows, batch, row_bytes, row_bytes * rows, 64, prm.box_rows,
                   CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -1959,8 +2082,11 @@ static mla_status launch_splitkv_stage(const DecodeParams& prm, const CUtensorMa
 {
     const int grid = 2 * prm.num_parts;
     cudaError_t e;
-    if (prm.indices)
+    if (prm.indices && prm.dtype == MLA_BF16_FP8KV)
         e = launch_splitkv_heads<true, false, true, true>(grid, st, maps, prm);
+    else if (prm.indices)
+        e = prm.dtype == MLA_FP16 ? launch_splitkv_heads<true, true, false, true>(grid, st, maps, prm)
+                                  : launch_splitkv_heads<true, false, false, true>(grid, st, maps, prm);
     else if (prm.dtype == MLA_BF16_FP8KV)
         e = launch_splitkv_heads<true, false, true>(grid, st, maps, prm);
     else if (prm.d_qk == 576)
@@ -2116,6 +2242,30 @@ mla_status mla_decode_sparse_splitkv(const void* q, int batch, int s_q, int h_q,
     return decode_sparse(q, batch, s_q, h_q, d_qk, kvcache, num_blocks, page_size, h_kv, indices, topk, dv, dtype,
                          tile_md, num_parts, num_splits, softmax_scale, active_heads, o, lse, workspace,
                          workspace_bytes, stream, true);
+}
+
+mla_status mla_sparse_prefill(const void* q, int s_q, int h_q, int d_qk, const void* kv, int s_kv, int h_kv,
+                              const int32_t* indices, int topk, int dv, int dtype, float sm_scale, const int32_t* tile_md,
+                              int num_parts, const int32_t* num_splits, void* out, float* max_logits, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (s_q < 0 || s_kv <= 0 || topk < 0 || (s_q > 0 && (!indices || !max_logits))) return MLA_ERR_INVALID_ARG;
+    if (dtype != MLA_BF16 && dtype != MLA_FP16) return dtype == MLA_BF16_FP8KV ? MLA_ERR_UNSUPPORTED : MLA_ERR_INVALID_ARG;
+    DecodeParams prm;
+    CUtensorMap maps[kNumMaps];
+    // every query token is a request; the kv rows are addressed directly (no pages, no table)
+    const int pages = (s_kv + kPage - 1) / kPage;
+    const int32_t* one = indices ? indices : reinterpret_cast<const int32_t*>(&prm);  // not read when s_q == 0
+    mla_status s = prepare_decode(q, s_q, 1, h_q, d_qk, kv, pages, kPage, h_kv, nullptr, 1, nullptr, dv, dtype, tile_md,
+                                  num_parts, num_splits, 0, sm_scale, 0, out, lse, workspace, workspace_bytes, one,
+                                  topk, prm, maps, s_kv);
+    if (s != MLA_OK || s_q == 0) return s;
+    prm.max_logits = max_logits;
+    prm.lse_base2 = 1;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = launch_splitkv_stage(prm, maps, st);
+    if (s != MLA_OK) return s;
+    return launch_combine_stage(prm, st);
 }
 
 mla_status mla_read_device_status(void* workspace, int clear, int* device_status, void* stream)

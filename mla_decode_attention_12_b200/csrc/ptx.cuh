@@ -387,6 +387,20 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void* map, 
         : "memory");
 }
 
+// Two-SM TMA gather: rows r0..r3 (any order, any rows of the tensor; a row outside the
+// tensor reads zeros) of the box that starts at column x, into 4 consecutive box rows of this
+// CTA's shared memory (swizzled as the tensor map says), completing on an mbarrier that may be
+// the peer's.  The tensor map's box is one row high.
+__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const void* map, uint32_t cluster_bar, int x, int r0,
+                                                 int r1, int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(map), "r"(cluster_bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
 // Arrive on an mbarrier given by cluster address (own or peer CTA) and register
 // an expected transaction byte count in the same step.
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_bar, uint32_t bytes)

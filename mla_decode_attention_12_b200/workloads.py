@@ -266,6 +266,91 @@ def make_sparse_problem(seqlens, topk: int, *, s_q: int = 1, invalid_frac: float
     return p
 
 
+@dataclasses.dataclass
+class PrefillProblem:
+    """Sparse MLA prefill inputs: q [s_q, h_q, d_qk], kv [s_kv, 1, d_qk] (16-bit bit patterns),
+    indices int32 [s_q, 1, topk] (-1 or >= s_kv invalid)."""
+
+    name: str
+    q: np.ndarray
+    kv: np.ndarray
+    indices: np.ndarray
+    sm_scale: float
+    dtype: int = BF16
+    dv: int = 512
+    seed: int = 0
+
+    @property
+    def s_q(self) -> int:
+        return self.q.shape[0]
+
+    @property
+    def h_q(self) -> int:
+        return self.q.shape[1]
+
+    @property
+    def d_qk(self) -> int:
+        return self.q.shape[2]
+
+    @property
+    def s_kv(self) -> int:
+        return self.kv.shape[0]
+
+    def valid_entries(self) -> np.ndarray:
+        return (self.indices >= 0) & (self.indices < self.s_kv)
+
+    def flops(self) -> float:
+        """2 * (d_qk + d_v) per (query row, valid entry) pair."""
+        return 2.0 * (self.d_qk + self.dv) * float(self.valid_entries().sum()) * self.h_q
+
+    active_heads = None
+    fp8_kv = False
+
+    def kv_bytes(self) -> int:
+        """The kv rows, once: every token's entries are rows of the same (L2-sized) kv."""
+        return self.s_kv * self.d_qk * 2
+
+    def gathered_bytes(self) -> int:
+        """The rows the query tokens' valid entries name, one read per entry."""
+        return int(self.valid_entries().sum()) * self.d_qk * 2
+
+    def io_bytes(self) -> int:
+        """Algorithmic bytes: q, the kv once, out (16-bit), lse and max_logits, the lists."""
+        rows = self.s_q * self.h_q
+        return self.kv_bytes() + rows * (self.d_qk * 2 + self.dv * 2 + 8) + self.indices.size * 4
+
+
+def make_prefill_problem(s_q: int, h_q: int, s_kv: int, topk: int, *, d_qk: int = 576, dtype: int = BF16,
+                         invalid_frac: float = 0.0, seed: int = 0, name: str = "prefill") -> PrefillProblem:
+    """Seeded sparse-prefill inputs: N(0, 1) q and kv, and for every query token `topk` distinct
+    kv rows drawn uniformly (all of them, shuffled, when s_kv < topk; the rest -1), a random
+    `invalid_frac` of which become -1 or a row past the end."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    q = _normal_bits(rng, (s_q, h_q, d_qk), 1.0, dtype)
+    kv = _normal_bits(rng, (s_kv, 1, d_qk), 1.0, dtype)
+    ind = np.full((s_q, 1, topk), -1, np.int32)
+    n = min(s_kv, topk)
+    for i in range(s_q):
+        ind[i, 0, :n] = rng.choice(s_kv, size=n, replace=False)
+    if invalid_frac > 0:
+        bad = rng.random(ind.shape) < invalid_frac
+        past = s_kv + rng.integers(0, 1000, ind.shape)
+        ind[bad] = np.where(rng.random(ind.shape) < 0.5, -1, past)[bad]
+    return PrefillProblem(name=name, q=q, kv=kv, indices=ind, sm_scale=1.0 / math.sqrt(d_qk), dtype=dtype, seed=seed)
+
+
+PREFILL_WORKLOADS = ("sparse_prefill",)
+
+
+def make_prefill_workload(name: str) -> PrefillProblem:
+    """The sparse-prefill workload: 2048 query tokens of 128 heads, each attending 2048 of 16384
+    kv rows (bf16 N(0, 1), sm_scale 1 / sqrt(576))."""
+    if name != "sparse_prefill":
+        raise KeyError(name)
+    k = len(WORKLOADS) + len(SPARSE_WORKLOADS) + 1
+    return make_prefill_problem(2048, 128, 16384, 2048, seed=1000 + k, name=name)
+
+
 # ----------------------------------------------------------------------------
 # The decode workloads: the five decode configurations, and the compute one over an
 # FP8 cache.  Workload k (1-based position in WORKLOADS) draws from seed 1000 + k.

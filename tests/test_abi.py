@@ -49,10 +49,11 @@ def test_sizes(lib):
     assert b.value == 32 * 2 + 1
     assert lib.mla_metadata_sizes(-1, 128, 1, 74, ctypes.byref(a), ctypes.byref(b)) == 1
     # workspace: a control block of fixed size (status word + 2 int32 counters for each of
-    # up to 16384 virtual batches), then (NV + parts) * 128 * (1 + 512) floats
+    # up to 16384 virtual batches), then (NV + parts) * 128 * (2 + 512) floats
     nv, parts = 64, 74
     control = 256 + 2 * 4 * 16384
-    want = control + ((nv + parts) * 128 * 4 + 255) // 256 * 256 + (nv + parts) * 128 * 512 * 4
+    # split LSEs and split maxima (one float per slot row each), then the split partial outputs
+    want = control + 2 * (((nv + parts) * 128 * 4 + 255) // 256 * 256) + (nv + parts) * 128 * 512 * 4
     assert lib.mla_decode_workspace_bytes(64, 1, 128, 1, 74) == want
     # the same control block for every problem size, so calls of different sizes can share
     # one workspace without one call's partials landing on another's counters
@@ -163,12 +164,11 @@ def _sparse(lib, **over):
 
 @pytest.mark.parametrize("over,code", [
     (dict(indices=None), 1), (dict(topk=-1), 1), (dict(s_q=0), 1), (dict(batch=-1), 1),
-    (dict(dtype=0), 2), (dict(dtype=1), 2), (dict(d_qk=512), 2), (dict(page_size=32), 2), (dict(h_kv=2), 2),
+    (dict(dtype=7), 1), (dict(d_qk=512), 2), (dict(page_size=32), 2), (dict(h_kv=2), 2),
     (dict(ws_bytes=1000), 3), (dict(kvcache=(1 << 20) + 8), 1),
 ])
 def test_sparse_decode_rejects_bad_arguments(lib, over, code):
-    # The sparse decode reads an FP8-with-scale cache through a list of entries: anything else is
-    # rejected on the host before a launch.
+    # Bad lists, sizes or formats are rejected on the host before a launch.
     assert _sparse(lib, **over) == code
 
 
@@ -178,3 +178,23 @@ def test_sparse_metadata_rejects_bad_arguments(lib):
     assert lib.mla_get_metadata_sparse(4, 64, 0, 1, 74, fake, fake, None) == 1
     assert lib.mla_get_metadata_sparse(4, 64, 128, 2, 74, fake, fake, None) == 2
     assert lib.mla_get_metadata_sparse(4, 64, 128, 1, 0, fake, fake, None) == 1
+
+
+def test_sparse_prefill_rejects_bad_arguments(lib):
+    fake = 1 << 20
+    base = dict(q=fake, s_q=4, h_q=128, d_qk=576, kv=fake, s_kv=1000, h_kv=1, indices=fake, topk=64, dv=512, dtype=0,
+                sm_scale=0.0, md=fake, num_parts=74, ns=fake, out=fake, max_logits=fake, lse=fake, ws=fake,
+                ws_bytes=1 << 40, stream=None)
+
+    def call(**over):
+        a = dict(base)
+        a.update(over)
+        return lib.mla_sparse_prefill(*a.values())
+
+    assert call(dtype=2) == 2           # an FP8 cache is the sparse decode's, not the prefill's
+    assert call(dtype=5) == 1
+    assert call(indices=None) == 1 and call(max_logits=None) == 1
+    assert call(s_kv=0) == 1 and call(topk=-1) == 1 and call(s_q=-1) == 1
+    assert call(d_qk=512) == 2 and call(h_kv=2) == 2 and call(dv=256) == 2
+    assert call(ws_bytes=100) == 3
+    assert call(s_q=0, q=None, out=None) == 0
