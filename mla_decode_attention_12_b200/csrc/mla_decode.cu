@@ -778,6 +778,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 }
             } else if constexpr (kSparse) {
                 static_assert(!kFp8, "16-bit rows");
+                if (lane == 0) TL_OPEN(2);
                 // Sparse, 16-bit rows: row i of this CTA's half of "page" blk is entry 64 blk + 32 cta + i.
                 // Lane g < 8 gathers rows 4 g .. 4 g + 3 of every 64-column box (TMA tile::gather4);
                 // an invalid entry names the row just past the tensor, which reads zeros.
@@ -798,6 +799,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                         const int row_next = blk + 1 < hi ? entry(blk + 1) : p.cache_rows;
                         const uint32_t st = ring.stage;
                         if (!(ok = wwait(bar(kBarKEmpty + st), ring.phase ^ 1))) break;
+                        if (lane == 0) TL_EV(kEvKLoad);
                         if (lane == 0 && leader) mbar_arrive_expect_tx(bar(kBarKFull + st), 2 * L::kKBytes);
                         const int g = lane & 7;
                         const int r0 = __shfl_sync(0xffffffffu, row, 4 * g), r1 = __shfl_sync(0xffffffffu, row, 4 * g + 1);
@@ -920,6 +922,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 }
             } else if constexpr (kSparse) {
                 static_assert(!kFp8, "16-bit rows");
+                if (lane == 0) TL_OPEN(4);
                 // ==================== V producer (sparse, 16-bit rows) ====================
                 // The page's 64 entries x this CTA's 4 V boxes, by gather4 (lane g < 16: rows 4 g ..
                 // 4 g + 3); invalid entries read zeros, so nothing needs clearing.
@@ -941,6 +944,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                         const int next_b = more ? entry(kPage * (blk + 1) + 32 + lane) : p.cache_rows;
                         const uint32_t st = ring.stage;
                         if (!(ok = wwait(bar(kBarVEmpty + st), ring.phase ^ 1))) break;
+                        if (lane == 0) TL_EV(kEvVLoad);
                         if (lane == 0 && leader) mbar_arrive_expect_tx(bar(kBarVFull + st), 2 * L::kVBytes);
                         const int g = lane & 15, src = 4 * (g & 7);  // rows 4 g .. 4 g + 3 of the page
                         const int r0a = __shfl_sync(0xffffffffu, row_a, src), r1a = __shfl_sync(0xffffffffu, row_a, src + 1);

@@ -75,22 +75,30 @@ def record(lib, p: W.Problem, launches: int = 6):
     sl = torch.from_numpy(p.cache_seqlens).cuda()
     rows = p.s_q * p.h_q
     parts = mla.num_sm_parts()
-    n_md, n_ns = mla.metadata_sizes(p.batch, rows, 1, parts)
+    sparse = p.indices is not None  # the token-level sparse decode: its own schedule and entry lists
+    tokens = p.batch * p.s_q
+    n_md, n_ns = mla.metadata_sizes(tokens if sparse else p.batch, p.h_q if sparse else rows, 1, parts)
     md = torch.zeros(parts, 8, dtype=torch.int32, device="cuda")
     ns = torch.zeros(n_ns, dtype=torch.int32, device="cuda")
     st = torch.cuda.current_stream().cuda_stream
-    _lib.check(lib.mla_get_metadata(sl.data_ptr(), p.batch, rows, 1, parts, md.data_ptr(), ns.data_ptr(), st),
-               "mla_get_metadata")
-    ws = torch.zeros(mla.workspace_bytes(p.batch, p.s_q, p.h_q, 1, parts), dtype=torch.uint8, device="cuda")
+    if sparse:
+        _lib.check(lib.mla_get_metadata_sparse(tokens, p.indices.shape[2], p.h_q, 1, parts, md.data_ptr(),
+                                               ns.data_ptr(), st), "mla_get_metadata_sparse")
+    else:
+        _lib.check(lib.mla_get_metadata(sl.data_ptr(), p.batch, rows, 1, parts, md.data_ptr(), ns.data_ptr(), st),
+                   "mla_get_metadata")
+    ws_b, ws_s = (tokens, 1) if sparse else (p.batch, p.s_q)
+    ws = torch.zeros(mla.workspace_bytes(ws_b, ws_s, p.h_q, 1, parts), dtype=torch.uint8, device="cuda")
+    ind = torch.from_numpy(p.indices).cuda() if sparse else None
     call = mla.DecodeCall(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale, workspace=ws,
-                          active_heads=p.active_heads, is_fp8_kvcache=p.fp8_kv)
+                          active_heads=p.active_heads, is_fp8_kvcache=p.fp8_kv, indices=ind)
     flush = torch.empty(2 * torch.cuda.get_device_properties(0).L2_cache_size, dtype=torch.uint8, device="cuda")
     us = []
     for _ in range(launches):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        _lib.check(lib.mla_decode_splitkv(*call.args, st), "mla_decode_splitkv")
+        _lib.check((lib.mla_decode_sparse_splitkv if sparse else lib.mla_decode_splitkv)(*call.args, st), "splitkv")
         e1.record()
         _lib.check(lib.mla_decode_combine(*call.combine_args, st), "mla_decode_combine")
         torch.cuda.synchronize()
@@ -194,7 +202,7 @@ def summarize(name: str, per, end: float, kernel_us: float) -> str:
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--workloads", default="compute,spec_padded,long_split,fp16_norope")
+    ap.add_argument("--workloads", default="compute,spec_padded,long_split,fp16_norope,sparse_fp8")
     ap.add_argument("--launches", type=int, default=6)
     ap.add_argument("--save", default=None, help="directory to save the raw event arrays (.npy) in")
     args = ap.parse_args(argv)
