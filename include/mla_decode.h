@@ -26,6 +26,9 @@
  *   - Errors that only the device can see (a block-table entry outside the
  *     cache, a pipeline wait that ran out of time) are recorded in a status
  *     word at the start of the workspace; mla_read_device_status reads it.
+ *     The outputs of a call that recorded one are unspecified: rows may hold
+ *     anything, including what they held before (a cluster that gave up, or a
+ *     combine that stopped waiting once the status word was set, writes nothing).
  *
  * Array layouts (all row-major / C order):
  *   q             [batch, s_q, h_q, d_qk]             bf16 or fp16

@@ -83,13 +83,18 @@ def load() -> ctypes.CDLL:
                 raise ImportError(
                     f"{LIB_PATH} is missing: build it with "
                     "`python -m mla_decode_attention_12_b200.build` (nvcc, sm_100a)")
-            lib = ctypes.CDLL(LIB_PATH)
-            for name, (argtypes, restype) in SIGNATURES.items():
-                fn = getattr(lib, name)
-                fn.argtypes = argtypes
-                fn.restype = restype
-            _lib = lib
+            _lib = bind(LIB_PATH)
     return _lib
+
+
+def bind(path: str) -> ctypes.CDLL:
+    """Open a build of the library at `path` with every entry point's signature set."""
+    lib = ctypes.CDLL(path)
+    for name, (argtypes, restype) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes = argtypes
+        fn.restype = restype
+    return lib
 
 
 def status_string(status: int) -> str:

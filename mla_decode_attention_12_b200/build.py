@@ -31,24 +31,28 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(out: str = LIB) -> bool:
+    if not os.path.exists(out):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(out)
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    """Compile the library if any source is newer than it; returns its path."""
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+def build(force: bool = False, verbose: bool = False, extra=(), out: str = LIB) -> str:
+    """Compile the library if any source is newer than it; returns its path.
+
+    ``extra`` adds nvcc flags and ``out`` names another file: instrumented or test-only
+    builds of the same sources (``-DMLA_TIMELINE``, ``-DMLA_TEST_WITHHOLD_K_PAGE=n``) go
+    to their own files, never to the product library's."""
+    if not force and up_to_date(out):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
     cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-o", tmp, *SOURCES]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

@@ -94,7 +94,11 @@ constexpr int kQTmemBoxes = 6;         // 64-column boxes of Q kept in tensor me
 constexpr int kQBoxesPerRound = 3;     // boxes of Q per round through the Q buffer
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kQPrefetchPages = 8;         // pages before a chunk's end at which the next Q goes to L2
-constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
+// The bound of every pipeline wait (a build may lower it, e.g. for a test of the abort path).
+#ifndef MLA_WAIT_TIMEOUT_NS
+#define MLA_WAIT_TIMEOUT_NS 2000000000ull
+#endif
+constexpr unsigned long long kWaitTimeoutNs = MLA_WAIT_TIMEOUT_NS;
 constexpr int kWorkspaceHeader = 256;
 // The workspace's control block has room for the counters of this many virtual batches
 // (requests x row groups of 128 query rows), whatever the call: its size does not depend on
@@ -821,13 +825,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 Ring<L::kKStages> ring;
                 int vb, lo, hi;
                 bool ok = true;
+#ifdef MLA_TEST_WITHHOLD_K_PAGE
+                // Test-only build: both CTAs of partition 0 never load page MLA_TEST_WITHHOLD_K_PAGE
+                // of their first chunk, so its K_full barrier never completes (a flag that nothing
+                // sets) and the MMA warp's bounded wait on it runs out.
+                bool first_chunk = true;
+#endif
                 while (ok && chunks.next(vb, lo, hi)) {
                     if (hi <= lo) continue;
                     const int b = vb / p.groups;
                     const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+#ifdef MLA_TEST_WITHHOLD_K_PAGE
+                    const int withheld = (part == 0 && first_chunk) ? lo + MLA_TEST_WITHHOLD_K_PAGE : -1;
+                    first_chunk = false;
+#endif
                     for (int blk = lo; blk < hi; ++blk, ring.advance()) {
                         const uint32_t st = ring.stage;
                         if (!(ok = sync.wait(bar(kBarKEmpty + st), ring.phase ^ 1))) break;
+#ifdef MLA_TEST_WITHHOLD_K_PAGE
+                        if (blk == withheld) continue;
+#endif
                         TL_EV(kEvKLoad);
                         const int page = page_of(p, table, blk);
                         if (leader) mbar_arrive_expect_tx(bar(kBarKFull + st), 2 * L::kKBytes);
@@ -1524,6 +1541,9 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
         while (!ready) {
             __nanosleep(200);
             ready = ld_acquire_gpu(split_done) >= want;
+            // A device error recorded by this call (a split-KV cluster that gave up, another
+            // combine CTA that timed out) means the splits may never all come: stop waiting.
+            if (!ready && ld_acquire_gpu(p.status) != 0) break;
             if (!ready && global_timer_ns() - t0 > kWaitTimeoutNs) {
                 atomicCAS(p.status, 0, MLA_ERR_TIMEOUT);
                 break;

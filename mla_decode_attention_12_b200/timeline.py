@@ -39,23 +39,11 @@ EV = dict(setup=1, chunk=2, sfull=4, pposted=5, ofull=6, epidone=7, exit=8, clus
 
 def build_timeline_lib(force: bool = False) -> str:
     """Compile the instrumented copy (same sources, -DMLA_TIMELINE) next to the product library."""
-    if not force and os.path.exists(LIB) and all(os.path.getmtime(d) <= os.path.getmtime(LIB) for d in _build.DEPS):
-        return LIB
-    import subprocess
-
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_build.nvcc(), *_build.NVCC_FLAGS, "-DMLA_TIMELINE", "-I", os.path.join(_build.ROOT, "include"), "-o", tmp,
-           *_build.SOURCES]
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    return _build.build(force=force, extra=["-DMLA_TIMELINE"], out=LIB)
 
 
 def load_timeline_lib() -> ctypes.CDLL:
-    lib = ctypes.CDLL(build_timeline_lib())
-    for name, (argtypes, restype) in _lib.SIGNATURES.items():
-        fn = getattr(lib, name)
-        fn.argtypes, fn.restype = argtypes, restype
+    lib = _lib.bind(build_timeline_lib())
     lib.mla_timeline_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
     lib.mla_timeline_read.restype = ctypes.c_int
     return lib
