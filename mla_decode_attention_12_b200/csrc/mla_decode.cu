@@ -34,9 +34,11 @@
 // * The metadata, split-KV and combine kernels are launched with programmatic launch
 //   overlap.
 // * "FP8 with scale" cache (the kFp8 instantiation, 512 threads): the K producer bulk-copies
-//   this CTA's raw 656-byte rows of each page and the V producer the peer rows' V slices and
-//   scales; two converter warpgroups dequantize them (e4m3 x float32 scale, rounded to
-//   bfloat16) into the same K and V stages, so the MMA, softmax and epilogue are unchanged.
+//   this CTA's raw 656-byte rows of each page; two converter warpgroups dequantize them
+//   (e4m3 x float32 scale, rounded to bfloat16) into the K stage; the V producer assembles
+//   the V stage from both CTAs' K stages with shared-memory bulk copies (its own rows
+//   locally, the peer's over distributed shared memory), so every token row is dequantized
+//   once and the MMA, softmax and epilogue are those of the 16-bit cache.
 //
 // Every mbarrier wait is bounded: after kWaitTimeoutNs the waiting thread sets
 // an abort flag (seen by both CTAs of the cluster) and MLA_ERR_TIMEOUT in the
@@ -71,8 +73,6 @@ constexpr int kConvWarp0 = 8;          // converter warps 8-15
 constexpr int kConvWarps = 8;
 constexpr int kFp8Row = 656;
 constexpr int kRawKBytes = 32 * kFp8Row;       // this CTA's 32 token rows of a page, as stored
-constexpr int kRawVBytes = 2 * 4096 + 512;     // the peer's 32 rows: this CTA's two 128-value latent
-                                               // slices (V columns) and the 4 scales of each row
 // Registers per thread in the FP8 kernel: the launch holds 65536 / 512 = 128 each; the loader /
 // MMA warpgroup and the two converter warpgroups give theirs up to the softmax warpgroup.
 constexpr uint32_t kRegsLaunchFp8 = 128;
@@ -109,7 +109,7 @@ static_assert(kControlBytes % 256 == 0, "split partials start 256-byte aligned")
 constexpr int kNumMaps = 3;  // tensor maps of the split-KV kernel: Q, K, V
 
 // Shared-memory plan of one CTA (each CTA of the pair owns 64 query rows).  The FP8 kernel
-// trades a K stage and a V stage for rings of raw cache rows.
+// trades a K stage for a ring of raw cache rows.
 template <bool kRope, bool kFp8 = false>
 struct Layout {
     static constexpr int kBoxes = kRope ? 9 : 8;               // 64-column boxes in a d_qk row
@@ -120,18 +120,16 @@ struct Layout {
     static constexpr int kKBytes = kBoxes * 4096;              // K: this CTA's 32 tokens of a page x d_qk
     static constexpr int kKStages = kFp8 ? 2 : 3;
     static constexpr int kVBytes = 4 * 8192;                   // V: 64 tokens x this CTA's 256 d_v columns
-    static constexpr int kVStages = kFp8 ? 1 : 2;
+    static constexpr int kVStages = 2;
     static constexpr int kPBytes = 8192;                       // P: 64 rows x 64 tokens, 16-bit
     static constexpr int kKSteps = kBoxes * 4;                 // K=16 MMA steps of Q K^T
-    static constexpr int kRawKStages = kFp8 ? 3 : 0;
-    static constexpr int kRawVStages = kFp8 ? 2 : 0;
+    static constexpr int kRawKStages = kFp8 ? 2 : 0;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;              // kKStages stages
     static constexpr int kOffV = kOffK + kKStages * kKBytes;   // kVStages stages
     static constexpr int kOffP = kOffV + kVStages * kVBytes;   // 2 buffers
     static constexpr int kOffRawK = kOffP + 2 * kPBytes;       // raw rows (FP8 cache only)
-    static constexpr int kOffRawV = kOffRawK + kRawKStages * kRawKBytes;
-    static constexpr int kOffRed = kOffRawV + kRawVStages * kRawVBytes;  // 3 x 128 floats: 2 page row-max halves, row sums
+    static constexpr int kOffRed = kOffRawK + kRawKStages * kRawKBytes;  // 3 x 128 floats: 2 page row-max halves, row sums
     static constexpr int kRedBytes = 3 * 128 * 4;
     static constexpr int kOffBar = kOffRed + kRedBytes;
     static constexpr int kBarBytes = 384;
@@ -153,13 +151,14 @@ enum BarSlot : int {
     kBarDrain = 20,   // leader
     kBarTail = 21,    // both: V load of a sequence's last page (local)
     kBarPair = 22,    // both: 2 slots, rendezvous of softmax warps {w, w ^ 2} (one arrive per warp)
-    // FP8 cache only (kBarKFull / kBarVFull then count the converter warps of both CTAs):
-    kBarRawKFull = 24,   // local, 3 stages: this CTA's raw rows of a page landed
-    kBarRawKEmpty = 27,  // local, 3 stages: the converter warps done with them
-    kBarRawVFull = 30,   // local, 2 stages: the peer rows' V slices and scales landed
-    kBarRawVEmpty = 32,  // local, 2 stages
+    // FP8 cache only (kBarKFull then counts the converter warps of both CTAs):
+    kBarRawKFull = 24,   // local, 2 stages: this CTA's raw rows of a page landed
+    kBarRawKEmpty = 27,  // local, 2 stages: the converter warps done with them
+    kBarKConv = 30,      // local, 2 K stages: this CTA's converter warps wrote the stage
+    kBarKCopied = 32,    // local, 2 K stages: the V copies out of the stage landed (own + peer's view)
     kBarQCopied = 34,    // both: a round of Q boxes copied from the Q buffer into tensor memory
-    kBarCount = 35
+    kBarVLand = 35,      // local, 2 V stages (FP8 cache): this CTA's V stage copies landed (bytes)
+    kBarCount = 37
 };
 
 // Position in a ring of kN stages: stage index and the parity of its current use.
@@ -177,8 +176,7 @@ struct Ring {
 constexpr int kOffTmemSlot = kBarCount * 8;  // uint32 written by tcgen05.alloc
 constexpr int kOffAbort = kOffTmemSlot + 4;  // int abort flag
 constexpr int kOffMaskK = kOffAbort + 4;     // sparse decode: validity bits of the raw K stages' 32 rows
-constexpr int kOffMaskV = kOffMaskK + 4 * 3; // ... and of the raw V stages' 32 (peer) rows
-static_assert(kOffMaskV + 4 * 2 <= Layout<true>::kBarBytes, "barrier area too small");
+static_assert(kOffMaskK + 4 * Layout<true, true>::kRawKStages <= Layout<true>::kBarBytes, "barrier area too small");
 static_assert(2 * Layout<true>::kPBytes >= 4 * 4096 && 2 * Layout<false>::kPBytes >= 4 * 4096,
               "epilogue staging (4 KB per softmax warp) must fit in the P buffers");
 static_assert(kTmemQ + 8 * 4 * kQTmemBoxes == kTmemCols, "tensor memory plan");
@@ -190,7 +188,7 @@ static_assert(Layout<true>::kSmemBytes <= 232448 && Layout<false>::kSmemBytes <=
               "shared memory plan exceeds 227 KB");
 static_assert(Layout<true, true>::kOffK % 1024 == 0 && Layout<true, true>::kOffV % 1024 == 0 &&
                   Layout<true, true>::kOffP % 1024 == 0 && Layout<true, true>::kOffRawK % 128 == 0 &&
-                  Layout<true, true>::kOffRawV % 128 == 0 && kRawKBytes % 128 == 0 && kRawVBytes % 128 == 0,
+                  kRawKBytes % 128 == 0,
               "FP8 kernel: operand tiles 1024-byte aligned, raw rows 128-byte aligned");
 static_assert(Layout<true>::kOffQ % 1024 == 0 && Layout<true>::kOffK % 1024 == 0 && Layout<true>::kOffV % 1024 == 0 &&
                   Layout<true>::kOffP % 1024 == 0 && Layout<false>::kOffK % 1024 == 0 &&
@@ -405,7 +403,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
     const uint32_t s_bar = s_base + L::kOffBar;
     float* red = reinterpret_cast<float*>(smem + L::kOffRed);
     volatile uint32_t* mask_k = reinterpret_cast<volatile uint32_t*>(smem + L::kOffBar + kOffMaskK);
-    volatile uint32_t* mask_v = reinterpret_cast<volatile uint32_t*>(smem + L::kOffBar + kOffMaskV);
     [[maybe_unused]] Timeline tl;
 #ifdef MLA_TIMELINE
     const uint64_t tl_start = global_timer_ns();
@@ -443,12 +440,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             mbar_init(bar(kBarRawKFull + s), 1);
             mbar_init(bar(kBarRawKEmpty + s), kConvWarps);
         }
-        for (int s = 0; s < L::kRawVStages; ++s) {
-            mbar_init(bar(kBarRawVFull + s), 1);
-            mbar_init(bar(kBarRawVEmpty + s), kConvWarps);
+        if constexpr (kFp8) {
+            for (int s = 0; s < L::kKStages; ++s) {
+                mbar_init(bar(kBarKConv + s), kConvWarps);
+                mbar_init(bar(kBarKCopied + s), 2);  // this CTA's V producer and the peer's
+            }
+            for (int s = 0; s < L::kVStages; ++s) mbar_init(bar(kBarVLand + s), 1);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(kBarVFull + s), kFp8 ? 2 * kConvWarps : 2);  // 16-bit: one V producer per CTA
+            mbar_init(bar(kBarVFull + s), 2);  // the V producers of both CTAs
             mbar_init(bar(kBarVEmpty + s), 1);
             mbar_init(bar(kBarSFull + s), 1);
             mbar_init(bar(kBarPFull + s), 8);
@@ -497,24 +497,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
 
     if (kFp8 && warp >= kConvWarp0) {
         // ============================ converters (FP8 cache) ============================
-        // Eight warps per CTA dequantize the raw rows into the bfloat16 K and V stages the
-        // MMAs read, in the layout TMA gives the 16-bit cache (SW128 boxes of 64 columns):
-        //   K(g): this CTA's 32 rows of page g, all 576 columns: latent value i becomes
-        //         bf16(e4m3_i * scale_{i/128}) (the product in float32, then rounded to
-        //         nearest even), the 64 RoPE values are copied;
-        //   V(g): the page's 64 rows x this CTA's 256 V columns: its own 32 rows copied from
-        //         K(g), the peer's 32 rows dequantized from their raw slices; rows past the
-        //         sequence end are zero so that P = 0 never meets NaN.
-        // K runs one page ahead of V (K(g) then V(g - 1)), in the order the MMA issuer
-        // consumes them (Q K^T of page g before P V of page g - 1).  Warp cw owns the 16-byte
-        // words 2 cq and 2 cq + 1 (cq = cw & 3) of K boxes [4 ch, 4 ch + 4) (ch = cw >> 2) in every
-        // row `lane`, and copies exactly those words into V.
+        // Eight warps per CTA dequantize this CTA's 32 raw rows of each page into the bfloat16 K
+        // stage the MMAs read, in the layout TMA gives the 16-bit cache (SW128 boxes of 64
+        // columns): latent value i becomes bf16(e4m3_i * scale_{i/128}) (the product in float32,
+        // then rounded to nearest even), the 64 RoPE values are copied.  Rows that are not
+        // visible (past the sequence end, invalid sparse entries) are written as zeros: the V
+        // stages are copied from these rows, and P = 0 must never meet NaN there.  Warp cw owns
+        // the 16-byte words 2 cq and 2 cq + 1 (cq = cw & 3) of K boxes [4 ch, 4 ch + 4)
+        // (ch = cw >> 2) in every row `lane`.
         set_max_registers<kRegsLaunchFp8, kRegsConvFp8>();
         const int cw = warp - kConvWarp0;
         const int cq = cw & 3, ch = cw >> 2;
         const int sw = lane & 7;  // swizzle phase of row `lane` (and of every row congruent mod 8)
         const uint32_t k_full_lead[2] = {lead_bar(kBarKFull), lead_bar(kBarKFull + 1)};
-        const uint32_t v_full_lead = lead_bar(kBarVFull);
         auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
         // 16 e4m3 values (one 16-byte word) times `s` -> 16 bfloat16 values (two 16-byte words).
         // Two values at a time: e4m3 -> half (exact: every e4m3 value, subnormals and NaN
@@ -536,108 +531,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             word(raw.z, hi.x, hi.y);
             word(raw.w, hi.z, hi.w);
         };
-        // Each converter warp makes its writes visible to the tensor core and arrives on the
-        // even CTA's barrier (16 arrivals: 8 warps x 2 CTAs).
-        auto publish = [&](uint32_t lead) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                if (leader)
-                    mbar_arrive(lead);
-                else
-                    mbar_arrive_remote(lead);
-            }
-        };
         Ring<L::kKStages> kring;
         Ring<L::kRawKStages> rk;
-        Ring<L::kRawVStages> rv;
-        uint32_t gv = 0;              // pages whose V stage has been filled
-        bool pending = false;         // a page waits for its V stage
-        uint32_t own_live = 0, peer_live = 0;  // its rows that are visible: bit i = own / peer row i
-        uint32_t prev_kstage = 0;
         bool ok = true;
-        // V stage of the previous page: own rows from its K stage, the peer's from raw slices;
-        // rows not visible (past the sequence end, or invalid sparse entries) are zero.
-        auto fill_v = [&]() -> bool {
-            if (!wwait(bar(kBarRawVFull + rv.stage), rv.phase)) return false;
-            if constexpr (kSparse) peer_live = mask_v[rv.stage];
-            if (!wwait(bar(kBarVEmpty), (gv & 1) ^ 1)) return false;
-            uint8_t* vst = smem + L::kOffV;
-            const uint8_t* kst = smem + L::kOffK + prev_kstage * L::kKBytes;
-            const int own0 = 32 * static_cast<int>(cta), peer0 = 32 - own0;
-            // All loads first, then the stores (as for K).  V box jv holds K box
-            // 4 (jv >> 1) + 2 cta + (jv & 1): this warp's own-row words are in V boxes 2 ch, 2 ch + 1.
-            const int kk = ch;  // peer rows: slice kk holds V columns [256 kk + 128 cta, +128)
-            const int chunk8 = lane & 7;
-            const uint8_t* rawv = smem + L::kOffRawV + rv.stage * kRawVBytes;
-            uint4 own[4], peer[2];
-            float ps[2];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {  // own rows: the 16-byte words this warp wrote into K(g)
-                const int jv = 2 * ch + (i >> 1), gbox = 4 * ch + 2 * static_cast<int>(cta) + (jv & 1);
-                own[i] = *reinterpret_cast<const uint4*>(kst + gbox * 4096 + lane * 128 + (((2 * cq + (i & 1)) ^ sw) << 4));
-            }
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int t = 8 * cq + 4 * m + (lane >> 3);
-                peer[m] = *reinterpret_cast<const uint4*>(rawv + kk * 4096 + t * 128 + chunk8 * 16);
-                ps[m] = *reinterpret_cast<const float*>(rawv + 8192 + t * 16 + 4 * (2 * kk + static_cast<int>(cta)));
-            }
-            {
-                const int tok = own0 + lane;
-                const bool live = (own_live >> lane) & 1u;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int jv = 2 * ch + (i >> 1);
-                    *reinterpret_cast<uint4*>(vst + jv * 8192 + tok * 128 + (((2 * cq + (i & 1)) ^ sw) << 4)) =
-                        live ? own[i] : make_uint4(0, 0, 0, 0);
-                }
-            }
-            {
-                const int jv = 2 * kk + (chunk8 >> 2);
-                const int c0 = 2 * (chunk8 & 3);
-#pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    const int t_peer = 8 * cq + 4 * m + (lane >> 3), tok = peer0 + t_peer;
-                    uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-                    if ((peer_live >> t_peer) & 1u) dequant16(peer[m], ps[m], lo, hi);
-                    uint8_t* row = vst + jv * 8192 + tok * 128;
-                    *reinterpret_cast<uint4*>(row + ((c0 ^ (tok & 7)) << 4)) = lo;
-                    *reinterpret_cast<uint4*>(row + (((c0 + 1) ^ (tok & 7)) << 4)) = hi;
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarRawVEmpty + rv.stage));
-            publish(v_full_lead);
-            rv.advance();
-            ++gv;
-            pending = false;
-            return true;
-        };
         int vb, lo, hi;
         while (ok && chunks.next(vb, lo, hi)) {
             if (hi <= lo) continue;
             const int Lb = request_len(p.seqlens, p.topk, vb / p.groups);
-            for (int blk = lo; blk < hi && ok; ++blk) {
-                // ---- K(g): this CTA's 32 rows
+            for (int blk = lo; blk < hi && ok; ++blk, rk.advance(), kring.advance()) {
                 if (!(ok = wwait(bar(kBarRawKFull + rk.stage), rk.phase))) break;
-                // visible rows of page g (read before the raw stage is handed back)
-                uint32_t own_g, peer_g = 0;
+                // this CTA's visible rows of the page (read before the raw stage is handed back)
+                uint32_t live_bits;
                 if constexpr (kSparse) {
-                    own_g = mask_k[rk.stage];
+                    live_bits = mask_k[rk.stage];
                 } else {
-                    const int valid = min(kPage, Lb - kPage * blk);  // rows [0, valid) of the page
-                    auto half_bits = [&](int first) {
-                        const int c = min(max(valid - first, 0), 32);
-                        return c >= 32 ? 0xffffffffu : ((1u << c) - 1u);
-                    };
-                    own_g = half_bits(32 * static_cast<int>(cta));
-                    peer_g = half_bits(32 - 32 * static_cast<int>(cta));
+                    const int c = min(max(min(kPage, Lb - kPage * blk) - 32 * static_cast<int>(cta), 0), 32);
+                    live_bits = c >= 32 ? 0xffffffffu : ((1u << c) - 1u);
                 }
+                // The stage is free once the Q K^T MMAs of its previous page and the V copies out
+                // of it (this CTA's and the peer's) are done.
                 if (!(ok = wwait(bar(kBarKEmpty + kring.stage), kring.phase ^ 1))) break;
+                if (!(ok = wwait(bar(kBarKCopied + kring.stage), kring.phase ^ 1))) break;
                 {
+                    const bool live = (live_bits >> lane) & 1u;
                     const uint8_t* rrow = smem + L::kOffRawK + rk.stage * kRawKBytes + lane * kFp8Row;
                     uint8_t* krow = smem + L::kOffK + kring.stage * L::kKBytes + lane * 128;
+                    const uint4 zero = make_uint4(0, 0, 0, 0);
                     const uint4 rope = *reinterpret_cast<const uint4*>(rrow + 528 + 16 * cw);
                     const float2 sc = *reinterpret_cast<const float2*>(rrow + 512 + 8 * ch);  // boxes 4 ch .. 4 ch + 3
                     // Two boxes per iteration: a smaller loop body keeps the instruction cache warm for
@@ -649,25 +568,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                         dequant16(*reinterpret_cast<const uint4*>(rrow + 64 * (4 * ch + m) + 16 * cq), m < 2 ? sc.x : sc.y,
                                   w0, w1);
                         uint8_t* box = krow + (4 * ch + m) * 4096;
-                        *reinterpret_cast<uint4*>(box + (((2 * cq) ^ sw) << 4)) = w0;
-                        *reinterpret_cast<uint4*>(box + (((2 * cq + 1) ^ sw) << 4)) = w1;
+                        *reinterpret_cast<uint4*>(box + (((2 * cq) ^ sw) << 4)) = live ? w0 : zero;
+                        *reinterpret_cast<uint4*>(box + (((2 * cq + 1) ^ sw) << 4)) = live ? w1 : zero;
                     }
-                    *reinterpret_cast<uint4*>(krow + 8 * 4096 + ((cw ^ sw) << 4)) = rope;  // RoPE: box 8, copied
+                    *reinterpret_cast<uint4*>(krow + 8 * 4096 + ((cw ^ sw) << 4)) = live ? rope : zero;  // RoPE: box 8
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(kBarRawKEmpty + rk.stage));
-                publish(k_full_lead[kring.stage]);
-                rk.advance();
-                // ---- V(g - 1)
-                if (pending && !(ok = fill_v())) break;
-                pending = true;
-                own_live = own_g;
-                peer_live = peer_g;  // (the sparse decode reads it with the raw V stage)
-                prev_kstage = kring.stage;
-                kring.advance();
+                // Visible to the tensor core and to the bulk copies (async proxy): arrive on the even
+                // CTA's K_full (16 arrivals: 8 warps x 2 CTAs) and on this CTA's K_conv.
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader)
+                        mbar_arrive(k_full_lead[kring.stage]);
+                    else
+                        mbar_arrive_remote(k_full_lead[kring.stage]);
+                    mbar_arrive(bar(kBarKConv + kring.stage));
+                }
             }
         }
-        if (ok && pending) ok = fill_v();
     } else if (warp >= 4) {
         // Warpgroup 1 (Q / K / V loaders and the MMA issuer): one thread issues; few registers.
         if constexpr (kFp8) set_max_registers<kRegsLaunchFp8, kRegsLoadersFp8>();  // before the role split: one
@@ -861,78 +781,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 }
             }
         } else if (warp == kVWarp) {
-            if constexpr (kSparse && kFp8) {
-                static_assert(L::kRawVStages > 0, "the FP8 layout's raw ring");
-                // ===================== V producer (sparse decode, FP8 cache) =====================
-                // The peer's 32 rows of "page" blk (entries 64 blk + 32 (1 - cta) + i): lane i copies
-                // this CTA's two 128-byte latent slices (its V columns) and the 16 bytes of scales
-                // of its row when the entry is valid, in the layout the TMA boxes give the dense
-                // decode; lane 0 records the validity bits with the stage.
-                Ring<L::kRawVStages> ring;
-                int vb, lo, hi;
-                bool ok = true;
-                const uint8_t* kv = static_cast<const uint8_t*>(p.kvcache);
-                auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
-                while (ok && chunks.next(vb, lo, hi)) {
-                    if (hi <= lo) continue;
-                    const int32_t* ent = p.indices + static_cast<size_t>(vb / p.groups) * p.topk;
-                    auto entry = [&](int blk) {
-                        const int e = kPage * blk + 32 * (1 - static_cast<int>(cta)) + lane;
-                        return e < p.topk ? __ldg(ent + e) : -1;
-                    };
-                    int idx = entry(lo);
-                    for (int blk = lo; blk < hi; ++blk, ring.advance()) {
-                        const int idx_next = blk + 1 < hi ? entry(blk + 1) : -1;
-                        const uint32_t st = ring.stage;
-                        if (!(ok = wwait(bar(kBarRawVEmpty + st), ring.phase ^ 1))) break;
-                        const bool valid = idx >= 0 && idx < p.cache_rows;
-                        const uint32_t mask = __ballot_sync(0xffffffffu, valid);
-                        if (lane == 0) {
-                            mask_v[st] = mask;
-                            mbar_arrive_expect_tx(bar(kBarRawVFull + st), __popc(mask) * (2 * 128 + 16));
-                        }
-                        __syncwarp();
-                        if (valid) {
-                            const uint8_t* row = kv + static_cast<size_t>(idx) * kFp8Row;
-                            const uint32_t dst = s_base + L::kOffRawV + st * kRawVBytes;
-                            bulk_load(dst + lane * 128, row + 128 * cta, 128, bar(kBarRawVFull + st));
-                            bulk_load(dst + 4096 + lane * 128, row + 256 + 128 * cta, 128, bar(kBarRawVFull + st));
-                            bulk_load(dst + 8192 + lane * 16, row + 512, 16, bar(kBarRawVFull + st));
-                        }
-                        idx = idx_next;
-                    }
-                }
-                if (!ok && lane == 0) {
-                    const uint64_t t0 = global_timer_ns();  // let issued loads land (see below)
-                    while (global_timer_ns() - t0 < 50000000ull) {
-                    }
-                }
-            } else if constexpr (kFp8) {
+            if constexpr (kFp8) {
                 // ============================ V producer (FP8 cache) ============================
-                // The peer's 32 rows of each page: this CTA's two 128-value latent slices (its V
-                // columns) and the rows' scales, by TMA (tm_k: 128-byte boxes, tm_v: 16-byte boxes).
+                // V(g) is the page's 64 tokens x this CTA's 256 d_v columns.  Its own 32 rows are
+                // in its K stage of page g, the peer's 32 rows in the peer's (the same dequantized
+                // bytes: every row is converted once).  V box jv holds K box 4 (jv >> 1) + 2 cta +
+                // (jv & 1); a K box's 32 rows are 4 KB of whole SW128 rows whose swizzle phase (row
+                // mod 8) is the same at token 32 c + row of the V box, so lane 0 moves each half
+                // with 4 shared-memory bulk copies: into its own V stage, and into the peer's over
+                // distributed shared memory, each completing on the receiving CTA's V_land.  Once
+                // its V_land completes (its copies and the peer's into it), it hands the stage to
+                // the MMA (the even CTA's V_full) and the K stage back to both CTAs' converters.
                 if (lane == 0) {
-                    Ring<L::kRawVStages> ring;
+                    TL_OPEN(4);
+                    Ring<L::kKStages> kring;
+                    uint32_t g = 0;
                     int vb, lo, hi;
                     bool ok = true;
+                    const uint32_t peer = cta ^ 1u;
+                    const uint32_t own_rows = 32u * cta * 128u;  // byte offset of this CTA's tokens in a V box
                     while (ok && chunks.next(vb, lo, hi)) {
                         if (hi <= lo) continue;
-                        const int b = vb / p.groups;
-                        const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-                        for (int blk = lo; blk < hi; ++blk, ring.advance()) {
-                            const uint32_t st = ring.stage;
-                            if (!(ok = sync.wait(bar(kBarRawVEmpty + st), ring.phase ^ 1))) break;
-                            const int page = page_of(p, table, blk);
-                            const int y = page * kPage + 32 * (1 - static_cast<int>(cta));
-                            const uint32_t dst = s_base + L::kOffRawV + st * kRawVBytes;
-                            mbar_arrive_expect_tx(bar(kBarRawVFull + st), kRawVBytes);
-                            tma_load_2d(dst, &tm_k, bar(kBarRawVFull + st), 128 * static_cast<int>(cta), y);
-                            tma_load_2d(dst + 4096, &tm_k, bar(kBarRawVFull + st), 256 + 128 * static_cast<int>(cta), y);
-                            tma_load_2d(dst + 8192, &tm_v, bar(kBarRawVFull + st), 512, y);
+                        for (int blk = lo; blk < hi; ++blk, ++g, kring.advance()) {
+                            const uint32_t vs = g & 1, vph = (g >> 1) & 1;
+                            if (!(ok = sync.wait(bar(kBarKConv + kring.stage), kring.phase))) break;
+                            if (!(ok = sync.wait(bar(kBarVEmpty + vs), vph ^ 1))) break;
+                            TL_EV(kEvVLoad);
+                            // (the peer's stage vs is free too: the same MMA commit arrives on both CTAs)
+                            mbar_arrive_expect_tx(bar(kBarVLand + vs), 2 * 4 * 4096);
+                            const uint32_t kst = s_k + kring.stage * L::kKBytes;
+                            const uint32_t vdst = s_v + vs * L::kVBytes + own_rows;
+                            const uint32_t peer_land = map_to_cta(bar(kBarVLand + vs), peer);
+                            for (int jv = 0; jv < 4; ++jv) {
+                                const int mine = 4 * (jv >> 1) + 2 * static_cast<int>(cta) + (jv & 1);
+                                const int theirs = 4 * (jv >> 1) + 2 * static_cast<int>(peer) + (jv & 1);
+                                bulk_copy_s2c(vdst + jv * 8192, kst + mine * 4096, 4096, bar(kBarVLand + vs));
+                                bulk_copy_s2c(map_to_cta(vdst + jv * 8192, peer), kst + theirs * 4096, 4096, peer_land);
+                            }
+                            if (!(ok = sync.wait(bar(kBarVLand + vs), vph))) break;
+                            // This CTA's copies and the peer's into it have landed: the copies out of
+                            // this K stage are done, and so are the peer's out of its own.
+                            mbar_arrive(bar(kBarKCopied + kring.stage));
+                            mbar_arrive_remote(map_to_cta(bar(kBarKCopied + kring.stage), peer));
+                            if (leader)
+                                mbar_arrive(bar(kBarVFull + vs));
+                            else
+                                mbar_arrive_remote(lead_bar(kBarVFull + vs));
                         }
                     }
                     if (!ok) {
-                        const uint64_t t0 = global_timer_ns();  // let issued loads land (see below)
+                        const uint64_t t0 = global_timer_ns();  // let issued copies land (see below)
                         while (global_timer_ns() - t0 < 50000000ull) {
                         }
                     }

@@ -155,6 +155,16 @@ __device__ __forceinline__ void tma_prefetch_3d(const void* map, int x, int y, i
 
 // Bulk copy of `bytes` contiguous bytes (a multiple of 16, both addresses 16-byte
 // aligned) from global memory into this CTA's shared memory, completing on an mbarrier.
+// Bulk copy of `bytes` (a multiple of 16) between shared memories of the cluster: from this
+// CTA's `src` to `dst` (this CTA's or another's, shared::cluster address), completing as
+// transaction bytes on the mbarrier `bar` in the destination CTA.
+__device__ __forceinline__ void bulk_copy_s2c(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
 {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
