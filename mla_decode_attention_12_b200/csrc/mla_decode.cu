@@ -247,6 +247,11 @@ enum TimelineEvent : uint32_t {
     kEvVLoad = 20,      // V producer: a V stage free, its loads issued
     kEvVTailLanded = 21,  // V producer: the V tile of a sequence's last page landed (before zeroing)
     kEvVTailDone = 22,    // V producer: its rows past the sequence end zeroed and the stage handed over
+    kEvConvStart = 23,    // FP8 converter warp 0 (in the K producer's slice): raw rows and K stage ready
+    kEvConvDone = 24,     // FP8 converter warp 0: its part of the K stage written and published
+    kEvConvRaw = 25,      // FP8 converter warp 0: the page's raw rows landed
+    kEvVLanded = 26,      // FP8 V producer: this CTA's V stage copies (its own and the peer's) landed
+    kEvVKConv = 27,       // FP8 V producer: all converter warps of this CTA wrote the K stage
 };
 #ifdef MLA_TIMELINE
 constexpr int kTlCtaWords = 1024;  // per CTA: 2 words of start time, then the roles' slices
@@ -361,12 +366,20 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, bool fp16)
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ int page_of(const DecodeParams& p, const int32_t* table, int blk)
+// Block-table entry of page blk of a request (-1 past max_blocks).  The producers read it one
+// page ahead of its use, so that its latency overlaps their wait for a free stage.
+__device__ __forceinline__ int table_entry(const DecodeParams& p, const int32_t* table, int blk)
 {
-    int page = blk < p.max_blocks ? __ldg(table + blk) : -1;
+    return blk < p.max_blocks ? __ldg(table + blk) : -1;
+}
+
+// The cache page of a block-table entry: one outside the cache is recorded in the status word
+// and replaced by page 0, so that every load stays inside the cache.
+__device__ __forceinline__ int checked_page(const DecodeParams& p, int page)
+{
     if (page < 0 || page >= p.num_blocks) {
         atomicCAS(p.status, 0, MLA_ERR_DEVICE_CHECK);
-        page = 0;  // keep every load inside the cache; the status word reports the error
+        page = 0;
     }
     return page;
 }
@@ -509,8 +522,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         const int cw = warp - kConvWarp0;
         const int cq = cw & 3, ch = cw >> 2;
         const int sw = lane & 7;  // swizzle phase of row `lane` (and of every row congruent mod 8)
-        const uint32_t k_full_lead[2] = {lead_bar(kBarKFull), lead_bar(kBarKFull + 1)};
+        const uint32_t k_full_lead = lead_bar(kBarKFull);  // + 8 per stage (slots are 8 bytes apart)
         auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
+        const bool tl_conv = (cw == 0 && lane == 0);
+        if (tl_conv) TL_OPEN(2);
         // 16 e4m3 values (one 16-byte word) times `s` -> 16 bfloat16 values (two 16-byte words).
         // Two values at a time: e4m3 -> half (exact: every e4m3 value, subnormals and NaN
         // included, is a half), half -> float32 (exact), one packed float32 multiply by s (the
@@ -540,6 +555,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
             const int Lb = request_len(p.seqlens, p.topk, vb / p.groups);
             for (int blk = lo; blk < hi && ok; ++blk, rk.advance(), kring.advance()) {
                 if (!(ok = wwait(bar(kBarRawKFull + rk.stage), rk.phase))) break;
+                if (tl_conv) TL_EV(kEvConvRaw);
                 // this CTA's visible rows of the page (read before the raw stage is handed back)
                 uint32_t live_bits;
                 if constexpr (kSparse) {
@@ -552,6 +568,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 // of it (this CTA's and the peer's) are done.
                 if (!(ok = wwait(bar(kBarKEmpty + kring.stage), kring.phase ^ 1))) break;
                 if (!(ok = wwait(bar(kBarKCopied + kring.stage), kring.phase ^ 1))) break;
+                if (tl_conv) TL_EV(kEvConvStart);
                 {
                     const bool live = (live_bits >> lane) & 1u;
                     const uint8_t* rrow = smem + L::kOffRawK + rk.stage * kRawKBytes + lane * kFp8Row;
@@ -559,19 +576,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     const uint4 zero = make_uint4(0, 0, 0, 0);
                     const uint4 rope = *reinterpret_cast<const uint4*>(rrow + 528 + 16 * cw);
                     const float2 sc = *reinterpret_cast<const float2*>(rrow + 512 + 8 * ch);  // boxes 4 ch .. 4 ch + 3
-                    // Two boxes per iteration: a smaller loop body keeps the instruction cache warm for
-                    // the other warp roles, and the other converter warp of the scheduler hides the
-                    // load latency.
-#pragma unroll 2
+                    // One box per iteration: a small loop body keeps the instruction cache warm for
+                    // the other warp roles (measured faster than unrolling), and the other converter
+                    // warp of the scheduler hides the load latency.
+#pragma unroll 1
                     for (int m = 0; m < 4; ++m) {  // box 4 ch + m: latent columns [64 (4 ch + m), +64); 16 of them
                         uint4 w0, w1;
                         dequant16(*reinterpret_cast<const uint4*>(rrow + 64 * (4 * ch + m) + 16 * cq), m < 2 ? sc.x : sc.y,
                                   w0, w1);
                         uint8_t* box = krow + (4 * ch + m) * 4096;
-                        *reinterpret_cast<uint4*>(box + (((2 * cq) ^ sw) << 4)) = live ? w0 : zero;
-                        *reinterpret_cast<uint4*>(box + (((2 * cq + 1) ^ sw) << 4)) = live ? w1 : zero;
+                        *reinterpret_cast<uint4*>(box + (((2 * cq) ^ sw) << 4)) = w0;
+                        *reinterpret_cast<uint4*>(box + (((2 * cq + 1) ^ sw) << 4)) = w1;
                     }
-                    *reinterpret_cast<uint4*>(krow + 8 * 4096 + ((cw ^ sw) << 4)) = live ? rope : zero;  // RoPE: box 8
+                    *reinterpret_cast<uint4*>(krow + 8 * 4096 + ((cw ^ sw) << 4)) = rope;  // RoPE: box 8
+                    if (!live) {  // rare (a sequence's last page, invalid sparse entries): zeros over the row
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            uint8_t* box = krow + (4 * ch + m) * 4096;
+                            *reinterpret_cast<uint4*>(box + (((2 * cq) ^ sw) << 4)) = zero;
+                            *reinterpret_cast<uint4*>(box + (((2 * cq + 1) ^ sw) << 4)) = zero;
+                        }
+                        *reinterpret_cast<uint4*>(krow + 8 * 4096 + ((cw ^ sw) << 4)) = zero;
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(kBarRawKEmpty + rk.stage));
@@ -581,11 +607,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 __syncwarp();
                 if (lane == 0) {
                     if (leader)
-                        mbar_arrive(k_full_lead[kring.stage]);
+                        mbar_arrive(k_full_lead + 8u * kring.stage);
                     else
-                        mbar_arrive_remote(k_full_lead[kring.stage]);
+                        mbar_arrive_remote(k_full_lead + 8u * kring.stage);
                     mbar_arrive(bar(kBarKConv + kring.stage));
                 }
+                if (tl_conv) TL_EV(kEvConvDone);
             }
         }
     } else if (warp >= 4) {
@@ -684,10 +711,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                         if (hi <= lo) continue;
                         const int b = vb / p.groups;
                         const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-                        for (int blk = lo; blk < hi; ++blk, ring.advance()) {
+                        int entry = table_entry(p, table, lo), entry_next = 0;
+                        for (int blk = lo; blk < hi; ++blk, ring.advance(), entry = entry_next) {
+                            entry_next = blk + 1 < hi ? table_entry(p, table, blk + 1) : 0;
                             const uint32_t st = ring.stage;
                             if (!(ok = sync.wait(bar(kBarRawKEmpty + st), ring.phase ^ 1))) break;
-                            const int page = page_of(p, table, blk);
+                            const int page = checked_page(p, entry);
                             mbar_arrive_expect_tx(bar(kBarRawKFull + st), kRawKBytes);
                             bulk_load(s_base + L::kOffRawK + st * kRawKBytes,
                                       kv + (static_cast<size_t>(page) * kPage + 32 * cta) * kFp8Row, kRawKBytes,
@@ -759,14 +788,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     const int withheld = (part == 0 && first_chunk) ? lo + MLA_TEST_WITHHOLD_K_PAGE : -1;
                     first_chunk = false;
 #endif
-                    for (int blk = lo; blk < hi; ++blk, ring.advance()) {
+                    int entry = table_entry(p, table, lo), entry_next = 0;
+                    for (int blk = lo; blk < hi; ++blk, ring.advance(), entry = entry_next) {
+                        entry_next = blk + 1 < hi ? table_entry(p, table, blk + 1) : 0;
                         const uint32_t st = ring.stage;
                         if (!(ok = sync.wait(bar(kBarKEmpty + st), ring.phase ^ 1))) break;
 #ifdef MLA_TEST_WITHHOLD_K_PAGE
                         if (blk == withheld) continue;
 #endif
                         TL_EV(kEvKLoad);
-                        const int page = page_of(p, table, blk);
+                        const int page = checked_page(p, entry);
                         if (leader) mbar_arrive_expect_tx(bar(kBarKFull + st), 2 * L::kKBytes);
                         const uint32_t dst = s_k + st * L::kKBytes;
                         for (int i = 0; i < L::kBoxes; ++i)
@@ -805,6 +836,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                         for (int blk = lo; blk < hi; ++blk, ++g, kring.advance()) {
                             const uint32_t vs = g & 1, vph = (g >> 1) & 1;
                             if (!(ok = sync.wait(bar(kBarKConv + kring.stage), kring.phase))) break;
+                            TL_EV(kEvVKConv);
                             if (!(ok = sync.wait(bar(kBarVEmpty + vs), vph ^ 1))) break;
                             TL_EV(kEvVLoad);
                             // (the peer's stage vs is free too: the same MMA commit arrives on both CTAs)
@@ -819,6 +851,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                                 bulk_copy_s2c(map_to_cta(vdst + jv * 8192, peer), kst + theirs * 4096, 4096, peer_land);
                             }
                             if (!(ok = sync.wait(bar(kBarVLand + vs), vph))) break;
+                            TL_EV(kEvVLanded);
                             // This CTA's copies and the peer's into it have landed: the copies out of
                             // this K stage are done, and so are the peer's out of its own.
                             mbar_arrive(bar(kBarKCopied + kring.stage));
@@ -908,11 +941,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     const int tail = Lb % kPage;
                     const int last_page = pages_of(Lb) - 1;
                     const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-                    for (int blk = lo; blk < hi; ++blk, ++g) {
+                    int entry = table_entry(p, table, lo), entry_next = 0;
+                    for (int blk = lo; blk < hi; ++blk, ++g, entry = entry_next) {
+                        entry_next = blk + 1 < hi ? table_entry(p, table, blk + 1) : 0;
                         const uint32_t st = g & 1;
                         if (!(ok = wwait(bar(kBarVEmpty + st), ((g >> 1) & 1) ^ 1))) break;
                         if (lane == 0) TL_EV(kEvVLoad);
-                        const int page = page_of(p, table, blk);
+                        const int page = checked_page(p, entry);
                         const uint32_t dst = s_v + st * L::kVBytes;
                         const bool is_tail = (blk == last_page) && tail != 0;
                         if (!is_tail) {
@@ -1086,7 +1121,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         const uint32_t pair_bar = bar(kBarPair + (warp & 1));  // rendezvous of warps {w, w ^ 2}
         uint32_t pair_phase = 0;
-        const uint32_t p_full_lead[2] = {lead_bar(kBarPFull), lead_bar(kBarPFull + 1)};
+        const uint32_t p_full_lead = lead_bar(kBarPFull);  // + 8 per P buffer
         const uint32_t o_free_lead = lead_bar(kBarOFree);
         auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
         auto q_row_ptr = [&](int qvb, bool& valid) {
@@ -1278,7 +1313,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     if (leader)
                         mbar_arrive(bar(kBarPFull + sb));
                     else
-                        mbar_arrive_remote(p_full_lead[sb]);
+                        mbar_arrive_remote(p_full_lead + 8u * sb);
                 }
                 if (t == 0) TL_EV(kEvPPosted);
             }

@@ -34,7 +34,8 @@ ROLE_BASE = {"softmax": 2, "mma": 402, "k": 802, "q": 914, "v": 924}
 ROLE_CAP = {"softmax": 400, "mma": 400, "k": 112, "q": 10, "v": 100}
 EV = dict(setup=1, chunk=2, sfull=4, pposted=5, ofull=6, epidone=7, exit=8, cluster_up=9, mma_qfull=10,
           mma_kfull=11, mma_pvgo=12, announced=15, first_tile=17, kload=16, qload=18, tile_loaded=19, vload=20,
-          vtail_landed=21, vtail_done=22)
+          vtail_landed=21, vtail_done=22, conv_start=23, conv_done=24,
+          conv_raw=25, v_landed=26, v_kconv=27)
 
 
 def build_timeline_lib(force: bool = False) -> str:
