@@ -146,7 +146,7 @@ def recorded_traffic(workload: str):
 class ClockSampler:
     """Samples SM clock, power and clock-event reasons through NVML while running."""
 
-    def __init__(self, device_index: int, uuid: str | None, period_s: float = 0.005):
+    def __init__(self, device_index: int, uuid: str | None, period_s: float = 0.001):
         self.samples = []
         self.max_mhz = None
         self.err = None
