@@ -265,6 +265,9 @@ MLA_API mla_status mla_decode_combine(int batch, int s_q, int h_q, int h_kv, int
  */
 MLA_API mla_status mla_get_metadata_sparse(int num_tokens, int topk, int h_q, int h_kv, int num_parts,
                                            int32_t* tile_md, int32_t* num_splits, void* stream);
+/* The same schedule computed on the host into host arrays (synchronous; for tests and tools). */
+MLA_API mla_status mla_get_metadata_sparse_host(int num_tokens, int topk, int h_q, int h_kv, int num_parts,
+                                                int32_t* tile_md, int32_t* num_splits);
 MLA_API mla_status mla_decode_sparse(const void* q, int batch, int s_q, int h_q, int d_qk, const void* kvcache,
                                      int num_blocks, int page_size, int h_kv, const int32_t* indices, int topk,
                                      int dv, int dtype, const int32_t* tile_md, int num_parts,

@@ -11,8 +11,10 @@ Both are thin wrappers over the C ABI in ``include/mla_decode.h``; the kernels
 live in ``csrc/``.  ``workloads`` generates seeded synthetic inputs.
 """
 from .api import (DecodeCall, flash_mla_sparse_fwd, flash_mla_with_kvcache, get_mla_metadata, get_mla_metadata_host,
-                  metadata_sizes, num_sm_parts, read_device_status, workspace_bytes, workspace_zero_bytes)
+                  get_mla_metadata_sparse_host, metadata_sizes, num_sm_parts, read_device_status, workspace_bytes,
+                  workspace_zero_bytes)
 from ._lib import MLAError
 
-__all__ = ["DecodeCall", "flash_mla_sparse_fwd", "flash_mla_with_kvcache", "get_mla_metadata", "get_mla_metadata_host", "metadata_sizes",
-           "num_sm_parts", "read_device_status", "workspace_bytes", "workspace_zero_bytes", "MLAError"]
+__all__ = ["DecodeCall", "flash_mla_sparse_fwd", "flash_mla_with_kvcache", "get_mla_metadata", "get_mla_metadata_host",
+           "get_mla_metadata_sparse_host", "metadata_sizes", "num_sm_parts", "read_device_status", "workspace_bytes",
+           "workspace_zero_bytes", "MLAError"]

@@ -48,6 +48,7 @@ SIGNATURES = {
                                          _P, _I, _P, _I, _F, _I, _P, _P, _P], _I),
     "mla_read_noalloc_status": ([_I, ctypes.POINTER(_I), _P], _I),
     "mla_get_metadata_sparse": ([_I, _I, _I, _I, _I, _P, _P, _P], _I),
+    "mla_get_metadata_sparse_host": ([_I, _I, _I, _I, _I, _P, _P], _I),
     "mla_decode_sparse": ([_P, _I, _I, _I, _I,          # q, batch, s_q, h_q, d_qk
                            _P, _I, _I, _I,              # kvcache, num_blocks, page_size, h_kv
                            _P, _I, _I, _I,              # indices, topk, dv, dtype

@@ -112,6 +112,18 @@ def get_mla_metadata_host(cache_seqlens, heads_per_kv: int, h_kv: int = 1, num_p
     return md.reshape(num_parts, 8), ns
 
 
+def get_mla_metadata_sparse_host(num_tokens: int, topk: int, h_q: int, h_kv: int = 1, num_parts: int = 74):
+    """The sparse decode's schedule (num_tokens query tokens of topk entries) computed on the host."""
+    import numpy as np
+
+    n_md, n_ns = metadata_sizes(num_tokens, h_q // h_kv, h_kv, num_parts)
+    md = np.zeros(n_md, np.int32)
+    ns = np.zeros(n_ns, np.int32)
+    _lib.check(_lib.load().mla_get_metadata_sparse_host(num_tokens, topk, h_q, h_kv, num_parts, md.ctypes.data,
+                                                        ns.ctypes.data), "mla_get_metadata_sparse_host")
+    return md.reshape(num_parts, 8), ns
+
+
 def workspace_bytes(batch: int, s_q: int, h_q: int, h_kv: int, num_parts: int) -> int:
     n = _lib.load().mla_decode_workspace_bytes(batch, s_q, h_q, h_kv, num_parts)
     if n == 0:

@@ -1615,8 +1615,8 @@ __device__ void block_exclusive_scan(T* data, int n, T* warp_tot, T& total)
 constexpr int kMetaThreads = 256;
 
 __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_t* seqlens, int const_len, int batch,
-                                                                    int groups, int num_parts, int32_t* md,
-                                                                    int32_t* num_splits)
+                                                                    int groups, int num_parts, int fixed_cost,
+                                                                    int32_t* md, int32_t* num_splits)
 {
     extern __shared__ __align__(16) uint8_t meta_smem[];
     grid_dependency_wait();
@@ -1630,7 +1630,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
     int32_t* begins = extra + nv;  // [num_parts][2]
     for (int v = threadIdx.x; v < nv; v += blockDim.x) {
         pages[v] = pages_of(seqlens ? seqlens[v / groups] : const_len);
-        C[v] = pages[v] + kFixedCost;
+        C[v] = pages[v] + fixed_cost;
         extra[v] = 0;
     }
     __syncthreads();
@@ -1638,7 +1638,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
     block_exclusive_scan(C, nv, warp_tot_ll, total);
     for (int p = threadIdx.x; p < num_parts; p += blockDim.x) {
         int32_t m[kMdInts];
-        partition_range(p, num_parts, C, pages, nv, total, m);
+        partition_range(p, num_parts, C, pages, nv, total, fixed_cost, m);
         begins[2 * p] = m[0];
         begins[2 * p + 1] = m[1];
         for (int i = 0; i < kMdInts; ++i) md[p * kMdInts + i] = m[i];
@@ -1820,9 +1820,10 @@ static cudaError_t launch_splitkv_heads(int grid, cudaStream_t st, const CUtenso
 }
 
 // The metadata kernel on `stream`: lengths from `seqlens`, or `const_len` for every request
-// when `seqlens` is null (the sparse decode).
+// when `seqlens` is null (the sparse decode), at `fixed_cost` page units per chunk.
 static mla_status launch_metadata(const int32_t* seqlens, int const_len, int batch, int heads_per_kv, int h_kv,
-                                  int num_parts, int32_t* tile_md, int32_t* num_splits, void* stream)
+                                  int num_parts, int fixed_cost, int32_t* tile_md, int32_t* num_splits,
+                                  void* stream)
 {
     if (batch < 0 || heads_per_kv <= 0 || h_kv <= 0 || num_parts <= 0 || !tile_md || !num_splits)
         return MLA_ERR_INVALID_ARG;
@@ -1842,7 +1843,7 @@ static mla_status launch_metadata(const int32_t* seqlens, int const_len, int bat
     cudaLaunchAttribute attr[1];
     programmatic_launch(cfg, attr, dim3(1), dim3(kMetaThreads), smem, static_cast<cudaStream_t>(stream));
     const cudaError_t e = cudaLaunchKernelEx(&cfg, mla_metadata_kernel, seqlens, const_len, batch,
-                                             row_groups(heads_per_kv), num_parts, tile_md, num_splits);
+                                             row_groups(heads_per_kv), num_parts, fixed_cost, tile_md, num_splits);
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -1901,7 +1902,24 @@ mla_status mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int he
     const size_t nv = static_cast<size_t>(batch) * groups;
     std::vector<long long> C(nv + 1);
     std::vector<int32_t> pages(nv + 1);
-    schedule_host(cache_seqlens, batch, groups, num_parts, tile_md, num_splits, C.data(), pages.data());
+    schedule_host(cache_seqlens, batch, groups, num_parts, kFixedCost, tile_md, num_splits, C.data(), pages.data());
+    return MLA_OK;
+}
+
+mla_status mla_get_metadata_sparse_host(int num_tokens, int topk, int h_q, int h_kv, int num_parts, int32_t* tile_md,
+                                        int32_t* num_splits)
+{
+    if (num_tokens < 0 || topk < 0 || h_q <= 0 || h_kv <= 0 || h_q % h_kv || num_parts <= 0 || !tile_md ||
+        !num_splits)
+        return MLA_ERR_INVALID_ARG;
+    if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
+    const int groups = row_groups(h_q / h_kv);
+    const size_t nv = static_cast<size_t>(num_tokens) * groups;
+    std::vector<int32_t> lens(static_cast<size_t>(num_tokens) + 1, topk);
+    std::vector<long long> C(nv + 1);
+    std::vector<int32_t> pages(nv + 1);
+    schedule_host(lens.data(), num_tokens, groups, num_parts, kFixedCostSparse, tile_md, num_splits, C.data(),
+                  pages.data());
     return MLA_OK;
 }
 
@@ -1909,14 +1927,16 @@ mla_status mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_p
                             int32_t* tile_md, int32_t* num_splits, void* stream)
 {
     if (batch > 0 && !cache_seqlens) return MLA_ERR_INVALID_ARG;
-    return launch_metadata(cache_seqlens, 0, batch, heads_per_kv, h_kv, num_parts, tile_md, num_splits, stream);
+    return launch_metadata(cache_seqlens, 0, batch, heads_per_kv, h_kv, num_parts, kFixedCost, tile_md, num_splits,
+                           stream);
 }
 
 mla_status mla_get_metadata_sparse(int num_tokens, int topk, int h_q, int h_kv, int num_parts, int32_t* tile_md,
                                    int32_t* num_splits, void* stream)
 {
     if (topk < 0 || h_kv <= 0 || h_q % h_kv) return MLA_ERR_INVALID_ARG;
-    return launch_metadata(nullptr, topk, num_tokens, h_q / h_kv, h_kv, num_parts, tile_md, num_splits, stream);
+    return launch_metadata(nullptr, topk, num_tokens, h_q / h_kv, h_kv, num_parts, kFixedCostSparse, tile_md,
+                           num_splits, stream);
 }
 
 size_t mla_decode_workspace_zero_bytes(int batch, int s_q, int h_q, int h_kv)

@@ -10,8 +10,10 @@
 //
 // Work units.  A "virtual batch" vb = b * row_groups + g is request b restricted
 // to query rows [128 g, 128 g + 128) of its s_q * h_q rows.  Every chunk (one
-// partition's share of one virtual batch) costs F = kFixedCost units of
-// overhead (the output epilogue, refilling the pipeline) plus one unit per 64-token page.
+// partition's share of one virtual batch) costs F units of overhead (the output
+// epilogue, refilling the pipeline) plus one unit per 64-token page: F = kFixedCost
+// for the paged decode, kFixedCostSparse for the sparse calls, whose "pages" of 64
+// gathered entries cost two to three times a contiguous page.
 // Lay the virtual batches on a line: vb takes F units followed by its pages,
 // starting at C[vb] = sum of the costs before it; W is the total.  A partition
 // that starts inside a virtual batch's pages opens one more chunk than the line
@@ -50,7 +52,8 @@ namespace mla {
 
 constexpr int kPage = 64;
 constexpr int kRowsPerGroup = 128;
-constexpr int kFixedCost = 12;  // per-chunk overhead in page units (epilogue, pipeline refill), tuned on B200
+constexpr int kFixedCost = 12;       // per-chunk overhead in page units (epilogue, pipeline refill), tuned on B200
+constexpr int kFixedCostSparse = 4;  // the same for the sparse decode and prefill, tuned on B200
 constexpr int kMdInts = 8;
 
 MLA_HD inline int row_groups(int heads_per_kv) { return (heads_per_kv + kRowsPerGroup - 1) / kRowsPerGroup; }
@@ -58,9 +61,9 @@ MLA_HD inline int row_groups(int heads_per_kv) { return (heads_per_kv + kRowsPer
 MLA_HD inline int pages_of(int seqlen) { return seqlen <= 0 ? 0 : (seqlen + kPage - 1) / kPage; }
 
 // Position on the page line of cost unit x.  C: exclusive prefix of the costs,
-// nv entries; total: W.  Returns (vb, blk) through the references.
+// nv entries; total: W; F: the per-chunk cost.  Returns (vb, blk) through the references.
 MLA_HD inline void unit_to_page(long long x, const long long* C, const int32_t* pages, int nv, long long total,
-                                int& vb, int& blk)
+                                int F, int& vb, int& blk)
 {
     if (x >= total || nv == 0) {
         vb = nv;
@@ -76,29 +79,29 @@ MLA_HD inline void unit_to_page(long long x, const long long* C, const int32_t* 
         else
             hi = mid - 1;
     }
-    long long b = x - C[lo] - kFixedCost;
+    long long b = x - C[lo] - F;
     if (b < 0) b = 0;
     vb = lo;
     blk = static_cast<int>(b);  // < pages[lo]: positions at or past the span's end belong to lo + 1
     (void)pages;
 }
 
-// Range of partition p: md row.  C / pages: per virtual batch.
+// Range of partition p: md row.  C / pages: per virtual batch; F: the per-chunk cost.
 MLA_HD inline void partition_range(int p, int num_parts, const long long* C, const int32_t* pages, int nv,
-                                   long long total, int32_t* m)
+                                   long long total, int F, int32_t* m)
 {
-    long long D = (total - kFixedCost + num_parts - 1) / num_parts;  // line units of a partition after its first F
+    long long D = (total - F + num_parts - 1) / num_parts;  // line units of a partition after its first F
     // A partition shorter than one chunk's overhead would cost more than it saves: small
     // batches use fewer partitions (the rest get empty ranges) instead of one-page splits.
-    if (D < kFixedCost) D = kFixedCost;
-    auto start = [&](int q) -> long long { return q == 0 ? 0 : kFixedCost + static_cast<long long>(q) * D; };
+    if (D < F) D = F;
+    auto start = [&](int q) -> long long { return q == 0 ? 0 : F + static_cast<long long>(q) * D; };
     int bv, bb, ev, eb;
-    unit_to_page(start(p), C, pages, nv, total, bv, bb);
+    unit_to_page(start(p), C, pages, nv, total, F, bv, bb);
     if (p == num_parts - 1) {
         ev = nv;
         eb = 0;
     } else {
-        unit_to_page(start(p + 1), C, pages, nv, total, ev, eb);
+        unit_to_page(start(p + 1), C, pages, nv, total, F, ev, eb);
     }
     m[0] = bv;
     m[1] = bb;
@@ -110,7 +113,7 @@ MLA_HD inline void partition_range(int p, int num_parts, const long long* C, con
 
 // Host reference of the whole schedule (the device kernel computes the same
 // values in parallel).  Scratch: C [nv] and pages [nv].
-inline void schedule_host(const int32_t* seqlens, int batch, int groups, int num_parts, int32_t* md,
+inline void schedule_host(const int32_t* seqlens, int batch, int groups, int num_parts, int F, int32_t* md,
                           int32_t* num_splits, long long* C, int32_t* pages)
 {
     const int nv = batch * groups;
@@ -118,9 +121,9 @@ inline void schedule_host(const int32_t* seqlens, int batch, int groups, int num
     for (int v = 0; v < nv; ++v) {
         pages[v] = pages_of(seqlens[v / groups]);
         C[v] = total;
-        total += pages[v] + kFixedCost;
+        total += pages[v] + F;
     }
-    for (int p = 0; p < num_parts; ++p) partition_range(p, num_parts, C, pages, nv, total, md + p * kMdInts);
+    for (int p = 0; p < num_parts; ++p) partition_range(p, num_parts, C, pages, nv, total, F, md + p * kMdInts);
     // split counts: 1 + number of partitions that start inside a virtual batch's pages
     for (int v = 0; v <= nv; ++v) num_splits[v] = 0;
     for (int p = 0; p < num_parts; ++p) {

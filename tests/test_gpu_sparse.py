@@ -108,11 +108,12 @@ def test_sparse_active_heads(oracle_mod):
 
 
 def test_sparse_metadata_kernel_matches_host_schedule():
-    # the device schedule of the sparse decode is the dense one over tokens of topk entries
+    # the device schedule of the sparse decode is the dense algorithm over tokens of topk entries
+    # (at the sparse calls' per-chunk cost)
     for tokens, topk, h_q in ((7, 2048, 128), (300, 100, 64), (3, 64, 256)):
         sl = torch.zeros(1, dtype=torch.int32, device="cuda")
         md, ns = mla.get_mla_metadata(sl.expand(tokens).contiguous(), h_q, 1, h_q=h_q, topk=topk)
-        md_h, ns_h = mla.get_mla_metadata_host(np.full(tokens, topk, np.int32), h_q, 1, md.shape[0])
+        md_h, ns_h = mla.get_mla_metadata_sparse_host(tokens, topk, h_q, 1, md.shape[0])
         assert np.array_equal(md.cpu().numpy(), md_h) and np.array_equal(ns.cpu().numpy(), ns_h)
 
 

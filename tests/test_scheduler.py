@@ -17,6 +17,7 @@ import mla_decode_attention_12_b200 as mla
 _SRC = os.path.join(os.path.dirname(os.path.dirname(__file__)), "mla_decode_attention_12_b200", "csrc",
                     "scheduler.cuh")
 FIXED = int(re.search(r"constexpr int kFixedCost = (\d+);", open(_SRC).read()).group(1))
+FIXED_SPARSE = int(re.search(r"constexpr int kFixedCostSparse = (\d+);", open(_SRC).read()).group(1))
 
 
 def pages(L):
@@ -36,9 +37,17 @@ def chunks_of(md, seqlens, groups):
     return out
 
 
-def check_schedule(seqlens, heads_per_kv, num_parts):
+def check_schedule(seqlens, heads_per_kv, num_parts, sparse_topk=None):
+    """The properties of the paged decode's schedule (or, with sparse_topk, of the sparse
+    decode's: len(seqlens) query tokens of sparse_topk entries each)."""
     seqlens = np.asarray(seqlens, np.int32)
-    md, ns = mla.get_mla_metadata_host(seqlens, heads_per_kv, 1, num_parts)
+    if sparse_topk is None:
+        md, ns = mla.get_mla_metadata_host(seqlens, heads_per_kv, 1, num_parts)
+        F = FIXED
+    else:
+        assert np.all(seqlens == sparse_topk)
+        md, ns = mla.get_mla_metadata_sparse_host(seqlens.size, sparse_topk, heads_per_kv, 1, num_parts)
+        F = FIXED_SPARSE
     groups = (heads_per_kv + 127) // 128
     nv = seqlens.size * groups
     assert md.shape == (num_parts, 8) and ns.shape == (nv + 1,)
@@ -66,11 +75,11 @@ def check_schedule(seqlens, heads_per_kv, num_parts):
     # balance: every partition's cost, pages plus the fixed cost of each of its
     # chunks, stays within the budget F + max(ceil((W - F) / num_parts), F) (a partition
     # is never given less than one chunk's overhead of pages)
-    W = sum((pages(L) + FIXED) * groups for L in seqlens)
-    T = max(-(-(W - FIXED) // num_parts), FIXED) + FIXED
+    W = sum((pages(L) + F) * groups for L in seqlens)
+    T = max(-(-(W - F) // num_parts), F) + F
     cost = np.zeros(num_parts, np.int64)
     for p, vb, lo, hi, _ in ch:
-        cost[p] += (hi - lo) + FIXED
+        cost[p] += (hi - lo) + F
     assert cost.max(initial=0) <= T
     return md, ns, cost, T
 
@@ -116,3 +125,16 @@ def test_long_sequences_are_split_evenly():
     md, ns, cost, T = check_schedule([65536, 49152, 32768, 8192], 128, 74)
     assert ns[-1] > 4  # at least one sequence is split, so the combine kernel runs
     assert cost.max() <= T
+
+
+@pytest.mark.parametrize("tokens,topk,h_q,parts", [(128, 2048, 128, 74), (7, 2048, 128, 74), (300, 100, 64, 74),
+                                                   (3, 64, 256, 74), (2048, 2048, 128, 74), (5, 0, 128, 3)])
+def test_sparse_schedule(tokens, topk, h_q, parts):
+    # the sparse calls' schedule: the same algorithm at their own per-chunk cost
+    check_schedule([topk] * tokens, h_q, parts, sparse_topk=topk)
+
+
+def test_sparse_schedule_uses_its_own_chunk_cost():
+    md_s, _ = mla.get_mla_metadata_sparse_host(64, 2048, 128, 1, 74)
+    md_d, _ = mla.get_mla_metadata_host(np.full(64, 2048, np.int32), 128, 1, 74)
+    assert FIXED_SPARSE != FIXED and not np.array_equal(md_s, md_d)
