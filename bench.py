@@ -307,7 +307,7 @@ class Runner:
         parts = mla.num_sm_parts(dev)
         sparse = p.indices is not None  # token-level sparse decode: the entry lists replace the block table
         self.ind = torch.from_numpy(p.indices).to(dev) if sparse else None
-        md_kw = dict(h_q=p.h_q, topk=p.indices.shape[2]) if sparse else {}
+        md_kw = dict(h_q=p.h_q, topk=p.indices.shape[2]) if sparse else dict(is_fp8_kvcache=p.fp8_kv)
         n_md, n_ns = mla.metadata_sizes(p.batch * p.s_q if sparse else p.batch, p.h_q if sparse else self.rows, 1,
                                         parts)
         self.md = torch.zeros(parts, 8, dtype=torch.int32, device=dev)

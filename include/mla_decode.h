@@ -110,7 +110,8 @@ MLA_API mla_status mla_metadata_sizes(int batch, int heads_per_kv, int h_kv, int
 /*
  * Tile scheduler ("FlashMLA" usage page: get_mla_metadata(cache_seqlens,
  * s_q * h_q // h_kv, h_kv) returns tile_scheduler_metadata and num_splits; the
- * page's Tile Scheduler "distributes work across GPU resources").
+ * page's Tile Scheduler "distributes work across GPU resources"; the upstream
+ * FlashMLA documentation's "Usage / MLA Decoding" call also takes is_fp8).
  *
  * Splits the work -- for each request b and row group of 128 query rows, the
  * ceil(L_b / 64) pages of its cache plus a fixed per-chunk overhead -- into
@@ -118,20 +119,25 @@ MLA_API mla_status mla_metadata_sizes(int batch, int heads_per_kv, int h_kv, int
  * whose pages fall into more than one range is split; num_splits holds the
  * prefix sums of the split counts, and the decode call merges split results.
  *
- *   cache_seqlens  device [batch] int32
- *   heads_per_kv   s_q * h_q / h_kv (> 0)
- *   h_kv           number of KV heads (must be 1: MQA mode)
- *   num_parts      from mla_num_sm_parts (the same value must be passed to decode)
- *   tile_md        device [num_parts, 8] int32, written
- *   num_splits     device [batch * row_groups + 1] int32, written
+ *   cache_seqlens    device [batch] int32
+ *   heads_per_kv     s_q * h_q / h_kv (> 0)
+ *   h_kv             number of KV heads (must be 1: MQA mode)
+ *   num_parts        from mla_num_sm_parts (the same value must be passed to decode)
+ *   is_fp8_kvcache   nonzero when the decode calls read an "FP8 with scale" cache:
+ *                    its pages take longer, so a chunk's fixed overhead counts for
+ *                    fewer pages (any schedule is valid for either cache; this one
+ *                    balances the work better)
+ *   tile_md          device [num_parts, 8] int32, written
+ *   num_splits       device [batch * row_groups + 1] int32, written
  * Runs one small kernel on `stream`; no host synchronisation.
  */
 MLA_API mla_status mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv,
-                            int num_parts, int32_t* tile_md, int32_t* num_splits, void* stream);
+                                    int num_parts, int is_fp8_kvcache, int32_t* tile_md, int32_t* num_splits,
+                                    void* stream);
 
 /* Same schedule computed on the host: every pointer is host memory. */
-MLA_API mla_status mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per_kv,
-                                 int h_kv, int num_parts, int32_t* tile_md, int32_t* num_splits);
+MLA_API mla_status mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv,
+                                         int num_parts, int is_fp8_kvcache, int32_t* tile_md, int32_t* num_splits);
 
 /*
  * Bytes of device workspace mla_decode_with_kvcache needs: a control block of

@@ -30,8 +30,8 @@ SIGNATURES = {
     "mla_status_string": ([_I], ctypes.c_char_p),
     "mla_num_sm_parts": ([_I, ctypes.POINTER(_I)], _I),
     "mla_metadata_sizes": ([_I, _I, _I, _I, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)], _I),
-    "mla_get_metadata": ([_P, _I, _I, _I, _I, _P, _P, _P], _I),
-    "mla_get_metadata_host": ([_P, _I, _I, _I, _I, _P, _P], _I),
+    "mla_get_metadata": ([_P, _I, _I, _I, _I, _I, _P, _P, _P], _I),
+    "mla_get_metadata_host": ([_P, _I, _I, _I, _I, _I, _P, _P], _I),
     "mla_decode_workspace_bytes": ([_I, _I, _I, _I, _I], _SZ),
     "mla_decode_workspace_zero_bytes": ([_I, _I, _I, _I], _SZ),
     "mla_decode_with_kvcache": ([_P, _I, _I, _I, _I,          # q, batch, s_q, h_q, d_qk

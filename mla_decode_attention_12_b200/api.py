@@ -47,14 +47,19 @@ def metadata_sizes(batch: int, heads_per_kv: int, h_kv: int, num_parts: int):
     return a.value, b.value
 
 
-def get_mla_metadata(cache_seqlens: torch.Tensor, heads_per_kv: int, h_kv: int = 1, num_parts: int | None = None,
-                     out=None, h_q: int | None = None, topk: int | None = None):
+def get_mla_metadata(cache_seqlens: torch.Tensor, heads_per_kv: int, h_kv: int = 1, h_q: int | None = None,
+                     is_fp8_kvcache: bool = False, topk: int | None = None, *, num_parts: int | None = None,
+                     out=None):
     """Tile-scheduler metadata for one decoding step.
 
-    ``cache_seqlens``: int32 [batch] on a CUDA device.  ``heads_per_kv`` is
-    ``s_q * h_q // h_kv``.  Returns ``(tile_scheduler_metadata [num_parts, 8] int32,
-    num_splits [batch * ceil(heads_per_kv / 128) + 1] int32)`` on the same device;
-    ``out`` = (md, ns) writes into existing tensors instead.
+    The arguments follow the upstream FlashMLA documentation's call ("Usage / MLA
+    Decoding": ``get_mla_metadata(cache_seqlens, s_q * h_q // h_kv, h_kv, h_q, is_fp8,
+    topk)``).  ``cache_seqlens``: int32 [batch] on a CUDA device.  ``heads_per_kv`` is
+    ``s_q * h_q // h_kv``.  ``is_fp8_kvcache``: the decode calls read an "FP8 with scale"
+    cache (a schedule tuned for its slower pages; any schedule is valid for either cache).
+    Returns ``(tile_scheduler_metadata [num_parts, 8] int32, num_splits [batch *
+    ceil(heads_per_kv / 128) + 1] int32)`` on the same device; ``out`` = (md, ns) writes
+    into existing tensors instead.
 
     With ``topk`` (and ``h_q``): the schedule of the token-level sparse decode, whose
     batch * s_q query tokens each attend ``topk`` listed entries (upstream FlashMLA
@@ -95,11 +100,13 @@ def get_mla_metadata(cache_seqlens: torch.Tensor, heads_per_kv: int, h_kv: int =
         ns = torch.empty(n_ns, dtype=torch.int32, device=dev)
     with torch.cuda.device(dev):
         _lib.check(_lib.load().mla_get_metadata(_ptr(cache_seqlens), batch, heads_per_kv, h_kv, num_parts,
-                                                _ptr(md), _ptr(ns), _stream(dev)), "mla_get_metadata")
+                                                int(bool(is_fp8_kvcache)), _ptr(md), _ptr(ns), _stream(dev)),
+                   "mla_get_metadata")
     return md, ns
 
 
-def get_mla_metadata_host(cache_seqlens, heads_per_kv: int, h_kv: int = 1, num_parts: int = 74):
+def get_mla_metadata_host(cache_seqlens, heads_per_kv: int, h_kv: int = 1, num_parts: int = 74,
+                          is_fp8_kvcache: bool = False):
     """The same schedule computed on the host (numpy in, numpy out)."""
     import numpy as np
 
@@ -108,7 +115,8 @@ def get_mla_metadata_host(cache_seqlens, heads_per_kv: int, h_kv: int = 1, num_p
     md = np.zeros(n_md, np.int32)
     ns = np.zeros(n_ns, np.int32)
     _lib.check(_lib.load().mla_get_metadata_host(sl.ctypes.data, sl.size, heads_per_kv, h_kv, num_parts,
-                                                 md.ctypes.data, ns.ctypes.data), "mla_get_metadata_host")
+                                                 int(bool(is_fp8_kvcache)), md.ctypes.data, ns.ctypes.data),
+               "mla_get_metadata_host")
     return md.reshape(num_parts, 8), ns
 
 

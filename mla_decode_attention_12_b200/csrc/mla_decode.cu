@@ -1890,7 +1890,7 @@ mla_status mla_metadata_sizes(int batch, int heads_per_kv, int h_kv, int num_par
 }
 
 mla_status mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv,
-                                 int num_parts, int32_t* tile_md, int32_t* num_splits)
+                                 int num_parts, int is_fp8_kvcache, int32_t* tile_md, int32_t* num_splits)
 {
     if (batch < 0 || heads_per_kv <= 0 || h_kv <= 0 || num_parts <= 0 || !tile_md || !num_splits ||
         (batch > 0 && !cache_seqlens))
@@ -1902,7 +1902,8 @@ mla_status mla_get_metadata_host(const int32_t* cache_seqlens, int batch, int he
     const size_t nv = static_cast<size_t>(batch) * groups;
     std::vector<long long> C(nv + 1);
     std::vector<int32_t> pages(nv + 1);
-    schedule_host(cache_seqlens, batch, groups, num_parts, kFixedCost, tile_md, num_splits, C.data(), pages.data());
+    schedule_host(cache_seqlens, batch, groups, num_parts, is_fp8_kvcache ? kFixedCostFp8 : kFixedCost, tile_md,
+                  num_splits, C.data(), pages.data());
     return MLA_OK;
 }
 
@@ -1924,11 +1925,11 @@ mla_status mla_get_metadata_sparse_host(int num_tokens, int topk, int h_q, int h
 }
 
 mla_status mla_get_metadata(const int32_t* cache_seqlens, int batch, int heads_per_kv, int h_kv, int num_parts,
-                            int32_t* tile_md, int32_t* num_splits, void* stream)
+                            int is_fp8_kvcache, int32_t* tile_md, int32_t* num_splits, void* stream)
 {
     if (batch > 0 && !cache_seqlens) return MLA_ERR_INVALID_ARG;
-    return launch_metadata(cache_seqlens, 0, batch, heads_per_kv, h_kv, num_parts, kFixedCost, tile_md, num_splits,
-                           stream);
+    return launch_metadata(cache_seqlens, 0, batch, heads_per_kv, h_kv, num_parts,
+                           is_fp8_kvcache ? kFixedCostFp8 : kFixedCost, tile_md, num_splits, stream);
 }
 
 mla_status mla_get_metadata_sparse(int num_tokens, int topk, int h_q, int h_kv, int num_parts, int32_t* tile_md,

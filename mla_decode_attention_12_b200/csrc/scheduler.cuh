@@ -12,8 +12,9 @@
 // to query rows [128 g, 128 g + 128) of its s_q * h_q rows.  Every chunk (one
 // partition's share of one virtual batch) costs F units of overhead (the output
 // epilogue, refilling the pipeline) plus one unit per 64-token page: F = kFixedCost
-// for the paged decode, kFixedCostSparse for the sparse calls, whose "pages" of 64
-// gathered entries cost two to three times a contiguous page.
+// for the paged decode (kFixedCostFp8 over an FP8 cache, whose pages take about twice
+// as long), kFixedCostSparse for the sparse calls, whose "pages" of 64 gathered
+// entries cost two to three times a contiguous page.
 // Lay the virtual batches on a line: vb takes F units followed by its pages,
 // starting at C[vb] = sum of the costs before it; W is the total.  A partition
 // that starts inside a virtual batch's pages opens one more chunk than the line
@@ -53,6 +54,7 @@ namespace mla {
 constexpr int kPage = 64;
 constexpr int kRowsPerGroup = 128;
 constexpr int kFixedCost = 12;       // per-chunk overhead in page units (epilogue, pipeline refill), tuned on B200
+constexpr int kFixedCostFp8 = 6;     // the same for the paged decode over an FP8 cache, tuned on B200
 constexpr int kFixedCostSparse = 4;  // the same for the sparse decode and prefill, tuned on B200
 constexpr int kMdInts = 8;
 

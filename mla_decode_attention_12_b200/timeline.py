@@ -74,7 +74,8 @@ def record(lib, p: W.Problem, launches: int = 6):
         _lib.check(lib.mla_get_metadata_sparse(tokens, p.indices.shape[2], p.h_q, 1, parts, md.data_ptr(),
                                                ns.data_ptr(), st), "mla_get_metadata_sparse")
     else:
-        _lib.check(lib.mla_get_metadata(sl.data_ptr(), p.batch, rows, 1, parts, md.data_ptr(), ns.data_ptr(), st),
+        _lib.check(lib.mla_get_metadata(sl.data_ptr(), p.batch, rows, 1, parts, int(p.fp8_kv), md.data_ptr(),
+                                        ns.data_ptr(), st),
                    "mla_get_metadata")
     ws_b, ws_s = (tokens, 1) if sparse else (p.batch, p.s_q)
     ws = torch.zeros(mla.workspace_bytes(ws_b, ws_s, p.h_q, 1, parts), dtype=torch.uint8, device="cuda")

@@ -36,7 +36,7 @@ def to_device(p: W.Problem, device="cuda"):
 
 def run_gpu(p: W.Problem, device="cuda", num_parts=None, check_status=True):
     q, kv, bt, sl = to_device(p, device)
-    md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q // p.h_kv, p.h_kv, num_parts=num_parts)
+    md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q // p.h_kv, p.h_kv, is_fp8_kvcache=p.fp8_kv, num_parts=num_parts)
     ws = torch.zeros(mla.workspace_bytes(p.batch, p.s_q, p.h_q, p.h_kv, md.shape[0]), dtype=torch.uint8,
                      device=device)
     o, lse = mla.flash_mla_with_kvcache(q, kv, bt, sl, p.dv, md, ns, causal=p.causal, softmax_scale=p.scale,

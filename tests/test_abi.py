@@ -109,10 +109,10 @@ def test_status_reads_reject_null_outputs(lib):
 
 def test_metadata_rejects_bad_arguments(lib):
     fake = 1 << 20
-    assert lib.mla_get_metadata(fake, 4, 0, 1, 74, fake, fake, None) == 1
-    assert lib.mla_get_metadata(fake, 4, 128, 2, 74, fake, fake, None) == 2
-    assert lib.mla_get_metadata(fake, 4, 128, 1, 0, fake, fake, None) == 1
-    assert lib.mla_get_metadata(None, 4, 128, 1, 74, fake, fake, None) == 1
+    assert lib.mla_get_metadata(fake, 4, 0, 1, 74, 0, fake, fake, None) == 1
+    assert lib.mla_get_metadata(fake, 4, 128, 2, 74, 0, fake, fake, None) == 2
+    assert lib.mla_get_metadata(fake, 4, 128, 1, 0, 1, fake, fake, None) == 1
+    assert lib.mla_get_metadata(None, 4, 128, 1, 74, 0, fake, fake, None) == 1
 
 
 def test_host_metadata_rejects_negative_lengths(lib):
@@ -121,7 +121,7 @@ def test_host_metadata_rejects_negative_lengths(lib):
     sl = np.array([5, -1], np.int32)
     md = np.zeros(74 * 8, np.int32)
     ns = np.zeros(3, np.int32)
-    assert lib.mla_get_metadata_host(sl.ctypes.data, 2, 16, 1, 74, md.ctypes.data, ns.ctypes.data) == 1
+    assert lib.mla_get_metadata_host(sl.ctypes.data, 2, 16, 1, 74, 0, md.ctypes.data, ns.ctypes.data) == 1
 
 
 @pytest.mark.parametrize("case", ["fp16_q", "bf16_cache", "row_bytes", "d_qk_512", "mixed_16bit"])

@@ -66,7 +66,7 @@ def test_fp8_few_partitions(oracle_mod, parts):
 def test_fp8_active_heads(oracle_mod):
     p = fp8([300, 420, 511, 129, 64, 2], s_q=2, h_q=64, causal=True, active_heads=16, seed=212)
     q, kv, bt, sl = to_device(p)
-    md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q, 1)
+    md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q, 1, is_fp8_kvcache=True)
     o = torch.full((p.batch, p.s_q, p.h_q, 512), 7.0, dtype=q.dtype, device="cuda")
     lse = torch.full((p.batch, p.s_q, p.h_q), 7.0, dtype=torch.float32, device="cuda")
     mla.flash_mla_with_kvcache(q, kv, bt, sl, p.dv, md, ns, causal=True, softmax_scale=p.scale, out=o, lse=lse,
@@ -114,7 +114,7 @@ def test_fp8_host_buffers_end_to_end(oracle_mod):
     # pinned host tensors through the public call: copied in, decoded, copied back
     p = fp8([700, 64], s_q=2, h_q=16, causal=True, seed=214)
     q, kv, bt, sl = (t.cpu().pin_memory() for t in to_device(p))
-    md, ns = mla.get_mla_metadata(sl.cuda(), p.s_q * p.h_q, 1)
+    md, ns = mla.get_mla_metadata(sl.cuda(), p.s_q * p.h_q, 1, is_fp8_kvcache=True)
     o, lse = mla.flash_mla_with_kvcache(q, kv, bt, sl, 512, md.cpu(), ns.cpu(), causal=True, softmax_scale=p.scale,
                                         is_fp8_kvcache=True)
     assert not o.is_cuda and kv.dtype == torch.uint8

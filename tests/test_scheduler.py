@@ -18,6 +18,7 @@ _SRC = os.path.join(os.path.dirname(os.path.dirname(__file__)), "mla_decode_atte
                     "scheduler.cuh")
 FIXED = int(re.search(r"constexpr int kFixedCost = (\d+);", open(_SRC).read()).group(1))
 FIXED_SPARSE = int(re.search(r"constexpr int kFixedCostSparse = (\d+);", open(_SRC).read()).group(1))
+FIXED_FP8 = int(re.search(r"constexpr int kFixedCostFp8 = (\d+);", open(_SRC).read()).group(1))
 
 
 def pages(L):
@@ -37,13 +38,13 @@ def chunks_of(md, seqlens, groups):
     return out
 
 
-def check_schedule(seqlens, heads_per_kv, num_parts, sparse_topk=None):
-    """The properties of the paged decode's schedule (or, with sparse_topk, of the sparse
-    decode's: len(seqlens) query tokens of sparse_topk entries each)."""
+def check_schedule(seqlens, heads_per_kv, num_parts, sparse_topk=None, fp8=False):
+    """The properties of the paged decode's schedule (over an FP8 cache with fp8), or, with
+    sparse_topk, of the sparse decode's: len(seqlens) query tokens of sparse_topk entries."""
     seqlens = np.asarray(seqlens, np.int32)
     if sparse_topk is None:
-        md, ns = mla.get_mla_metadata_host(seqlens, heads_per_kv, 1, num_parts)
-        F = FIXED
+        md, ns = mla.get_mla_metadata_host(seqlens, heads_per_kv, 1, num_parts, is_fp8_kvcache=fp8)
+        F = FIXED_FP8 if fp8 else FIXED
     else:
         assert np.all(seqlens == sparse_topk)
         md, ns = mla.get_mla_metadata_sparse_host(seqlens.size, sparse_topk, heads_per_kv, 1, num_parts)
@@ -138,3 +139,11 @@ def test_sparse_schedule_uses_its_own_chunk_cost():
     md_s, _ = mla.get_mla_metadata_sparse_host(64, 2048, 128, 1, 74)
     md_d, _ = mla.get_mla_metadata_host(np.full(64, 2048, np.int32), 128, 1, 74)
     assert FIXED_SPARSE != FIXED and not np.array_equal(md_s, md_d)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_fp8_cache_schedule(seed):
+    # the paged decode over an FP8 cache: the same algorithm at that cache's per-chunk cost
+    rng = np.random.default_rng(100 + seed)
+    L = rng.integers(0, 20000, int(rng.integers(1, 200))).astype(np.int32)
+    check_schedule(L, int(rng.choice([16, 64, 128, 256])), int(rng.choice([1, 7, 74])), fp8=True)
