@@ -190,9 +190,38 @@ def summarize(name: str, per, end: float, kernel_us: float) -> str:
     return "\n".join(lines) + "\n"
 
 
+def fp8_pipeline(B, grid) -> str:
+    """The FP8 cache's K-stage cycle (converter warp 0 and the V producer of each CTA), per page:
+    conversion, the wait for the other converter warps, the wait for a free V stage, the V copies
+    until they land.  Empty when the record has no converter events (16-bit cache)."""
+    start = B[:grid, 0].astype(np.int64) | (B[:grid, 1].astype(np.int64) << 32)
+    t_off = (start - start.min()) / 1e3
+    R = {k: [] for k in ("conversion (converter warp 0)", "rest of the converter warps", "wait for the V stage",
+                         "V copies issued -> landed")}
+    for c in range(grid):
+        ik, tk = events(B, c, "k", t_off)
+        st, dn = tk[ik == EV["conv_start"]], tk[ik == EV["conv_done"]]
+        iv, tv = events(B, c, "v", t_off)
+        kc, vl, vd = tv[iv == EV["v_kconv"]], tv[iv == EV["vload"]], tv[iv == EV["v_landed"]]
+        n = min(len(st), len(dn), len(kc), len(vl), len(vd))
+        if n == 0:
+            continue
+        R["conversion (converter warp 0)"] += list(dn[:n] - st[:n])
+        R["rest of the converter warps"] += list(kc[:n] - dn[:n])
+        R["wait for the V stage"] += list(vl[:n] - kc[:n])
+        R["V copies issued -> landed"] += list(vd[:n] - vl[:n])
+    if not R["conversion (converter warp 0)"]:
+        return ""
+    lines = ["| FP8 K-stage cycle, per page | p10 | median | p90 |", "|---|---|---|---|"]
+    for k, v in R.items():
+        v = np.array(v)
+        lines.append(f"| {k} | {np.percentile(v, 10):6.2f} | {np.median(v):6.2f} | {np.percentile(v, 90):6.2f} |")
+    return "\n".join(lines) + "\n"
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--workloads", default="compute,spec_padded,long_split,fp16_norope,sparse_fp8")
+    ap.add_argument("--workloads", default="compute,spec_padded,long_split,fp16_norope,fp8_compute,sparse_fp8")
     ap.add_argument("--launches", type=int, default=6)
     ap.add_argument("--save", default=None, help="directory to save the raw event arrays (.npy) in")
     args = ap.parse_args(argv)
@@ -209,7 +238,7 @@ def main(argv=None):
             os.makedirs(args.save, exist_ok=True)
             np.save(os.path.join(args.save, f"timeline_{name}.npy"), B)
         per, end = phases(B, grid)
-        out.append(summarize(name, per, end, us))
+        out.append(summarize(name, per, end, us) + fp8_pipeline(B, grid))
         print(out[-1], flush=True)
     return out
 
