@@ -245,10 +245,10 @@ class DecodeCall:
 
 def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: torch.Tensor,
                            cache_seqlens: torch.Tensor, dv: int, tile_scheduler_metadata: torch.Tensor,
-                           num_splits: torch.Tensor, causal: bool = False, softmax_scale: float | None = None,
+                           num_splits: torch.Tensor, causal: bool = False, is_fp8_kvcache: bool = False,
+                           indices: torch.Tensor | None = None, *, softmax_scale: float | None = None,
                            workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
-                           lse: torch.Tensor | None = None, active_heads: int | None = None,
-                           is_fp8_kvcache: bool = False, indices: torch.Tensor | None = None):
+                           lse: torch.Tensor | None = None, active_heads: int | None = None):
     """MLA decode over a paged cache; returns ``(o [b, s_q, h_q, dv], lse [b, s_q, h_q] float32)``.
 
     ``is_fp8_kvcache``: ``kvcache`` is uint8 [num_blocks, 64, h_kv, 656] in the "FP8

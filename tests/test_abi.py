@@ -198,3 +198,24 @@ def test_sparse_prefill_rejects_bad_arguments(lib):
     assert call(d_qk=512) == 2 and call(h_kv=2) == 2 and call(dv=256) == 2
     assert call(ws_bytes=100) == 3
     assert call(s_q=0, q=None, out=None) == 0
+
+
+def test_python_calls_take_the_documented_positional_order():
+    # upstream FlashMLA documentation, "Usage / MLA Decoding":
+    #   get_mla_metadata(cache_seqlens, s_q * h_q // h_kv, h_kv, h_q, is_fp8, topk)
+    #   flash_mla_with_kvcache(q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata,
+    #                          num_splits, is_causal, is_fp8_kvcache, indices)
+    import inspect
+
+    import mla_decode_attention_12_b200 as mla
+
+    def positional(fn):
+        return [p.name for p in inspect.signature(fn).parameters.values()
+                if p.kind in (p.POSITIONAL_ONLY, p.POSITIONAL_OR_KEYWORD)]
+
+    assert positional(mla.get_mla_metadata) == ["cache_seqlens", "heads_per_kv", "h_kv", "h_q", "is_fp8_kvcache",
+                                                "topk"]
+    assert positional(mla.flash_mla_with_kvcache) == ["q", "kvcache", "block_table", "cache_seqlens", "dv",
+                                                      "tile_scheduler_metadata", "num_splits", "causal",
+                                                      "is_fp8_kvcache", "indices"]
+    assert positional(mla.flash_mla_sparse_fwd)[:4] == ["q", "kv", "indices", "sm_scale"]
