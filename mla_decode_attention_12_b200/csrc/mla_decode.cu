@@ -1497,50 +1497,86 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
     // uniform over the CTA in the split-parallel layout; padding heads are not combined
     if (r >= rows_here || (rg * kRowsPerGroup + r) % p.h_q >= p.active_heads) return;
     const float* lse_k = p.lse_accum + static_cast<size_t>(slot0) * kRowsPerGroup + r;
-    float mx = -INFINITY;
-    for (int k = lane; k < nsplit; k += 32) mx = fmaxf(mx, __ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup));
+    const float* max_k = p.max_accum + static_cast<size_t>(slot0) * kRowsPerGroup + r;
+    // The splits' LSEs (and maxima) are read once, in one round trip: lane i holds splits i,
+    // i + 32 and i + 64 (a virtual batch has at most one split per partition; further splits,
+    // for a caller's partition count above 96, are read again where needed).
+    constexpr int kLseRegs = 3;
+    float lk[kLseRegs], mk[kLseRegs];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    for (int i = 0; i < kLseRegs; ++i) {
+        const int k = lane + 32 * i;
+        lk[i] = k < nsplit ? __ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup) : -INFINITY;
+        mk[i] = (p.max_logits && k < nsplit) ? __ldcg(max_k + static_cast<size_t>(k) * kRowsPerGroup) : -INFINITY;
+    }
+    float mx = fmaxf(fmaxf(lk[0], lk[1]), lk[2]);
+    float row_max = fmaxf(fmaxf(mk[0], mk[1]), mk[2]);  // the largest base-2 scaled logit (the prefill's max_logits)
+    for (int k = lane + 32 * kLseRegs; k < nsplit; k += 32) {
+        mx = fmaxf(mx, __ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup));
+        if (p.max_logits) row_max = fmaxf(row_max, __ldcg(max_k + static_cast<size_t>(k) * kRowsPerGroup));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        row_max = fmaxf(row_max, __shfl_xor_sync(0xffffffffu, row_max, o));
+    }
     float sum = 0.f;
-    if (mx != -INFINITY)
-        for (int k = lane; k < nsplit; k += 32) sum += expf(__ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup) - mx);
+    if (mx != -INFINITY) {
+#pragma unroll
+        for (int i = 0; i < kLseRegs; ++i) sum += expf(lk[i] - mx);  // exp(-inf) = 0 for absent splits
+        for (int k = lane + 32 * kLseRegs; k < nsplit; k += 32) sum += expf(__ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup) - mx);
+    }
 #pragma unroll
     for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float lse = (mx == -INFINITY) ? -INFINITY : mx + logf(sum);
-    float row_max = -INFINITY;  // the largest base-2 scaled logit over the splits (the prefill's max_logits)
-    if (p.max_logits) {
-        const float* max_k = p.max_accum + static_cast<size_t>(slot0) * kRowsPerGroup + r;
-        for (int k = lane; k < nsplit; k += 32) row_max = fmaxf(row_max, __ldcg(max_k + static_cast<size_t>(k) * kRowsPerGroup));
+    // weight of split k = exp(lse_k - lse), from lane k % 32's registers (k warp-uniform)
+    float wk[kLseRegs];
 #pragma unroll
-        for (int o = 16; o; o >>= 1) row_max = fmaxf(row_max, __shfl_xor_sync(0xffffffffu, row_max, o));
-    }
+    for (int i = 0; i < kLseRegs; ++i) wk[i] = expf(lk[i] - lse);
+    auto weight = [&](int k) {
+        if (k >= 32 * kLseRegs) return expf(__ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup) - lse);
+        const float w = k < 32 ? wk[0] : (k < 64 ? wk[1] : wk[2]);
+        return __shfl_sync(0xffffffffu, w, k & 31);
+    };
     float4 acc[4];  // float4 columns lane, lane + 32, lane + 64, lane + 96
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    auto add_split = [&](const float4* s4, float w) {
-        const float4 v0 = __ldcg(s4), v1 = __ldcg(s4 + 32), v2 = __ldcg(s4 + 64), v3 = __ldcg(s4 + 96);
-        acc[0].x += w * v0.x; acc[0].y += w * v0.y; acc[0].z += w * v0.z; acc[0].w += w * v0.w;
-        acc[1].x += w * v1.x; acc[1].y += w * v1.y; acc[1].z += w * v1.z; acc[1].w += w * v1.w;
-        acc[2].x += w * v2.x; acc[2].y += w * v2.y; acc[2].z += w * v2.z; acc[2].w += w * v2.w;
-        acc[3].x += w * v3.x; acc[3].y += w * v3.y; acc[3].z += w * v3.z; acc[3].w += w * v3.w;
+    auto fma4 = [](float4& a, const float4& v, float w) {
+        a.x += w * v.x; a.y += w * v.y; a.z += w * v.z; a.w += w * v.w;
     };
     if (mx != -INFINITY) {
         const float4* src = reinterpret_cast<const float4*>(p.o_accum + (static_cast<size_t>(slot0) * kRowsPerGroup + r) * kDv) + lane;
         const size_t stride4 = static_cast<size_t>(kRowsPerGroup) * kDv / 4;  // float4s between splits
-        if (kSplitParallel) {
-#pragma unroll 2
-            for (int k = warp; k < nsplit; k += 4)
-                add_split(src + static_cast<size_t>(k) * stride4,
-                          expf(__ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup) - lse));
-        } else {
-            for (int kb = 0; kb < nsplit; kb += 32) {
-                const int k = kb + lane;
-                const float w_mine = (k < nsplit) ? expf(__ldcg(lse_k + static_cast<size_t>(k) * kRowsPerGroup) - lse) : 0.f;
-                const int cnt = min(32, nsplit - kb);
-#pragma unroll 4
-                for (int kk = 0; kk < cnt; ++kk)
-                    add_split(src + static_cast<size_t>(kb + kk) * stride4, __shfl_sync(0xffffffffu, w_mine, kk));
+        // Splits k0, k0 + step, ... (up to 4 at a time): all their partials in flight at once.
+        auto add_splits = [&](int k0, int step) {
+            float4 v[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int k = k0 + step * j;
+                if (k < nsplit) {
+                    const float4* s4 = src + static_cast<size_t>(k) * stride4;
+                    v[j][0] = __ldcg(s4);
+                    v[j][1] = __ldcg(s4 + 32);
+                    v[j][2] = __ldcg(s4 + 64);
+                    v[j][3] = __ldcg(s4 + 96);
+                }
             }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int k = k0 + step * j;
+                if (k < nsplit) {
+                    const float w = weight(k);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) fma4(acc[i], v[j][i], w);
+                }
+            }
+        };
+        if (kSplitParallel) {
+#pragma unroll 1
+            for (int kb = warp; kb < nsplit; kb += 16) add_splits(kb, 4);  // this warp's splits warp, warp + 4, ...
+        } else {
+#pragma unroll 1
+            for (int kb = 0; kb < nsplit; kb += 4) add_splits(kb, 1);
         }
     }
     if (kSplitParallel) {
