@@ -66,6 +66,16 @@ def test_parity_few_partitions(oracle_mod, parts):
     print(compare(o, lse, o_ref, lse_ref, p.dtype, f"parts={parts}"))
 
 
+def test_parity_more_partitions_than_sm_pairs(oracle_mod):
+    # A caller's partition count above the SM pairs (clusters run in two waves) and one
+    # sequence split more than 96 ways: the combine reads its splits' LSEs past its registers.
+    p = W.make_problem([80000, 3000], s_q=1, h_q=128, seed=140)
+    o, lse, md, ns = run_gpu(p, num_parts=110)
+    assert int(ns[1].item() - ns[0].item()) > 96, "the long sequence must be split more than 96 ways"
+    o_ref, lse_ref = oracle_full(oracle_mod, p)
+    print(compare(o, lse, o_ref, lse_ref, p.dtype, "110 partitions"))
+
+
 @pytest.mark.parametrize("parts", [1, 2])
 def test_parity_leading_empty_chunks(oracle_mod, parts):
     # A partition whose first chunks are empty sequences: the first non-empty
