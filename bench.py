@@ -202,14 +202,15 @@ class ClockSampler:
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
                     "note": self.err or "no samples"}
-        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        # Every sample is taken inside the timed region, which keeps the GPU busy (NVML's
+        # utilization counter averages over a longer window, so it is not used to filter).
         reasons = set()
-        for _, r, _ in loaded:
+        for _, r, _ in self.samples:
             for bit, name in NVML_REASONS.items():
                 if r & bit:
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(s[0] for s in loaded), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(reasons), "samples": len(loaded)}
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
 
 
 # ----------------------------------------------------------------------------- GPU arm
