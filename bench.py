@@ -170,20 +170,26 @@ class ClockSampler:
             self.nv = None
             self.err = str(e)
 
-    def _run(self):
+    def sample(self) -> bool:
+        """One reading of the SM clock and the clock-event reasons (False once NVML fails)."""
         nv, h = self.nv, self.h
-        while not self._stop.is_set():
+        if nv is None:
+            return False
+        try:
+            mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
             try:
-                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                try:
-                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                except Exception:
-                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
-                util = nv.nvmlDeviceGetUtilizationRates(h).gpu
-                self.samples.append((mhz, int(reasons), util))
-            except Exception as e:
-                self.err = str(e)
-                return
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+            self.samples.append((mhz, int(reasons), None))
+            return True
+        except Exception as e:
+            self.err = str(e)
+            self.nv = None
+            return False
+
+    def _run(self):
+        while not self._stop.is_set() and self.sample():
             time.sleep(self.period)
 
     def __enter__(self):
@@ -389,6 +395,8 @@ def time_steps(torch, runner, flush, steps, warmup, barrier, sampler=None, stage
         for _ in range(steps):
             flush.zero_()  # L2 flush between steps, outside the events
             runner.step()
+            if sampler is not None:
+                sampler.sample()  # while the step runs (the launch is asynchronous)
             torch.cuda.synchronize()
             t.append(runner.times_ms())
     barrier()
