@@ -339,14 +339,14 @@ __device__ __forceinline__ int request_len(const int32_t* seqlens, int const_len
 
 // Iterates the chunks (vb, blk_lo, blk_hi) of one scheduler partition.
 struct ChunkIter {
-    int vb, blk, end_vb, end_blk, groups;
+    int vb, blk, end_vb, end_blk, batch;
     const int32_t* seqlens;
     int const_len;  // the length of every request when seqlens is null
 
     __device__ bool next(int& out_vb, int& lo, int& hi)
     {
         if (!(vb < end_vb || (vb == end_vb && blk < end_blk))) return false;
-        const int n = pages_of(request_len(seqlens, const_len, vb / groups));
+        const int n = pages_of(request_len(seqlens, const_len, vb_request(vb, batch)));
         out_vb = vb;
         lo = blk;
         hi = (vb == end_vb) ? end_blk : n;
@@ -504,7 +504,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
 
     Sync sync{s_bar + kOffAbort, map_to_cta(s_bar + kOffAbort, cta ^ 1u), p.status};
     const int32_t* md = p.md + part * kMdInts;
-    ChunkIter chunks{md[0], md[1], md[2], md[3], p.groups, p.seqlens, p.topk};
+    ChunkIter chunks{md[0], md[1], md[2], md[3], p.batch, p.seqlens, p.topk};
     const int begin_vb = md[0];
     const int begin_split = md[4];
 
@@ -552,7 +552,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         int vb, lo, hi;
         while (ok && chunks.next(vb, lo, hi)) {
             if (hi <= lo) continue;
-            const int Lb = request_len(p.seqlens, p.topk, vb / p.groups);
+            const int Lb = request_len(p.seqlens, p.topk, vb_request(vb, p.batch));
             for (int blk = lo; blk < hi && ok; ++blk, rk.advance(), kring.advance()) {
                 if (!(ok = wwait(bar(kBarRawKFull + rk.stage), rk.phase))) break;
                 if (tl_conv) TL_EV(kEvConvRaw);
@@ -634,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 bool ok = true;
                 while (ok && chunks.next(vb, lo, hi)) {
                     if (hi <= lo) continue;
-                    const int b = vb / p.groups, rg = vb % p.groups;
+                    const int b = vb_request(vb, p.batch), rg = vb_group(vb, p.batch);
                     const int y = rg * kRowsPerGroup + y_off;
                     if (!(ok = sync.wait(bar(kBarQFree), (k & 1) ^ 1))) break;
                     TL_EV(kEvQLoad);
@@ -671,7 +671,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
                 while (ok && chunks.next(vb, lo, hi)) {
                     if (hi <= lo) continue;
-                    const int32_t* ent = p.indices + static_cast<size_t>(vb / p.groups) * p.topk;
+                    const int32_t* ent = p.indices + static_cast<size_t>(vb_request(vb, p.batch)) * p.topk;
                     auto entry = [&](int blk) {
                         const int e = kPage * blk + 32 * static_cast<int>(cta) + lane;
                         return e < p.topk ? __ldg(ent + e) : -1;
@@ -709,7 +709,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                     const uint8_t* kv = static_cast<const uint8_t*>(p.kvcache);
                     while (ok && chunks.next(vb, lo, hi)) {
                         if (hi <= lo) continue;
-                        const int b = vb / p.groups;
+                        const int b = vb_request(vb, p.batch);
                         const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
                         int entry = table_entry(p, table, lo), entry_next = 0;
                         for (int blk = lo; blk < hi; ++blk, ring.advance(), entry = entry_next) {
@@ -741,7 +741,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
                 while (ok && chunks.next(vb, lo, hi)) {
                     if (hi <= lo) continue;
-                    const int32_t* ent = p.indices + static_cast<size_t>(vb / p.groups) * p.topk;
+                    const int32_t* ent = p.indices + static_cast<size_t>(vb_request(vb, p.batch)) * p.topk;
                     auto entry = [&](int blk) {
                         const int e = kPage * blk + 32 * static_cast<int>(cta) + lane;
                         const int idx = e < p.topk ? __ldg(ent + e) : -1;
@@ -782,7 +782,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
 #endif
                 while (ok && chunks.next(vb, lo, hi)) {
                     if (hi <= lo) continue;
-                    const int b = vb / p.groups;
+                    const int b = vb_request(vb, p.batch);
                     const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
 #ifdef MLA_TEST_WITHHOLD_K_PAGE
                     const int withheld = (part == 0 && first_chunk) ? lo + MLA_TEST_WITHHOLD_K_PAGE : -1;
@@ -880,7 +880,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
                 while (ok && chunks.next(vb, lo, hi)) {
                     if (hi <= lo) continue;
-                    const int32_t* ent = p.indices + static_cast<size_t>(vb / p.groups) * p.topk;
+                    const int32_t* ent = p.indices + static_cast<size_t>(vb_request(vb, p.batch)) * p.topk;
                     auto entry = [&](int e) {
                         const int idx = e < p.topk ? __ldg(ent + e) : -1;
                         return (idx >= 0 && idx < p.cache_rows) ? idx : p.cache_rows;
@@ -936,7 +936,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
                 auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
                 while (ok && chunks.next(vb, lo, hi)) {
                     if (hi <= lo) continue;
-                    const int b = vb / p.groups;
+                    const int b = vb_request(vb, p.batch);
                     const int Lb = request_len(p.seqlens, p.topk, b);
                     const int tail = Lb % kPage;
                     const int last_page = pages_of(Lb) - 1;
@@ -1125,10 +1125,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         const uint32_t o_free_lead = lead_bar(kBarOFree);
         auto wwait = [&](uint32_t b_, uint32_t par) { return __all_sync(0xffffffffu, sync.wait(b_, par)); };
         auto q_row_ptr = [&](int qvb, bool& valid) {
-            const int qrow_idx = (qvb % p.groups) * kRowsPerGroup + 64 * static_cast<int>(cta) + r;
+            const int qrow_idx = vb_group(qvb, p.batch) * kRowsPerGroup + 64 * static_cast<int>(cta) + r;
             valid = qrow_idx < p.rows;
             return reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
-                                                  (static_cast<size_t>(qvb / p.groups) * p.rows + qrow_idx) * p.d_qk * 2);
+                                                  (static_cast<size_t>(vb_request(qvb, p.batch)) * p.rows + qrow_idx) * p.d_qk * 2);
         };
         // The whole row (the tensor-memory columns this warp stores and the shared-memory
         // ones the Q producer loads), once per row: threads t and t ^ 64 share it.
@@ -1161,7 +1161,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp8 ? kThreadsFp8 :
         if (t == 0) TL_EV(kEvSetupDone);
         bool have = chunks.next(vb, lo, hi);
         while (ok && have) {
-            const int b = vb / p.groups, rg = vb % p.groups;
+            const int b = vb_request(vb, p.batch), rg = vb_group(vb, p.batch);
             const int Lb = request_len(p.seqlens, p.topk, b);
             const int row = rg * kRowsPerGroup + 64 * static_cast<int>(cta) + r;
             const bool row_valid = row < p.rows;
@@ -1490,7 +1490,7 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(DecodeParams p)
     }
     __syncthreads();
     if (!go) return;
-    const int b = vb / p.groups, rg = vb % p.groups;
+    const int b = vb_request(vb, p.batch), rg = vb_group(vb, p.batch);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = kSplitParallel ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y) * 4 + warp;
     const int rows_here = min(kRowsPerGroup, p.rows - rg * kRowsPerGroup);
@@ -1665,7 +1665,7 @@ __global__ void __launch_bounds__(kMetaThreads) mla_metadata_kernel(const int32_
     int32_t* extra = pages + nv;
     int32_t* begins = extra + nv;  // [num_parts][2]
     for (int v = threadIdx.x; v < nv; v += blockDim.x) {
-        pages[v] = pages_of(seqlens ? seqlens[v / groups] : const_len);
+        pages[v] = pages_of(seqlens ? seqlens[vb_request(v, batch)] : const_len);
         C[v] = pages[v] + fixed_cost;
         extra[v] = 0;
     }

@@ -8,8 +8,11 @@
 // variable-length sequence serving", sourcepulse summary).  The pages do not
 // print the algorithm or the metadata format; this one is our own.
 //
-// Work units.  A "virtual batch" vb = b * row_groups + g is request b restricted
-// to query rows [128 g, 128 g + 128) of its s_q * h_q rows.  Every chunk (one
+// Work units.  A "virtual batch" vb = g * batch + b is request b restricted to query
+// rows [128 g, 128 g + 128) of its s_q * h_q rows.  The numbering is group-major: row
+// group 0 of every request comes before row group 1 of any, so on the line below the
+// groups of one request lie half a line (for two groups) apart, and the partitions that
+// cover them stream the same pages at about the same time (the second read hits L2).  Every chunk (one
 // partition's share of one virtual batch) costs F units of overhead (the output
 // epilogue, refilling the pipeline) plus one unit per 64-token page: F = kFixedCost
 // for the paged decode (kFixedCostFp8 over an FP8 cache, whose pages take about twice
@@ -61,6 +64,10 @@ constexpr int kMdInts = 8;
 MLA_HD inline int row_groups(int heads_per_kv) { return (heads_per_kv + kRowsPerGroup - 1) / kRowsPerGroup; }
 
 MLA_HD inline int pages_of(int seqlen) { return seqlen <= 0 ? 0 : (seqlen + kPage - 1) / kPage; }
+
+// Request and row group of virtual batch vb (group-major numbering, batch requests).
+MLA_HD inline int vb_request(int vb, int batch) { return vb % batch; }
+MLA_HD inline int vb_group(int vb, int batch) { return vb / batch; }
 
 // Position on the page line of cost unit x.  C: exclusive prefix of the costs,
 // nv entries; total: W; F: the per-chunk cost.  Returns (vb, blk) through the references.
@@ -121,7 +128,7 @@ inline void schedule_host(const int32_t* seqlens, int batch, int groups, int num
     const int nv = batch * groups;
     long long total = 0;
     for (int v = 0; v < nv; ++v) {
-        pages[v] = pages_of(seqlens[v / groups]);
+        pages[v] = pages_of(seqlens[vb_request(v, batch)]);
         C[v] = total;
         total += pages[v] + F;
     }

@@ -31,7 +31,7 @@ def chunks_of(md, seqlens, groups):
     for p, (bv, bb, ev, eb, bs, *_rest) in enumerate(md):
         vb, blk = bv, bb
         while vb < ev or (vb == ev and blk < eb):
-            n = pages(seqlens[vb // groups])
+            n = pages(seqlens[vb % len(seqlens)])  # group-major: vb = g * batch + b
             hi = eb if vb == ev else n
             out.append((p, vb, blk, hi, bs if vb == bv else 0))
             vb, blk = vb + 1, 0
@@ -58,7 +58,7 @@ def check_schedule(seqlens, heads_per_kv, num_parts, sparse_topk=None, fp8=False
     per_vb = {}
     for p, vb, lo, hi, sidx in ch:
         assert 0 <= vb < nv
-        n = pages(seqlens[vb // groups])
+        n = pages(seqlens[vb % seqlens.size])
         assert 0 <= lo <= hi <= n
         assert hi > lo or n == 0, "non-empty sequences never get empty chunks"
         for blk in range(lo, hi):
@@ -66,7 +66,7 @@ def check_schedule(seqlens, heads_per_kv, num_parts, sparse_topk=None, fp8=False
             covered[(vb, blk)] = p
         per_vb.setdefault(vb, []).append((p, lo, sidx))
     for vb in range(nv):
-        n = pages(seqlens[vb // groups])
+        n = pages(seqlens[vb % seqlens.size])
         for blk in range(n):
             assert (vb, blk) in covered, f"page {blk} of vb {vb} never processed"
         lst = per_vb.get(vb, [])
