@@ -148,3 +148,13 @@ def test_sparse_full_size_sampled(oracle_mod):
     print(compare(o.reshape(rows_total, 512)[idx], lse.reshape(rows_total)[idx], o_r, l_r, p.dtype,
                   "sparse_fp8 sampled"))
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
+@pytest.mark.parametrize("h_q,s_q", [(256, 1), (192, 2)])
+def test_sparse_several_row_groups(oracle_mod, h_q, s_q):
+    # more than 128 heads per token: each token's rows form two row groups (virtual batches
+    # numbered group-major), both reading the token's own entry list
+    p = W.make_sparse_problem([2500, 900, 300], 400, s_q=s_q, h_q=h_q, fp8_kv=True, invalid_frac=0.1, seed=440 + h_q)
+    o, lse, md, ns = _run(p)
+    o_ref, lse_ref = _oracle(oracle_mod, p)
+    print(compare(o, lse, o_ref, lse_ref, p.dtype, f"sparse h_q={h_q} s_q={s_q}"))

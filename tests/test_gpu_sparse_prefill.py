@@ -105,3 +105,22 @@ def test_prefill_full_size_sampled(oracle_mod):
     idx = torch.from_numpy(toks).cuda()
     _check_prefill(p, out[idx], mx[idx], lse[idx], o_ref, mx_ref, lse_ref, "sparse_prefill sampled")
     assert torch.isfinite(out).all() and torch.isfinite(lse).all() and torch.isfinite(mx).all()
+
+
+def test_prefill_several_row_groups(oracle_mod):
+    # 256 heads per token: two row groups per query token over the same list
+    p = W.make_prefill_problem(10, 256, 600, 200, invalid_frac=0.1, seed=530)
+    out, mx, lse = _prefill(p)
+    o_ref, mx_ref, lse_ref = oracle_mod.sparse_prefill(p.q, p.kv, p.indices, p.sm_scale)
+    _check_prefill(p, out, mx, lse, o_ref, mx_ref, lse_ref, "h_q=256")
+
+
+def test_sparse_decode_16bit_several_row_groups(oracle_mod):
+    p = W.make_sparse_problem([1500, 400], 250, s_q=2, h_q=256, invalid_frac=0.2, seed=531)
+    q, kv = _dev(p.q), _dev(p.kvcache)
+    ind, sl = torch.from_numpy(p.indices).cuda(), torch.from_numpy(p.cache_seqlens).cuda()
+    md, ns = mla.get_mla_metadata(sl, p.s_q * p.h_q, 1, h_q=p.h_q, topk=250)
+    o, lse = mla.flash_mla_with_kvcache(q, kv, None, sl, 512, md, ns, softmax_scale=p.scale, indices=ind)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle_mod.decode_sparse(p.q, p.kvcache, p.indices, scale=p.scale)
+    print(compare(o, lse, o_ref, lse_ref, p.dtype, "sparse decode, bf16 cache, h_q=256"))
